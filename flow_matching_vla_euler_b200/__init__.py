@@ -1,0 +1,284 @@
+"""Python binding of the B200 flow-matching action-expert library (libvla_b200.so).
+
+Argument marshalling only: every step of the denoise loop runs in the library's CUDA
+kernels. The functions ``vla_*`` below mirror the C ABI in include/vla.h one to one;
+``Expert`` wraps a handle for torch callers (CUDA tensors in, CUDA tensors out, on
+``torch.cuda.current_stream()``). There is no CPU fallback: if the shared library is
+missing or the device is not a B200, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvla_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vla.h")
+
+VLA_OK, VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_STATE = 0, 1, 2, 3
+VLA_ERR_OOM, VLA_ERR_CUDA, VLA_ERR_TIMEOUT, VLA_ERR_UNSUPPORTED = 4, 5, 6, 7
+VLA_TIME_PI0_MLP, VLA_TIME_ADA_SINCOS, VLA_TIME_ADA_MLP = 0, 1, 2
+VLA_FLAG_NO_PDL = 1
+KERNEL_KINDS = ["gemm_qkv", "attention", "gemm_o", "gemm_gateup", "gemm_down", "norm", "embed",
+                "final_euler", "time_mlp"]
+
+_CFG_INT_FIELDS = ["n_layers", "width", "n_heads", "n_kv_heads", "head_dim", "mlp_dim", "action_dim",
+                   "chunk", "state_dim", "time_kind", "time_dim", "n_static_max", "n_sliding",
+                   "max_batch", "max_steps"]
+
+WEIGHT_FIELDS = [
+    "action_in_w", "action_in_b", "action_out_w", "action_out_b",
+    "state_in_w", "state_in_b",
+    "time_mlp_in_w", "time_mlp_in_b", "time_mlp_out_w", "time_mlp_out_b",
+    "time_cond1_w", "time_cond1_b", "time_cond2_w", "time_cond2_b",
+    "norm1_w", "norm2_w", "final_norm_w",
+    "norm1_mod_w", "norm1_mod_b", "norm2_mod_w", "norm2_mod_b",
+    "final_norm_mod_w", "final_norm_mod_b",
+    "wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down",
+]
+
+
+class vla_config(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_int) for n in _CFG_INT_FIELDS] +
+                [("eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("flags", ctypes.c_uint)])
+
+
+class vla_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+class vla_kernel_times(ctypes.Structure):
+    _fields_ = [("total_ms", ctypes.c_float * 9), ("launches", ctypes.c_int * 9),
+                ("bytes", ctypes.c_double * 9), ("flops", ctypes.c_double * 9)]
+
+
+class VlaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"vla error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+_SIGNATURES = {
+    "vla_expert_create": (_I, [ctypes.POINTER(vla_config), ctypes.POINTER(vla_weights), ctypes.POINTER(_P)]),
+    "vla_expert_destroy": (None, [_P]),
+    "vla_cache_set_prefix": (_I, [_P, _P, _P, _I, _I, _P]),
+    "vla_cache_append_sliding": (_I, [_P, _P, _P, _I, _P]),
+    "vla_denoise": (_I, [_P, _P, _P, _I, _P, _I, _P]),
+    "vla_denoise_host": (_I, [_P, _P, _P, _I, _P, _I, _P]),
+    "vla_cache_export": (_I, [_P, _P, _P, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                              ctypes.POINTER(_I), _P]),
+    "vla_device_status": (_I, [_P, _P]),
+    "vla_profile_kernels": (_I, [_P, _P, _P, _I, _P, _I, ctypes.POINTER(vla_kernel_times), _P]),
+    "vla_gemm_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "vla_last_error": (ctypes.c_char_p, []),
+    "vla_version": (ctypes.c_char_p, []),
+}
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libvla_b200.so (built by ``python -m flow_matching_vla_euler_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m flow_matching_vla_euler_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def header_functions(path: str = HEADER_PATH):
+    """Names of the entry points declared in include/vla.h."""
+    with open(path) as f:
+        text = f.read()
+    return re.findall(r"^VLA_API\s+[\w\s\*]+?\b(vla_\w+)\s*\(", text, flags=re.M)
+
+
+def _check(code: int):
+    if code != VLA_OK:
+        raise VlaError(code, load_library().vla_last_error().decode())
+
+
+# ---- one-to-one wrappers of the C ABI ------------------------------------------------
+
+def vla_expert_create(cfg: vla_config, weights: vla_weights) -> int:
+    h = _P()
+    _check(load_library().vla_expert_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
+    return h.value
+
+
+def vla_expert_destroy(h: int):
+    load_library().vla_expert_destroy(h)
+
+
+def vla_cache_set_prefix(h, K_ptr, V_ptr, n_tokens, batch, stream):
+    _check(load_library().vla_cache_set_prefix(h, K_ptr, V_ptr, n_tokens, batch, stream))
+
+
+def vla_cache_append_sliding(h, K_ptr, V_ptr, batch, stream):
+    _check(load_library().vla_cache_append_sliding(h, K_ptr, V_ptr, batch, stream))
+
+
+def vla_denoise(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream):
+    _check(load_library().vla_denoise(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream))
+
+
+def vla_denoise_host(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream):
+    _check(load_library().vla_denoise_host(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream))
+
+
+def vla_cache_export(h, K_ptr, V_ptr, batch, stream):
+    head, ns, nr = _I(), _I(), _I()
+    _check(load_library().vla_cache_export(h, K_ptr, V_ptr, batch, ctypes.byref(head), ctypes.byref(ns),
+                                           ctypes.byref(nr), stream))
+    return head.value, ns.value, nr.value
+
+
+def vla_device_status(h, stream):
+    _check(load_library().vla_device_status(h, stream))
+
+
+def vla_profile_kernels(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream) -> vla_kernel_times:
+    t = vla_kernel_times()
+    _check(load_library().vla_profile_kernels(h, noise_ptr, state_ptr, steps, out_ptr, batch,
+                                              ctypes.byref(t), stream))
+    return t
+
+
+def vla_gemm_bf16(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, stream):
+    _check(load_library().vla_gemm_bf16(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, stream))
+
+
+def gemm(W, X, split_k: int = 0):
+    """Y = X @ W^T on the tensor-core kernel; W [n, k], X [m, k] CUDA bf16 -> fp32 [m, n]."""
+    import torch
+    Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.float32, device=X.device)
+    vla_gemm_bf16(_dev_ptr(W, 2), _dev_ptr(X, 2), _dev_ptr(Y, 4), int(W.shape[0]), int(W.shape[1]),
+                  int(X.shape[0]), int(split_k), _stream())
+    return Y
+
+
+def vla_last_error() -> str:
+    return load_library().vla_last_error().decode()
+
+
+def vla_version() -> str:
+    return load_library().vla_version().decode()
+
+
+# ---- torch-facing handle -------------------------------------------------------------
+
+def _stream():
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev_ptr(t, dtype_bytes):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("expected a CUDA tensor")
+    if not t.is_contiguous() or t.element_size() != dtype_bytes:
+        raise TypeError(f"expected a contiguous tensor of {dtype_bytes}-byte elements")
+    return t.data_ptr()
+
+
+class Expert:
+    """One library handle. ``cfg`` has the attributes of vla_config's model fields
+    (n_layers, width, n_heads, n_kv_heads, head_dim, mlp_dim, action_dim, chunk,
+    state_dim, time_kind, time_dim, eps, rope_base); ``params`` maps parameter names
+    ("wq", "norm1.mod_w", ...) to uint16 numpy arrays of bf16 bits."""
+
+    def __init__(self, cfg, params: dict, n_static_max: int, n_sliding: int = 0, max_batch: int = 1,
+                 max_steps: int = 10, flags: int = 0):
+        import numpy as np
+        c = vla_config()
+        for n in ["n_layers", "width", "n_heads", "n_kv_heads", "head_dim", "mlp_dim", "action_dim",
+                  "chunk", "state_dim", "time_kind", "time_dim"]:
+            setattr(c, n, int(getattr(cfg, n)))
+        c.n_static_max, c.n_sliding = int(n_static_max), int(n_sliding)
+        c.max_batch, c.max_steps = int(max_batch), int(max_steps)
+        c.eps, c.rope_base, c.flags = float(cfg.eps), float(cfg.rope_base), int(flags)
+        w = vla_weights()
+        keep = []
+        for name, arr in params.items():
+            field = name.replace(".", "_")
+            if field not in WEIGHT_FIELDS:
+                raise KeyError(f"unknown parameter {name}")
+            a = np.ascontiguousarray(arr, dtype=np.uint16)
+            keep.append(a)
+            setattr(w, field, a.ctypes.data)
+        self.cfg = cfg
+        self.n_static_max, self.n_sliding, self.max_batch = n_static_max, n_sliding, max_batch
+        self.handle = vla_expert_create(c, w)
+        del keep
+
+    def close(self):
+        if getattr(self, "handle", None):
+            vla_expert_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_prefix(self, K, V):
+        """K, V: CUDA tensors (2-byte elements, bf16 bits) [L, batch, n_tokens, D]."""
+        batch, n = int(K.shape[1]), int(K.shape[2])
+        vla_cache_set_prefix(self.handle, _dev_ptr(K, 2), _dev_ptr(V, 2), n, batch, _stream())
+
+    def append_sliding(self, K_tok, V_tok):
+        """K_tok, V_tok: CUDA tensors [L, batch, D] of bf16 bits."""
+        vla_cache_append_sliding(self.handle, _dev_ptr(K_tok, 2), _dev_ptr(V_tok, 2),
+                                 int(K_tok.shape[1]), _stream())
+
+    def denoise(self, noise, state=None, steps: int = 10, out=None):
+        """noise: CUDA fp32 [batch, C, A]; state: CUDA fp32 [batch, state_dim] or None."""
+        import torch
+        out = torch.empty_like(noise) if out is None else out
+        sp = _dev_ptr(state, 4) if state is not None else None
+        vla_denoise(self.handle, _dev_ptr(noise, 4), sp, int(steps), _dev_ptr(out, 4),
+                    int(noise.shape[0]), _stream())
+        return out
+
+    def denoise_host(self, noise, state=None, steps: int = 10):
+        """Host (numpy fp32) buffers in and out; synchronous."""
+        import numpy as np
+        noise = np.ascontiguousarray(noise, dtype=np.float32)
+        out = np.empty_like(noise)
+        st = None if state is None else np.ascontiguousarray(state, dtype=np.float32)
+        vla_denoise_host(self.handle, noise.ctypes.data, None if st is None else st.ctypes.data,
+                         int(steps), out.ctypes.data, int(noise.shape[0]), _stream())
+        return out
+
+    def cache_export(self, batch: int):
+        import torch
+        L, D = int(self.cfg.n_layers), int(self.cfg.head_dim)
+        shape = (L, batch, self.n_static_max + self.n_sliding, D)
+        K = torch.empty(shape, dtype=torch.int16, device="cuda")
+        V = torch.empty(shape, dtype=torch.int16, device="cuda")
+        head, ns, nr = vla_cache_export(self.handle, K.data_ptr(), V.data_ptr(), batch, _stream())
+        return K, V, head, ns, nr
+
+    def device_status(self):
+        vla_device_status(self.handle, _stream())
+
+    def profile_kernels(self, noise, state=None, steps: int = 10):
+        import torch
+        out = torch.empty_like(noise)
+        sp = _dev_ptr(state, 4) if state is not None else None
+        t = vla_profile_kernels(self.handle, _dev_ptr(noise, 4), sp, int(steps), _dev_ptr(out, 4),
+                                int(noise.shape[0]), _stream())
+        res = {k: {"ms": t.total_ms[i], "launches": t.launches[i], "bytes": t.bytes[i],
+                   "flops": t.flops[i]} for i, k in enumerate(KERNEL_KINDS)}
+        return out, res

@@ -1,0 +1,1030 @@
+// api.cu -- host runtime behind include/vla.h.
+//
+// Owns every device buffer (allocated once in vla_expert_create: FlowEdge README,
+// "warmup (malloc 0)" and its pre-sized arena), repacks the weights for the kernels,
+// builds the TMA descriptors, plans the launches, keeps the per-step time tables and
+// captures the whole denoise loop as one CUDA graph per (batch, steps) (InstinctFlash
+// README, GRAPH layer: CUDA-graph capture and memory planning).
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/vla.h"
+#include "kernels.h"
+
+using namespace vla;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CU(expr)                                                                          \
+  do {                                                                                    \
+    cudaError_t e_ = (expr);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail(e_ == cudaErrorMemoryAllocation ? VLA_ERR_OOM : VLA_ERR_CUDA, "%s: %s (%s:%d)", \
+                  #expr, cudaGetErrorString(e_), __FILE__, __LINE__);                     \
+  } while (0)
+
+constexpr int kTableSlots = 4;
+constexpr int kMaxSteps = 64;
+
+inline int cdiv(long a, long b) { return static_cast<int>((a + b - 1) / b); }
+
+float bf16_to_f32(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+struct GemmPlan {
+  int tn, n_tiles, m_tiles, splits, kb_per_split;
+};
+
+// Token tile, split-K factor: enough CTAs to keep >= 148 SMs streaming weights, each
+// split covering >= 2 K blocks (128 K) so partial tiles stay small next to the weights.
+GemmPlan plan_gemm(int n_feat, int k_dim, int m_tok, int sm_count) {
+  GemmPlan g;
+  g.tn = m_tok <= 64 ? 64 : (m_tok <= 512 ? 128 : 256);
+  g.n_tiles = n_feat / 128;
+  g.m_tiles = cdiv(m_tok, g.tn);
+  const int nkb = k_dim / 64;
+  const int resident = g.tn == 64 ? 2 : 1;   // CTAs per SM that fit in shared memory
+  const int target = sm_count * resident;
+  const int base = g.n_tiles * g.m_tiles;
+  int splits = 1;
+  if (base < target) splits = std::min(cdiv(target, base), std::max(1, nkb / 2));
+  g.kb_per_split = cdiv(nkb, splits);
+  g.splits = cdiv(nkb, g.kb_per_split);
+  return g;
+}
+
+struct AttnPlan {
+  int q_tiles, splits;
+};
+
+AttnPlan plan_attn(int rows, int batch, int max_key_tiles, int sm_count) {
+  AttnPlan a;
+  a.q_tiles = cdiv(rows, attn_q_tile());
+  const int base = a.q_tiles * batch;
+  int splits = 1;
+  if (base < sm_count) splits = std::min(cdiv(sm_count, base), std::max(1, max_key_tiles / 2));
+  a.splits = std::max(1, splits);
+  return a;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows][inner] row-major, boxes of 64 (inner) x box_rows, 128-byte swizzle.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llu x %llu, box rows %u",
+                static_cast<int>(r), static_cast<unsigned long long>(rows),
+                static_cast<unsigned long long>(inner), box_rows);
+  return VLA_OK;
+}
+
+}  // namespace
+
+struct vla_expert {
+  vla_config cfg;
+  int dev = 0, sm_count = 148;
+  int L, W, H, D, F, A, C, Sd, S, hs, HD, Td, Cd, qkv_rows, kcap, ring_off, dyn_off, max_M;
+  bool ada, pi0;
+
+  std::vector<void*> allocs;
+
+  // weights
+  bf16 *wqkv = nullptr, *wo = nullptr, *wgu = nullptr, *wdown = nullptr;
+  bf16 *w1a = nullptr, *w2 = nullptr, *tin_full = nullptr, *tin_b = nullptr;
+  bf16 *cond1_w = nullptr, *cond1_b = nullptr, *cond2_w = nullptr, *cond2_b = nullptr;
+  bf16 *mod_w = nullptr, *mod_b = nullptr;
+  float *ain_w = nullptr, *ain_b = nullptr, *aout_w = nullptr, *aout_b = nullptr;
+  float *st_w = nullptr, *st_b = nullptr, *t2_b = nullptr;
+  float *n1_w = nullptr, *n2_w = nullptr, *nf_w = nullptr;
+
+  // time tables
+  float* tables[kTableSlots] = {};
+  int table_steps[kTableSlots] = {};
+  int table_age[kTableSlots] = {};
+  int table_clock = 0;
+  long table_stride = 0;   // floats per step
+  float *temb = nullptr, *tscr1 = nullptr, *tscr2 = nullptr;
+
+  // activations and cache
+  float *x = nullptr, *state = nullptr, *resid = nullptr, *rope = nullptr;
+  bf16 *hb = nullptr, *qb = nullptr, *ob = nullptr, *ub = nullptr, *eb = nullptr, *h1b = nullptr;
+  bf16 *kc = nullptr, *vc = nullptr;
+  CacheDesc* desc = nullptr;
+  float *ws = nullptr, *part_o = nullptr, *part_ml = nullptr;
+  int *ctr = nullptr, *attn_ctr = nullptr, *err = nullptr;
+  size_t ws_floats = 0, part_floats = 0, ctr_ints = 0, attn_ctr_ints = 0;
+  float *hx = nullptr, *hstate = nullptr;   // staging for vla_denoise_host (device)
+
+  // host mirror of the cache state
+  bool prefix_loaded = false;
+  int prefix_batch = 0, n_static = 0, n_ring = 0, head = 0;
+
+  CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
+
+  struct GraphEntry {
+    cudaGraph_t g = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    int slot = -1;
+  };
+  std::map<std::pair<int, int>, GraphEntry> graphs;
+  cudaStream_t cap = nullptr;
+};
+
+namespace {
+
+template <typename T>
+int dalloc(vla_expert* h, T** p, size_t count) {
+  void* q = nullptr;
+  cudaError_t e = cudaMalloc(&q, std::max<size_t>(count, 1) * sizeof(T));
+  if (e != cudaSuccess)
+    return fail(e == cudaErrorMemoryAllocation ? VLA_ERR_OOM : VLA_ERR_CUDA,
+                "cudaMalloc(%zu bytes): %s", count * sizeof(T), cudaGetErrorString(e));
+  h->allocs.push_back(q);
+  cudaMemset(q, 0, std::max<size_t>(count, 1) * sizeof(T));
+  *p = static_cast<T*>(q);
+  return VLA_OK;
+}
+
+int upload_bf16(vla_expert* h, bf16** dst, const uint16_t* src, size_t n) {
+  int rc = dalloc(h, dst, n);
+  if (rc) return rc;
+  CU(cudaMemcpy(*dst, src, n * 2, cudaMemcpyHostToDevice));
+  return VLA_OK;
+}
+
+int upload_f32(vla_expert* h, float** dst, const uint16_t* src, size_t n) {
+  std::vector<float> tmp(n);
+  for (size_t i = 0; i < n; ++i) tmp[i] = bf16_to_f32(src[i]);
+  int rc = dalloc(h, dst, n);
+  if (rc) return rc;
+  CU(cudaMemcpy(*dst, tmp.data(), n * 4, cudaMemcpyHostToDevice));
+  return VLA_OK;
+}
+
+int validate(const vla_config* c, const vla_weights* w) {
+  if (!c || !w) return fail(VLA_ERR_ARG, "null config or weights");
+  if (c->n_layers < 1 || c->width < 128 || c->width % 128)
+    return fail(VLA_ERR_SHAPE, "width must be a positive multiple of 128 (got %d)", c->width);
+  if (c->n_kv_heads != 1) return fail(VLA_ERR_UNSUPPORTED, "only one K/V head is supported");
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
+    return fail(VLA_ERR_SHAPE, "head_dim must be 32, 64, 128 or 256 (got %d)", c->head_dim);
+  if (c->n_heads < 1 || (c->n_heads * c->head_dim) % 64)
+    return fail(VLA_ERR_SHAPE, "n_heads * head_dim must be a multiple of 64");
+  if (c->mlp_dim < 64 || c->mlp_dim % 64) return fail(VLA_ERR_SHAPE, "mlp_dim must be a multiple of 64");
+  if (c->action_dim < 1 || c->action_dim > 64) return fail(VLA_ERR_SHAPE, "action_dim must be in [1, 64]");
+  if (c->chunk < 1) return fail(VLA_ERR_SHAPE, "chunk must be >= 1");
+  if (c->state_dim < 0 || c->state_dim > 256) return fail(VLA_ERR_SHAPE, "state_dim must be in [0, 256]");
+  if (c->time_kind < 0 || c->time_kind > 2) return fail(VLA_ERR_ARG, "bad time_kind %d", c->time_kind);
+  if (c->time_dim < 4 || c->time_dim % 2) return fail(VLA_ERR_SHAPE, "time_dim must be even and >= 4");
+  if (c->time_kind == VLA_TIME_ADA_SINCOS && c->time_dim % 64)
+    return fail(VLA_ERR_SHAPE, "ADA_SINCOS conditioning needs time_dim % 64 == 0");
+  if (c->time_kind == VLA_TIME_PI0_MLP && c->time_dim % 64)
+    return fail(VLA_ERR_SHAPE, "PI0_MLP needs time_dim % 64 == 0");
+  if (c->n_static_max < 0 || c->n_sliding < 0 || c->n_static_max + c->n_sliding < 1)
+    return fail(VLA_ERR_SHAPE, "need n_static_max + n_sliding >= 1");
+  if (c->max_batch < 1) return fail(VLA_ERR_SHAPE, "max_batch must be >= 1");
+  if (c->max_steps < 1 || c->max_steps > kMaxSteps)
+    return fail(VLA_ERR_SHAPE, "max_steps must be in [1, %d]", kMaxSteps);
+  if (!(c->eps > 0.0f)) return fail(VLA_ERR_ARG, "eps must be > 0");
+  const bool need_common = w->action_in_w && w->action_in_b && w->action_out_w && w->action_out_b &&
+                           w->wq && w->wk && w->wv && w->wo && w->w_gate && w->w_up && w->w_down;
+  if (!need_common) return fail(VLA_ERR_ARG, "missing a projection weight");
+  if (c->state_dim > 0 && !(w->state_in_w && w->state_in_b)) return fail(VLA_ERR_ARG, "missing state_in weights");
+  if (c->time_kind == VLA_TIME_PI0_MLP &&
+      !(w->time_mlp_in_w && w->time_mlp_in_b && w->time_mlp_out_w && w->time_mlp_out_b && w->norm1_w &&
+        w->norm2_w && w->final_norm_w))
+    return fail(VLA_ERR_ARG, "missing Pi0 time-MLP or norm weights");
+  if (c->time_kind != VLA_TIME_PI0_MLP &&
+      !(w->norm1_mod_w && w->norm1_mod_b && w->norm2_mod_w && w->norm2_mod_b && w->final_norm_mod_w &&
+        w->final_norm_mod_b))
+    return fail(VLA_ERR_ARG, "missing AdaRMSNorm modulation weights");
+  if (c->time_kind == VLA_TIME_ADA_MLP &&
+      !(w->time_cond1_w && w->time_cond1_b && w->time_cond2_w && w->time_cond2_b))
+    return fail(VLA_ERR_ARG, "missing time-conditioning MLP weights");
+  return VLA_OK;
+}
+
+int compute_tables(vla_expert* h, int slot, int steps, cudaStream_t s) {
+  float* tbl = h->tables[slot];
+  CU(launch_temb(h->temb, steps, h->Td, s));
+  if (h->pi0) {
+    // tau_k = time half of the first action-time MLP layer applied to temb_k, + bias
+    CU(launch_rowgemv(h->temb, steps, h->Td, h->tin_full + h->W, h->W + h->Td, h->tin_b, h->W, tbl, 0, s));
+  } else {
+    const float* cond = h->temb;
+    if (h->cfg.time_kind == VLA_TIME_ADA_MLP) {
+      CU(launch_rowgemv(h->temb, steps, h->Td, h->cond1_w, h->Td, h->cond1_b, h->W, h->tscr1, 1, s));
+      CU(launch_rowgemv(h->tscr1, steps, h->W, h->cond2_w, h->W, h->cond2_b, h->W, h->tscr2, 1, s));
+      cond = h->tscr2;
+    }
+    CU(launch_rowgemv(cond, steps, h->Cd, h->mod_w, h->Cd, h->mod_b, (2 * h->L + 1) * 3 * h->W, tbl, 0, s));
+  }
+  h->table_steps[slot] = steps;
+  return VLA_OK;
+}
+
+// Slot holding the tables for `steps`, computing them (into the least recently used
+// slot) if needed. Graphs that used an evicted slot are dropped.
+int ensure_tables(vla_expert* h, int steps, cudaStream_t s, int* slot_out) {
+  for (int i = 0; i < kTableSlots; ++i)
+    if (h->table_steps[i] == steps) {
+      h->table_age[i] = ++h->table_clock;
+      *slot_out = i;
+      return VLA_OK;
+    }
+  int victim = 0;
+  for (int i = 1; i < kTableSlots; ++i)
+    if (h->table_age[i] < h->table_age[victim]) victim = i;
+  for (auto it = h->graphs.begin(); it != h->graphs.end();) {
+    if (it->second.slot == victim) {
+      cudaGraphExecDestroy(it->second.exec);
+      cudaGraphDestroy(it->second.g);
+      it = h->graphs.erase(it);
+    } else {
+      ++it;
+    }
+  }
+  int rc = compute_tables(h, victim, steps, s);
+  if (rc) return rc;
+  h->table_age[victim] = ++h->table_clock;
+  *slot_out = victim;
+  return VLA_OK;
+}
+
+struct ActMaps {
+  CUtensorMap hb, ob, ub, eb, h1b;
+};
+
+struct Recorder {
+  // optional per-launch timing (vla_profile_kernels)
+  std::vector<cudaEvent_t>* events = nullptr;
+  std::vector<int>* kinds = nullptr;
+  cudaStream_t s;
+  int begin(int) {
+    if (events) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return fail(VLA_ERR_CUDA, "cudaEventCreate");
+      cudaEventRecord(e, s);
+      events->push_back(e);
+    }
+    return VLA_OK;
+  }
+  int end(int kind) {
+    if (events) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return fail(VLA_ERR_CUDA, "cudaEventCreate");
+      cudaEventRecord(e, s);
+      events->push_back(e);
+      kinds->push_back(kind);
+    }
+    return VLA_OK;
+  }
+};
+
+int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensorMap& tw,
+                 const CUtensorMap& tx, GemmParams p, int n_feat, int k_dim, int M, bool pdl) {
+  const GemmPlan g = plan_gemm(n_feat, k_dim, M, h->sm_count);
+  p.n_feat = n_feat;
+  p.k_dim = k_dim;
+  p.m_tok = M;
+  p.splits = g.splits;
+  p.kb_per_split = g.kb_per_split;
+  p.ws = h->ws;
+  p.counters = h->ctr;
+  p.err = h->err;
+  rec.begin(kind);
+  CU(launch_gemm(g.tn, epi, tw, tx, p, g.n_tiles, g.m_tiles, rec.s, pdl));
+  return rec.end(kind);
+}
+
+// Enqueue one full denoise (all steps) for `batch` observations on rec.s.
+int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am, Recorder& rec) {
+  const bool pdl = !(h->cfg.flags & VLA_FLAG_NO_PDL) && rec.events == nullptr;
+  const int M = B * h->S, W = h->W, L = h->L;
+  const float* tbl = h->tables[slot];
+  const int key_tiles_max = cdiv(h->cfg.n_static_max, attn_key_tile(h->D)) +
+                            cdiv(h->cfg.n_sliding, attn_key_tile(h->D)) + cdiv(h->S, attn_key_tile(h->D));
+  const AttnPlan ap = plan_attn(h->S * h->H, B, key_tiles_max, h->sm_count);
+  const float dt = -1.0f / static_cast<float>(steps);
+  for (int k = 0; k < steps; ++k) {
+    const float* tk = tbl + static_cast<long>(k) * h->table_stride;
+    EmbedParams e{};
+    e.x = h->x;
+    e.state = h->state;
+    e.w_in = h->ain_w;
+    e.b_in = h->ain_b;
+    e.w_st = h->st_w;
+    e.b_st = h->st_b;
+    e.resid = h->resid;
+    e.e_out = h->pi0 ? h->eb : nullptr;
+    e.B = B;
+    e.C = h->C;
+    e.A = h->A;
+    e.S = h->S;
+    e.Sd = h->Sd;
+    e.W = W;
+    e.has_state = h->hs;
+    rec.begin(VLA_K_EMBED);
+    CU(launch_embed(e, rec.s, pdl));
+    rec.end(VLA_K_EMBED);
+    if (h->pi0) {
+      GemmParams p{};
+      p.vec = tk;   // tau_k
+      p.out = h->h1b;
+      p.ld_out = W;
+      int rc = enqueue_gemm(h, rec, VLA_K_TIME_MLP, EPI_SWISH_VEC, h->tm_w1a, am.eb, p, W, W, M, pdl);
+      if (rc) return rc;
+      GemmParams q{};
+      q.vec = h->t2_b;
+      q.resid = h->resid;
+      q.ld_resid = W;
+      q.has_state = h->hs;
+      q.seq = h->S;
+      rc = enqueue_gemm(h, rec, VLA_K_TIME_MLP, EPI_BIAS_STORE, h->tm_w2, am.h1b, q, W, W, M, pdl);
+      if (rc) return rc;
+    }
+    for (int l = 0; l < L; ++l) {
+      for (int half = 0; half < 2; ++half) {
+        const int j = 2 * l + half;
+        NormParams n{};
+        n.x = h->resid;
+        n.y = h->hb;
+        if (h->ada) {
+          n.scale = tk + (static_cast<long>(j) * 3 + 0) * W;
+          n.shift = tk + (static_cast<long>(j) * 3 + 1) * W;
+        } else {
+          n.w = (half == 0 ? h->n1_w : h->n2_w) + static_cast<long>(l) * W;
+        }
+        n.M = M;
+        n.W = W;
+        n.eps = h->cfg.eps;
+        rec.begin(VLA_K_NORM);
+        CU(launch_norm(n, rec.s, pdl));
+        rec.end(VLA_K_NORM);
+        const float* gate = h->ada ? tk + (static_cast<long>(j) * 3 + 2) * W : nullptr;
+        if (half == 0) {
+          GemmParams p{};
+          p.w_row0 = l * h->qkv_rows;
+          p.out = h->qb;
+          p.ld_out = h->HD;
+          p.kc = h->kc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
+          p.vc = h->vc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
+          p.kcap = h->kcap;
+          p.dyn_off = h->dyn_off;
+          p.seq = h->S;
+          p.n_heads = h->H;
+          p.head_dim = h->D;
+          p.rope = h->rope;
+          int rc = enqueue_gemm(h, rec, VLA_K_GEMM_QKV, EPI_QKV, h->tm_wqkv, am.hb, p, h->qkv_rows, W, M, pdl);
+          if (rc) return rc;
+          AttnParams a{};
+          a.q = h->qb;
+          a.kc = p.kc;
+          a.vc = p.vc;
+          a.out = h->ob;
+          a.cache = h->desc;
+          a.seq = h->S;
+          a.n_heads = h->H;
+          a.kcap = h->kcap;
+          a.ring_off = h->ring_off;
+          a.dyn_off = h->dyn_off;
+          a.has_state = h->hs;
+          a.n_splits = ap.splits;
+          a.part_o = h->part_o;
+          a.part_ml = h->part_ml;
+          a.counters = h->attn_ctr;
+          a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h->D));
+          a.err = h->err;
+          rec.begin(VLA_K_ATTN);
+          CU(launch_attention(h->D, a, B, ap.q_tiles, rec.s, pdl));
+          rec.end(VLA_K_ATTN);
+          GemmParams o{};
+          o.w_row0 = l * W;
+          o.resid = h->resid;
+          o.ld_resid = W;
+          o.vec = gate;
+          rc = enqueue_gemm(h, rec, VLA_K_GEMM_O, EPI_RESID, h->tm_wo, am.ob, o, W, h->HD, M, pdl);
+          if (rc) return rc;
+        } else {
+          GemmParams p{};
+          p.w_row0 = l * 2 * h->F;
+          p.out = h->ub;
+          p.ld_out = h->F;
+          int rc = enqueue_gemm(h, rec, VLA_K_GEMM_GATEUP, EPI_GEGLU, h->tm_wgu, am.hb, p, 2 * h->F, W, M, pdl);
+          if (rc) return rc;
+          GemmParams d{};
+          d.w_row0 = l * W;
+          d.resid = h->resid;
+          d.ld_resid = W;
+          d.vec = gate;
+          rc = enqueue_gemm(h, rec, VLA_K_GEMM_DOWN, EPI_RESID, h->tm_wdown, am.ub, d, W, h->F, M, pdl);
+          if (rc) return rc;
+        }
+      }
+    }
+    FinalParams f{};
+    f.resid = h->resid;
+    f.x = h->x;
+    if (h->ada) {
+      f.scale = tk + (static_cast<long>(2 * L) * 3 + 0) * W;
+      f.shift = tk + (static_cast<long>(2 * L) * 3 + 1) * W;
+    } else {
+      f.w = h->nf_w;
+    }
+    f.w_out = h->aout_w;
+    f.b_out = h->aout_b;
+    f.B = B;
+    f.C = h->C;
+    f.A = h->A;
+    f.S = h->S;
+    f.W = W;
+    f.has_state = h->hs;
+    f.eps = h->cfg.eps;
+    f.dt = dt;
+    rec.begin(VLA_K_FINAL);
+    CU(launch_final(f, rec.s, pdl));
+    rec.end(VLA_K_FINAL);
+  }
+  return VLA_OK;
+}
+
+int make_act_maps(vla_expert* h, int B, ActMaps* am) {
+  const int M = B * h->S;
+  const uint32_t tn = static_cast<uint32_t>(plan_gemm(128, 128, M, h->sm_count).tn);
+  int rc;
+  if ((rc = make_tmap(&am->hb, h->hb, h->W, M, tn))) return rc;
+  if ((rc = make_tmap(&am->ob, h->ob, h->HD, M, tn))) return rc;
+  if ((rc = make_tmap(&am->ub, h->ub, h->F, M, tn))) return rc;
+  if (h->pi0) {
+    if ((rc = make_tmap(&am->eb, h->eb, h->W, M, tn))) return rc;
+    if ((rc = make_tmap(&am->h1b, h->h1b, h->W, M, tn))) return rc;
+  } else {
+    am->eb = am->hb;
+    am->h1b = am->hb;
+  }
+  return VLA_OK;
+}
+
+int get_graph(vla_expert* h, int B, int steps, int slot, cudaGraphExec_t* out) {
+  auto key = std::make_pair(B, steps);
+  auto it = h->graphs.find(key);
+  if (it != h->graphs.end() && it->second.slot == slot) {
+    *out = it->second.exec;
+    return VLA_OK;
+  }
+  if (it != h->graphs.end()) {
+    cudaGraphExecDestroy(it->second.exec);
+    cudaGraphDestroy(it->second.g);
+    h->graphs.erase(it);
+  }
+  ActMaps am;
+  int rc = make_act_maps(h, B, &am);
+  if (rc) return rc;
+  CU(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+  Recorder rec;
+  rec.s = h->cap;
+  rc = enqueue_denoise(h, B, steps, slot, am, rec);
+  cudaGraph_t g = nullptr;
+  cudaError_t e = cudaStreamEndCapture(h->cap, &g);
+  if (rc) {
+    if (g) cudaGraphDestroy(g);
+    return rc;
+  }
+  if (e != cudaSuccess) return fail(VLA_ERR_CUDA, "graph capture: %s", cudaGetErrorString(e));
+  cudaGraphExec_t ex = nullptr;
+  e = cudaGraphInstantiate(&ex, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return fail(VLA_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+  }
+  vla_expert::GraphEntry ge;
+  ge.g = g;
+  ge.exec = ex;
+  ge.slot = slot;
+  h->graphs[key] = ge;
+  *out = ex;
+  return VLA_OK;
+}
+
+int check_denoise_args(vla_expert* h, const float* noise, const float* state, int steps, float* out,
+                       int batch) {
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (!noise || !out) return fail(VLA_ERR_ARG, "null noise or out_actions");
+  if (h->Sd > 0 && !state) return fail(VLA_ERR_ARG, "state is required (state_dim = %d)", h->Sd);
+  if (batch < 1 || batch > h->cfg.max_batch)
+    return fail(VLA_ERR_SHAPE, "batch %d outside [1, %d]", batch, h->cfg.max_batch);
+  if (steps < 1 || steps > h->cfg.max_steps)
+    return fail(VLA_ERR_SHAPE, "steps %d outside [1, %d]", steps, h->cfg.max_steps);
+  if (!h->prefix_loaded) return fail(VLA_ERR_STATE, "no prefix K/V set (call vla_cache_set_prefix first)");
+  if (h->prefix_batch < batch)
+    return fail(VLA_ERR_STATE, "prefix was set for %d observations, denoise asked for %d", h->prefix_batch, batch);
+  return VLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vla_last_error(void) { return g_err.c_str(); }
+
+const char* vla_version(void) { return "vla-b200 0.1 (sm_100a)"; }
+
+int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** out) {
+  g_err.clear();
+  if (!out) return fail(VLA_ERR_ARG, "null out");
+  *out = nullptr;
+  int rc = validate(cfg, w);
+  if (rc) return rc;
+  int dev = 0;
+  CU(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  CU(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(VLA_ERR_UNSUPPORTED, "device %s is sm_%d%d; this library is built for sm_100a", prop.name,
+                prop.major, prop.minor);
+
+  CU(configure_gemm_kernels());
+  CU(configure_attention_kernels());
+  vla_expert* h = new vla_expert();
+  h->cfg = *cfg;
+  h->dev = dev;
+  h->sm_count = prop.multiProcessorCount;
+  h->L = cfg->n_layers;
+  h->W = cfg->width;
+  h->H = cfg->n_heads;
+  h->D = cfg->head_dim;
+  h->F = cfg->mlp_dim;
+  h->A = cfg->action_dim;
+  h->C = cfg->chunk;
+  h->Sd = cfg->state_dim;
+  h->hs = cfg->state_dim > 0 ? 1 : 0;
+  h->S = h->C + h->hs;
+  h->HD = h->H * h->D;
+  h->Td = cfg->time_dim;
+  h->ada = cfg->time_kind != VLA_TIME_PI0_MLP;
+  h->pi0 = !h->ada;
+  h->Cd = cfg->time_kind == VLA_TIME_ADA_MLP ? h->W : h->Td;
+  h->qkv_rows = cdiv((h->H + 2) * h->D, 128) * 128;
+  h->ring_off = cfg->n_static_max;
+  h->dyn_off = cfg->n_static_max + cfg->n_sliding;
+  h->kcap = h->dyn_off + h->S;
+  h->max_M = cfg->max_batch * h->S;
+  const int L = h->L, W = h->W, H = h->H, D = h->D, F = h->F, DH = D / 2;
+
+  auto cleanup = [&](int code) {
+    vla_expert_destroy(h);
+    return code;
+  };
+
+  // ---- projection weights, repacked for the GEMM epilogues
+  {
+    std::vector<uint16_t> pk(static_cast<size_t>(L) * h->qkv_rows * W, 0);
+    for (int l = 0; l < L; ++l)
+      for (int r = 0; r < (H + 2) * D; ++r) {
+        const int pr = r >> 1, second = r & 1;
+        const uint16_t* src;
+        if (pr < H * DH) {
+          const int head = pr / DH, i = pr % DH;
+          src = w->wq + (static_cast<size_t>(l) * H * D + head * D + i + second * DH) * W;
+        } else if (pr < (H + 1) * DH) {
+          const int i = pr - H * DH;
+          src = w->wk + (static_cast<size_t>(l) * D + i + second * DH) * W;
+        } else {
+          const int i = pr - (H + 1) * DH;
+          src = w->wv + (static_cast<size_t>(l) * D + i + second * DH) * W;
+        }
+        std::memcpy(&pk[(static_cast<size_t>(l) * h->qkv_rows + r) * W], src, W * 2);
+      }
+    if ((rc = upload_bf16(h, &h->wqkv, pk.data(), pk.size()))) return cleanup(rc);
+  }
+  if ((rc = upload_bf16(h, &h->wo, w->wo, static_cast<size_t>(L) * W * h->HD))) return cleanup(rc);
+  {
+    std::vector<uint16_t> pk(static_cast<size_t>(L) * 2 * F * W);
+    for (int l = 0; l < L; ++l)
+      for (int f = 0; f < F; ++f) {
+        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f) * W], w->w_gate + (static_cast<size_t>(l) * F + f) * W, W * 2);
+        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f + 1) * W], w->w_up + (static_cast<size_t>(l) * F + f) * W, W * 2);
+      }
+    if ((rc = upload_bf16(h, &h->wgu, pk.data(), pk.size()))) return cleanup(rc);
+  }
+  if ((rc = upload_bf16(h, &h->wdown, w->w_down, static_cast<size_t>(L) * W * F))) return cleanup(rc);
+
+  // ---- small fp32 parameters
+  if ((rc = upload_f32(h, &h->ain_w, w->action_in_w, static_cast<size_t>(W) * h->A))) return cleanup(rc);
+  if ((rc = upload_f32(h, &h->ain_b, w->action_in_b, W))) return cleanup(rc);
+  if ((rc = upload_f32(h, &h->aout_w, w->action_out_w, static_cast<size_t>(h->A) * W))) return cleanup(rc);
+  if ((rc = upload_f32(h, &h->aout_b, w->action_out_b, h->A))) return cleanup(rc);
+  if (h->hs) {
+    if ((rc = upload_f32(h, &h->st_w, w->state_in_w, static_cast<size_t>(W) * h->Sd))) return cleanup(rc);
+    if ((rc = upload_f32(h, &h->st_b, w->state_in_b, W))) return cleanup(rc);
+  }
+  if (h->pi0) {
+    std::vector<uint16_t> w1a(static_cast<size_t>(W) * W);
+    for (int n = 0; n < W; ++n)
+      std::memcpy(&w1a[static_cast<size_t>(n) * W], w->time_mlp_in_w + static_cast<size_t>(n) * (W + h->Td), W * 2);
+    if ((rc = upload_bf16(h, &h->w1a, w1a.data(), w1a.size()))) return cleanup(rc);
+    if ((rc = upload_bf16(h, &h->w2, w->time_mlp_out_w, static_cast<size_t>(W) * W))) return cleanup(rc);
+    if ((rc = upload_bf16(h, &h->tin_full, w->time_mlp_in_w, static_cast<size_t>(W) * (W + h->Td)))) return cleanup(rc);
+    if ((rc = upload_bf16(h, &h->tin_b, w->time_mlp_in_b, W))) return cleanup(rc);
+    if ((rc = upload_f32(h, &h->t2_b, w->time_mlp_out_b, W))) return cleanup(rc);
+    if ((rc = upload_f32(h, &h->n1_w, w->norm1_w, static_cast<size_t>(L) * W))) return cleanup(rc);
+    if ((rc = upload_f32(h, &h->n2_w, w->norm2_w, static_cast<size_t>(L) * W))) return cleanup(rc);
+    if ((rc = upload_f32(h, &h->nf_w, w->final_norm_w, W))) return cleanup(rc);
+  } else {
+    if (cfg->time_kind == VLA_TIME_ADA_MLP) {
+      if ((rc = upload_bf16(h, &h->cond1_w, w->time_cond1_w, static_cast<size_t>(W) * h->Td))) return cleanup(rc);
+      if ((rc = upload_bf16(h, &h->cond1_b, w->time_cond1_b, W))) return cleanup(rc);
+      if ((rc = upload_bf16(h, &h->cond2_w, w->time_cond2_w, static_cast<size_t>(W) * W))) return cleanup(rc);
+      if ((rc = upload_bf16(h, &h->cond2_b, w->time_cond2_b, W))) return cleanup(rc);
+    }
+    // norm j: 2l = norm1 of layer l, 2l + 1 = norm2, 2L = final; each [3W][Cd]
+    const size_t per = static_cast<size_t>(3) * W * h->Cd;
+    std::vector<uint16_t> mw(per * (2 * L + 1)), mb(static_cast<size_t>(3) * W * (2 * L + 1));
+    for (int j = 0; j <= 2 * L; ++j) {
+      const uint16_t *sw, *sb;
+      if (j == 2 * L) {
+        sw = w->final_norm_mod_w;
+        sb = w->final_norm_mod_b;
+      } else {
+        const int l = j / 2;
+        sw = ((j & 1) ? w->norm2_mod_w : w->norm1_mod_w) + per * l;
+        sb = ((j & 1) ? w->norm2_mod_b : w->norm1_mod_b) + static_cast<size_t>(3) * W * l;
+      }
+      std::memcpy(&mw[per * j], sw, per * 2);
+      std::memcpy(&mb[static_cast<size_t>(3) * W * j], sb, static_cast<size_t>(3) * W * 2);
+    }
+    if ((rc = upload_bf16(h, &h->mod_w, mw.data(), mw.size()))) return cleanup(rc);
+    if ((rc = upload_bf16(h, &h->mod_b, mb.data(), mb.size()))) return cleanup(rc);
+  }
+
+  // ---- activations, cache, workspaces
+  const int Mx = h->max_M;
+  if ((rc = dalloc(h, &h->x, static_cast<size_t>(cfg->max_batch) * h->C * h->A))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->hx, static_cast<size_t>(cfg->max_batch) * h->C * h->A))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->state, static_cast<size_t>(cfg->max_batch) * std::max(1, h->Sd)))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->hstate, static_cast<size_t>(cfg->max_batch) * std::max(1, h->Sd)))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->resid, static_cast<size_t>(Mx) * W))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->hb, static_cast<size_t>(Mx) * W))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->qb, static_cast<size_t>(Mx) * h->HD))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->ob, static_cast<size_t>(Mx) * h->HD))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->ub, static_cast<size_t>(Mx) * F))) return cleanup(rc);
+  if (h->pi0) {
+    if ((rc = dalloc(h, &h->eb, static_cast<size_t>(Mx) * W))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->h1b, static_cast<size_t>(Mx) * W))) return cleanup(rc);
+  }
+  const size_t cache_elems = static_cast<size_t>(L) * cfg->max_batch * h->kcap * D;
+  if ((rc = dalloc(h, &h->kc, cache_elems))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->vc, cache_elems))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->rope, static_cast<size_t>(h->S) * D))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->desc, 1))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->err, 1))) return cleanup(rc);
+
+  // workspace sizes: the largest plan over every batch size up to max_batch
+  {
+    const int shapes[6][2] = {{h->qkv_rows, W}, {W, h->HD}, {2 * F, W}, {W, F}, {W, W}, {W, W}};
+    const int key_tiles_max = cdiv(cfg->n_static_max, attn_key_tile(D)) + cdiv(cfg->n_sliding, attn_key_tile(D)) +
+                              cdiv(h->S, attn_key_tile(D));
+    for (int b = 1; b <= cfg->max_batch; ++b) {
+      for (auto& sh : shapes) {
+        const GemmPlan g = plan_gemm(sh[0], sh[1], b * h->S, h->sm_count);
+        h->ws_floats = std::max(h->ws_floats, static_cast<size_t>(g.n_tiles) * g.m_tiles * g.splits * g.tn * 128);
+        h->ctr_ints = std::max(h->ctr_ints, static_cast<size_t>(g.n_tiles) * g.m_tiles);
+      }
+      const AttnPlan a = plan_attn(h->S * H, b, key_tiles_max, h->sm_count);
+      if (a.splits > 1)
+        h->part_floats = std::max(h->part_floats, static_cast<size_t>(b) * a.q_tiles * a.splits * attn_q_tile() * D);
+      h->attn_ctr_ints = std::max(h->attn_ctr_ints, static_cast<size_t>(b) * a.q_tiles);
+    }
+  }
+  if ((rc = dalloc(h, &h->ws, h->ws_floats))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->ctr, h->ctr_ints))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->part_o, h->part_floats))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->part_ml, h->part_floats / std::max(1, D) * 2 + 2))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->attn_ctr, h->attn_ctr_ints))) return cleanup(rc);
+
+  // ---- time tables
+  h->table_stride = h->ada ? static_cast<long>(2 * L + 1) * 3 * W : W;
+  for (int i = 0; i < kTableSlots; ++i) {
+    if ((rc = dalloc(h, &h->tables[i], static_cast<size_t>(cfg->max_steps) * h->table_stride))) return cleanup(rc);
+    h->table_steps[i] = 0;
+  }
+  if ((rc = dalloc(h, &h->temb, static_cast<size_t>(cfg->max_steps) * h->Td))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->tscr1, static_cast<size_t>(cfg->max_steps) * W))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->tscr2, static_cast<size_t>(cfg->max_steps) * W))) return cleanup(rc);
+
+  // ---- TMA descriptors of the stacked weights
+  if ((rc = make_tmap(&h->tm_wqkv, h->wqkv, W, static_cast<uint64_t>(L) * h->qkv_rows, 128))) return cleanup(rc);
+  if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
+  if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  if (h->pi0) {
+    if ((rc = make_tmap(&h->tm_w1a, h->w1a, W, W, 128))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_w2, h->w2, W, W, 128))) return cleanup(rc);
+  } else {
+    h->tm_w1a = h->tm_wo;
+    h->tm_w2 = h->tm_wo;
+  }
+
+  cudaError_t e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cleanup(fail(VLA_ERR_CUDA, "stream create: %s", cudaGetErrorString(e)));
+  int slot;
+  if ((rc = ensure_tables(h, cfg->max_steps, h->cap, &slot))) return cleanup(rc);
+  e = cudaStreamSynchronize(h->cap);
+  if (e != cudaSuccess) return cleanup(fail(VLA_ERR_CUDA, "create: %s", cudaGetErrorString(e)));
+  *out = h;
+  return VLA_OK;
+}
+
+void vla_expert_destroy(vla_expert* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  for (auto& kv : h->graphs) {
+    cudaGraphExecDestroy(kv.second.exec);
+    cudaGraphDestroy(kv.second.g);
+  }
+  for (void* p : h->allocs) cudaFree(p);
+  if (h->cap) cudaStreamDestroy(h->cap);
+  delete h;
+}
+
+int vla_cache_set_prefix(vla_expert* h, const uint16_t* K, const uint16_t* V, int n_tokens, int batch,
+                         void* cuda_stream) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (n_tokens > 0 && (!K || !V)) return fail(VLA_ERR_ARG, "null K or V");
+  if (batch < 1 || batch > h->cfg.max_batch)
+    return fail(VLA_ERR_SHAPE, "batch %d outside [1, %d]", batch, h->cfg.max_batch);
+  if (n_tokens < 0 || n_tokens > h->cfg.n_static_max + h->cfg.n_sliding)
+    return fail(VLA_ERR_SHAPE, "n_tokens %d outside [0, %d]", n_tokens, h->cfg.n_static_max + h->cfg.n_sliding);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  CU(launch_prefix_set(reinterpret_cast<const bf16*>(K), reinterpret_cast<const bf16*>(V), n_tokens, batch, h->L,
+                       h->D, h->cfg.max_batch, h->kcap, h->cfg.n_static_max, h->kc, h->vc, s));
+  const int n_static = std::min(n_tokens, h->cfg.n_static_max);
+  const int n_ring = n_tokens - n_static;
+  CU(launch_cache_update(h->desc, n_static, n_ring, h->rope, h->S, h->D, h->cfg.rope_base, s));
+  h->n_static = n_static;
+  h->n_ring = n_ring;
+  h->head = h->cfg.n_sliding > 0 ? n_ring % h->cfg.n_sliding : 0;
+  h->prefix_batch = batch;
+  h->prefix_loaded = true;
+  return VLA_OK;
+}
+
+int vla_cache_append_sliding(vla_expert* h, const uint16_t* K_tok, const uint16_t* V_tok, int batch,
+                             void* cuda_stream) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (!K_tok || !V_tok) return fail(VLA_ERR_ARG, "null K_tok or V_tok");
+  if (h->cfg.n_sliding < 1) return fail(VLA_ERR_STATE, "no sliding region (n_sliding = 0)");
+  if (!h->prefix_loaded) return fail(VLA_ERR_STATE, "no prefix set");
+  if (batch < 1 || batch > h->cfg.max_batch || batch != h->prefix_batch)
+    return fail(VLA_ERR_SHAPE, "batch %d must equal the prefix batch %d", batch, h->prefix_batch);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  CU(launch_ring_append(reinterpret_cast<const bf16*>(K_tok), reinterpret_cast<const bf16*>(V_tok), batch, h->L,
+                        h->D, h->cfg.max_batch, h->kcap, h->ring_off + h->head, h->kc, h->vc, s));
+  const int n_ring = std::min(h->n_ring + 1, h->cfg.n_sliding);
+  if (n_ring != h->n_ring)
+    CU(launch_cache_update(h->desc, h->n_static, n_ring, h->rope, h->S, h->D, h->cfg.rope_base, s));
+  h->n_ring = n_ring;
+  h->head = (h->head + 1) % h->cfg.n_sliding;
+  return VLA_OK;
+}
+
+int vla_denoise(vla_expert* h, const float* noise, const float* state, int steps, float* out_actions,
+                int batch, void* cuda_stream) {
+  g_err.clear();
+  int rc = check_denoise_args(h, noise, state, steps, out_actions, batch);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  int slot;
+  if ((rc = ensure_tables(h, steps, s, &slot))) return rc;
+  cudaGraphExec_t ex;
+  if ((rc = get_graph(h, batch, steps, slot, &ex))) return rc;
+  const size_t xb = static_cast<size_t>(batch) * h->C * h->A * sizeof(float);
+  CU(cudaMemcpyAsync(h->x, noise, xb, cudaMemcpyDeviceToDevice, s));
+  if (h->Sd > 0)
+    CU(cudaMemcpyAsync(h->state, state, static_cast<size_t>(batch) * h->Sd * sizeof(float),
+                       cudaMemcpyDeviceToDevice, s));
+  CU(cudaGraphLaunch(ex, s));
+  CU(cudaMemcpyAsync(out_actions, h->x, xb, cudaMemcpyDeviceToDevice, s));
+  return VLA_OK;
+}
+
+int vla_denoise_host(vla_expert* h, const float* noise, const float* state, int steps, float* out_actions,
+                     int batch, void* cuda_stream) {
+  g_err.clear();
+  int rc = check_denoise_args(h, noise, state, steps, out_actions, batch);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t xb = static_cast<size_t>(batch) * h->C * h->A * sizeof(float);
+  CU(cudaMemcpyAsync(h->hx, noise, xb, cudaMemcpyHostToDevice, s));
+  if (h->Sd > 0)
+    CU(cudaMemcpyAsync(h->hstate, state, static_cast<size_t>(batch) * h->Sd * sizeof(float),
+                       cudaMemcpyHostToDevice, s));
+  int slot;
+  if ((rc = ensure_tables(h, steps, s, &slot))) return rc;
+  cudaGraphExec_t ex;
+  if ((rc = get_graph(h, batch, steps, slot, &ex))) return rc;
+  CU(cudaMemcpyAsync(h->x, h->hx, xb, cudaMemcpyDeviceToDevice, s));
+  if (h->Sd > 0)
+    CU(cudaMemcpyAsync(h->state, h->hstate, static_cast<size_t>(batch) * h->Sd * sizeof(float),
+                       cudaMemcpyDeviceToDevice, s));
+  CU(cudaGraphLaunch(ex, s));
+  CU(cudaMemcpyAsync(out_actions, h->x, xb, cudaMemcpyDeviceToHost, s));
+  CU(cudaStreamSynchronize(s));
+  return VLA_OK;
+}
+
+int vla_cache_export(vla_expert* h, uint16_t* K_out, uint16_t* V_out, int batch, int* head, int* n_static,
+                     int* n_ring, void* cuda_stream) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (batch < 1 || batch > h->cfg.max_batch)
+    return fail(VLA_ERR_SHAPE, "batch %d outside [1, %d]", batch, h->cfg.max_batch);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const int rows = h->cfg.n_static_max + h->cfg.n_sliding;
+  if (K_out) CU(launch_copy_region(h->kc, reinterpret_cast<bf16*>(K_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D, s));
+  if (V_out) CU(launch_copy_region(h->vc, reinterpret_cast<bf16*>(V_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D, s));
+  if (head) *head = h->head;
+  if (n_static) *n_static = h->n_static;
+  if (n_ring) *n_ring = h->n_ring;
+  return VLA_OK;
+}
+
+int vla_device_status(vla_expert* h, void* cuda_stream) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  CU(cudaStreamSynchronize(s));
+  int v = 0;
+  CU(cudaMemcpy(&v, h->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    cudaMemset(h->err, 0, sizeof(int));
+    cudaMemset(h->ctr, 0, h->ctr_ints * sizeof(int));
+    cudaMemset(h->attn_ctr, 0, h->attn_ctr_ints * sizeof(int));
+    cudaDeviceSynchronize();
+    return fail(VLA_ERR_TIMEOUT, "a kernel wait timed out (device status %d); split counters were reset", v);
+  }
+  return VLA_OK;
+}
+
+int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, int steps, float* out_actions,
+                        int batch, vla_kernel_times* times, void* cuda_stream) {
+  g_err.clear();
+  int rc = check_denoise_args(h, noise, state, steps, out_actions, batch);
+  if (rc) return rc;
+  if (!times) return fail(VLA_ERR_ARG, "null times");
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  int slot;
+  if ((rc = ensure_tables(h, steps, s, &slot))) return rc;
+  ActMaps am;
+  if ((rc = make_act_maps(h, batch, &am))) return rc;
+  const size_t xb = static_cast<size_t>(batch) * h->C * h->A * sizeof(float);
+  CU(cudaMemcpyAsync(h->x, noise, xb, cudaMemcpyDeviceToDevice, s));
+  if (h->Sd > 0)
+    CU(cudaMemcpyAsync(h->state, state, static_cast<size_t>(batch) * h->Sd * sizeof(float),
+                       cudaMemcpyDeviceToDevice, s));
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> kinds;
+  Recorder rec;
+  rec.s = s;
+  rec.events = &ev;
+  rec.kinds = &kinds;
+  rc = enqueue_denoise(h, batch, steps, slot, am, rec);
+  if (rc == VLA_OK) {
+    cudaError_t e = cudaMemcpyAsync(out_actions, h->x, xb, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) rc = fail(VLA_ERR_CUDA, "profile run: %s", cudaGetErrorString(e));
+  }
+  if (rc == VLA_OK) {
+    std::memset(times, 0, sizeof(*times));
+    for (size_t i = 0; i < kinds.size(); ++i) {
+      float ms = 0.0f;
+      cudaEventElapsedTime(&ms, ev[2 * i], ev[2 * i + 1]);
+      times->total_ms[kinds[i]] += ms;
+      times->launches[kinds[i]] += 1;
+    }
+    // algorithmic bytes / FLOPs per denoise (weights read once per launch, activations once)
+    const double B = batch, M = static_cast<double>(batch) * h->S, W = h->W, L = h->L, N = steps;
+    const double HD = h->HD, D = h->D, F = h->F;
+    const double qkv = static_cast<double>((h->H + 2) * h->D);
+    const double keys = static_cast<double>(h->n_static + h->n_ring + h->S);
+    times->bytes[VLA_K_GEMM_QKV] = N * L * (2.0 * qkv * W + 2.0 * M * W + 2.0 * M * qkv);
+    times->flops[VLA_K_GEMM_QKV] = N * L * 2.0 * M * qkv * W;
+    times->bytes[VLA_K_GEMM_O] = N * L * (2.0 * W * HD + 2.0 * M * HD + 8.0 * M * W);
+    times->flops[VLA_K_GEMM_O] = N * L * 2.0 * M * W * HD;
+    times->bytes[VLA_K_GEMM_GATEUP] = N * L * (2.0 * 2 * F * W + 2.0 * M * W + 2.0 * M * F);
+    times->flops[VLA_K_GEMM_GATEUP] = N * L * 2.0 * M * 2 * F * W;
+    times->bytes[VLA_K_GEMM_DOWN] = N * L * (2.0 * W * F + 2.0 * M * F + 8.0 * M * W);
+    times->flops[VLA_K_GEMM_DOWN] = N * L * 2.0 * M * W * F;
+    times->bytes[VLA_K_ATTN] = N * L * (B * keys * D * 2 * 2 + 2.0 * 2 * M * HD);
+    times->flops[VLA_K_ATTN] = N * L * 4.0 * M * h->H * keys * D;
+    times->bytes[VLA_K_NORM] = N * L * 2 * (4.0 * M * W + 2.0 * M * W);
+    times->bytes[VLA_K_EMBED] = N * (4.0 * M * W);
+    times->bytes[VLA_K_FINAL] = N * (4.0 * B * h->C * W + 4.0 * h->A * W);
+    if (h->pi0) {
+      times->bytes[VLA_K_TIME_MLP] = N * (2.0 * 2 * W * W + 2.0 * 2 * M * W + 2.0 * M * W + 4.0 * M * W);
+      times->flops[VLA_K_TIME_MLP] = N * 2.0 * 2.0 * M * W * W;
+    }
+  }
+  for (auto e : ev) cudaEventDestroy(e);
+  return rc;
+}
+
+int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim, int m_tok,
+                  int split_k, void* cuda_stream) {
+  g_err.clear();
+  if (!W || !X || !Y) return fail(VLA_ERR_ARG, "null W, X or Y");
+  if (n_feat < 128 || n_feat % 128 || k_dim < 64 || k_dim % 64 || m_tok < 1)
+    return fail(VLA_ERR_SHAPE, "need n_feat %% 128 == 0, k_dim %% 64 == 0, m_tok >= 1 (got %d, %d, %d)", n_feat,
+                k_dim, m_tok);
+  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(X)) & 15)
+    return fail(VLA_ERR_ARG, "W and X must be 16-byte aligned");
+  if (split_k < 0) return fail(VLA_ERR_ARG, "split_k must be >= 0");
+  int dev = 0, major = 0, sms = 148;
+  CU(cudaGetDevice(&dev));
+  CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (major != 10) return fail(VLA_ERR_UNSUPPORTED, "device is sm_%d0; this library is built for sm_100a", major);
+  CU(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  CU(configure_gemm_kernels());
+  GemmPlan g = plan_gemm(n_feat, k_dim, m_tok, sms);
+  if (split_k > 0) {
+    const int nkb = k_dim / 64;
+    g.kb_per_split = cdiv(nkb, std::min(split_k, nkb));
+    g.splits = cdiv(nkb, g.kb_per_split);
+  }
+  CUtensorMap tw, tx;
+  int rc;
+  if ((rc = make_tmap(&tw, W, k_dim, n_feat, 128))) return rc;
+  if ((rc = make_tmap(&tx, X, k_dim, m_tok, g.tn))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t n_ctr = static_cast<size_t>(g.n_tiles) * g.m_tiles + 1;
+  const size_t ws_bytes = g.splits > 1 ? static_cast<size_t>(g.n_tiles) * g.m_tiles * g.splits * g.tn * 128 * 4 : 0;
+  void* scratch = nullptr;
+  CU(cudaMallocAsync(&scratch, ws_bytes + n_ctr * sizeof(int), s));
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(scratch) + ws_bytes);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, n_ctr * sizeof(int), s);
+  GemmParams p{};
+  p.n_feat = n_feat;
+  p.k_dim = k_dim;
+  p.m_tok = m_tok;
+  p.splits = g.splits;
+  p.kb_per_split = g.kb_per_split;
+  p.resid = Y;
+  p.ld_resid = n_feat;
+  p.ws = static_cast<float*>(scratch);
+  p.counters = ctr;
+  p.err = ctr + n_ctr - 1;
+  if (e == cudaSuccess) e = launch_gemm(g.tn, EPI_STORE, tw, tx, p, g.n_tiles, g.m_tiles, s, false);
+  cudaError_t e2 = cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) return fail(VLA_ERR_CUDA, "vla_gemm_bf16 launch: %s", cudaGetErrorString(e));
+  if (e2 != cudaSuccess) return fail(VLA_ERR_CUDA, "vla_gemm_bf16 free: %s", cudaGetErrorString(e2));
+  return VLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,401 @@
+// attention.cu -- suffix attention against the partitioned K/V cache.
+//
+// Reflex abstract: the attention context is partitioned into a static region (cached
+// perception / prompt keys), a sliding region (a ring of recent tokens, O(1) updates)
+// and a dynamic region (the action chunk, recomputed at every Euler step); the cached
+// computation matches full recompute for fixed inputs. realtime-vla write-up: the
+// action expert attends to the LLM's prefix.
+//
+// All H query heads share the single K/V head (GQA), so an observation's S*H query rows
+// form one [S*H, D] matrix against one key sequence. A CTA takes 64 query rows (4 warps
+// x 16) and one contiguous range of key tiles ("split"); keys are walked segment by
+// segment (static [0, n_static), ring [ring_off, ring_off + n_ring), dynamic
+// [dyn_off, dyn_off + S)), staged through shared memory by a 2-deep cp.async pipeline,
+// and contracted with bf16 mma.sync (fp32 accumulate) with an online softmax in fp32.
+// Splits write unnormalised partials; the last CTA of a query tile to arrive merges them
+// in split order (deterministic).
+//
+// Mask (prefix-LM): every suffix row sees every cached key; action rows see the whole
+// suffix; with a state token, suffix row 0 sees the cached keys and itself only.
+#include <cfloat>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace vla {
+
+constexpr int kQT = 64;   // query rows per CTA
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+template <int D>
+struct AttnCfg {
+  static constexpr int KT = D >= 256 ? 32 : 64;            // keys per stage
+  static constexpr int CPR = D / 8;                        // 16-byte chunks per row
+  static constexpr int SWZ = (CPR >= 8 ? 8 : CPR) - 1;     // XOR mask for chunk swizzle
+  static constexpr size_t SMEM = (size_t)(kQT + 4 * KT) * D * 2;
+};
+
+// byte offset of (row, chunk) in a swizzled [rows][D] bf16 tile
+template <int D>
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  using C = AttnCfg<D>;
+  return static_cast<uint32_t>((row * C::CPR + (chunk ^ (row & C::SWZ))) * 16);
+}
+
+// Key tile t of the concatenated segment list -> (segment row offset, first key, count).
+struct Segs {
+  int off[3], cnt[3], ntile[3];
+};
+
+template <int D>
+__device__ __forceinline__ void tile_info(const Segs& sg, int t, int& row, int& cnt, int& dyn_start) {
+  using C = AttnCfg<D>;
+  int seg = 0;
+  while (seg < 2 && t >= sg.ntile[seg]) {
+    t -= sg.ntile[seg];
+    ++seg;
+  }
+  const int start = t * C::KT;
+  row = sg.off[seg] + start;
+  cnt = min(C::KT, sg.cnt[seg] - start);
+  dyn_start = seg == 2 ? start : -1;
+}
+
+template <int D>
+__device__ __forceinline__ void load_kv_tile(const bf16* kbase, const bf16* vbase, int row, int cnt,
+                                             uint32_t sk, uint32_t sv) {
+  using C = AttnCfg<D>;
+  for (int idx = threadIdx.x; idx < C::KT * C::CPR; idx += blockDim.x) {
+    const int r = idx / C::CPR, c = idx % C::CPR;
+    const bool ok = r < cnt;
+    const size_t g = static_cast<size_t>(ok ? row + r : row) * D + c * 8;
+    cp_async16(sk + swz<D>(r, c), kbase + g, ok ? 16 : 0);
+    cp_async16(sv + swz<D>(r, c), vbase + g, ok ? 16 : 0);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
+  using C = AttnCfg<D>;
+  constexpr int KT = C::KT;
+  constexpr int NB = KT / 8;     // 8-key column blocks of S
+  constexpr int OB = D / 8;      // 8-dim column blocks of O
+  extern __shared__ __align__(128) uint8_t sm[];
+  const uint32_t sQ = smem_u32(sm);
+  const uint32_t sK0 = sQ + kQT * D * 2;
+  const uint32_t sV0 = sK0 + 2 * KT * D * 2;
+
+  const int qt = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = p.n_heads, R = p.seq * H;
+  const int row0 = qt * kQT;
+
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const CacheDesc cd = *p.cache;
+  Segs sg;
+  sg.off[0] = 0;
+  sg.cnt[0] = cd.n_static;
+  sg.off[1] = p.ring_off;
+  sg.cnt[1] = cd.n_ring;
+  sg.off[2] = p.dyn_off;
+  sg.cnt[2] = p.seq;
+  int T = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    sg.ntile[i] = (sg.cnt[i] + KT - 1) / KT;
+    T += sg.ntile[i];
+  }
+  const int t_begin = static_cast<int>((static_cast<long long>(split) * T) / p.n_splits);
+  const int t_end = static_cast<int>((static_cast<long long>(split + 1) * T) / p.n_splits);
+
+  const bf16* qbase = p.q + static_cast<size_t>(b) * R * D;
+  const bf16* kbase = p.kc + static_cast<size_t>(b) * p.kcap * D;
+  const bf16* vbase = p.vc + static_cast<size_t>(b) * p.kcap * D;
+
+  // Q tile, zero rows past the end
+  for (int idx = threadIdx.x; idx < kQT * C::CPR; idx += blockDim.x) {
+    const int r = idx / C::CPR, c = idx % C::CPR;
+    const bool ok = row0 + r < R;
+    cp_async16(sQ + swz<D>(r, c), qbase + static_cast<size_t>(ok ? row0 + r : 0) * D + c * 8,
+               ok ? 16 : 0);
+  }
+  if (t_begin < t_end) {
+    int row, cnt, ds;
+    tile_info<D>(sg, t_begin, row, cnt, ds);
+    load_kv_tile<D>(kbase, vbase, row, cnt, sK0, sV0);
+  }
+  cp_async_commit();
+
+  float o[OB][4];
+#pragma unroll
+  for (int i = 0; i < OB; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.0f, 0.0f};
+
+  const int wrow = warp * 16;                      // this warp's first row in the tile
+  const int g = lane >> 2, qd = lane & 3;          // fragment row group / quad position
+  const int s_row[2] = {(row0 + wrow + g) / H, (row0 + wrow + g + 8) / H};
+
+  for (int t = t_begin; t < t_end; ++t) {
+    const int st = (t - t_begin) & 1;
+    if (t + 1 < t_end) {
+      int row, cnt, ds;
+      tile_info<D>(sg, t + 1, row, cnt, ds);
+      load_kv_tile<D>(kbase, vbase, row, cnt, sK0 + (st ^ 1) * KT * D * 2, sV0 + (st ^ 1) * KT * D * 2);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint32_t sK = sK0 + st * KT * D * 2, sV = sV0 + st * KT * D * 2;
+    int trow, tcnt, dyn_start;
+    tile_info<D>(sg, t, trow, tcnt, dyn_start);
+
+    // S = Q K^T for this warp's 16 rows x KT keys
+    float sacc[NB][4];
+#pragma unroll
+    for (int i = 0; i < NB; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(a, sQ + swz<D>(wrow + (lane & 15), kk * 2 + (lane >> 4)));
+#pragma unroll
+      for (int nb2 = 0; nb2 < KT / 16; ++nb2) {
+        uint32_t bf[4];
+        ldsm_x4(bf, sK + swz<D>(nb2 * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
+        mma_bf16_16816(sacc[2 * nb2], a, bf[0], bf[1]);
+        mma_bf16_16816(sacc[2 * nb2 + 1], a, bf[2], bf[3]);
+      }
+    }
+    // scale into the log2 domain and mask
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int col = nb * 8 + qd * 2 + (e & 1);
+        bool ok = col < tcnt;
+        if (dyn_start >= 0 && p.has_state && s_row[e >> 1] == 0 && dyn_start + col != 0) ok = false;
+        const float v = ok ? sacc[nb][e] * p.scale_log2 : -INFINITY;
+        sacc[nb][e] = v;
+        mx[e >> 1] = fmaxf(mx[e >> 1], v);
+      }
+    }
+    float corr[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
+      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+      const float m_new = fmaxf(m_run[h2], mx[h2]);
+      corr[h2] = (m_run[h2] == -INFINITY) ? 0.0f : exp2f(m_run[h2] - m_new);
+      m_run[h2] = m_new;
+    }
+    float lsum[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float mref = m_run[e >> 1];
+        const float pv = (mref == -INFINITY) ? 0.0f : exp2f(sacc[nb][e] - mref);
+        sacc[nb][e] = pv;
+        lsum[e >> 1] += pv;
+      }
+    }
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) l_run[h2] = l_run[h2] * corr[h2] + lsum[h2];
+#pragma unroll
+    for (int i = 0; i < OB; ++i) {
+      o[i][0] *= corr[0];
+      o[i][1] *= corr[0];
+      o[i][2] *= corr[1];
+      o[i][3] *= corr[1];
+    }
+    // O += P V
+#pragma unroll
+    for (int kb = 0; kb < KT / 16; ++kb) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(sacc[2 * kb][0], sacc[2 * kb][1]);
+      pa[1] = pack_bf16(sacc[2 * kb][2], sacc[2 * kb][3]);
+      pa[2] = pack_bf16(sacc[2 * kb + 1][0], sacc[2 * kb + 1][1]);
+      pa[3] = pack_bf16(sacc[2 * kb + 1][2], sacc[2 * kb + 1][3]);
+#pragma unroll
+      for (int db = 0; db < D / 16; ++db) {
+        uint32_t vf[4];
+        ldsm_x4_t(vf, sV + swz<D>(kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), db * 2 + (lane >> 4)));
+        mma_bf16_16816(o[2 * db], pa, vf[0], vf[1]);
+        mma_bf16_16816(o[2 * db + 1], pa, vf[2], vf[3]);
+      }
+    }
+    __syncthreads();
+  }
+
+  // quad-reduce the row sums
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    l_run[h2] += __shfl_xor_sync(0xffffffffu, l_run[h2], 1);
+    l_run[h2] += __shfl_xor_sync(0xffffffffu, l_run[h2], 2);
+  }
+  const int rloc[2] = {wrow + g, wrow + g + 8};
+
+  if (p.n_splits == 1) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int r = row0 + rloc[h2];
+      if (r >= R) continue;
+      const float inv = l_run[h2] > 0.0f ? 1.0f / l_run[h2] : 0.0f;
+      bf16* dst = p.out + (static_cast<size_t>(b) * R + r) * D;
+#pragma unroll
+      for (int i = 0; i < OB; ++i) {
+        const __nv_bfloat162 v2 = __floats2bfloat162_rn(o[i][2 * h2] * inv, o[i][2 * h2 + 1] * inv);
+        *reinterpret_cast<__nv_bfloat162*>(dst + i * 8 + qd * 2) = v2;
+      }
+    }
+    return;
+  }
+
+  // split partials, then the last CTA of this query tile merges them in split order
+  const int q_tiles = gridDim.x;
+  const size_t slot = (static_cast<size_t>(b) * q_tiles + qt) * p.n_splits + split;
+  float* po = p.part_o + slot * kQT * D;
+  float* pml = p.part_ml + slot * kQT * 2;
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+    for (int i = 0; i < OB; ++i)
+      __stcg(reinterpret_cast<float2*>(po + rloc[h2] * D + i * 8 + qd * 2),
+             make_float2(o[i][2 * h2], o[i][2 * h2 + 1]));
+    if (qd == 0) __stcg(reinterpret_cast<float2*>(pml + rloc[h2] * 2), make_float2(m_run[h2], l_run[h2]));
+  }
+  __threadfence();
+  __syncthreads();
+  __shared__ int s_last;
+  int* ctr = p.counters + static_cast<size_t>(b) * q_tiles + qt;
+  if (threadIdx.x == 0) s_last = (atomicAdd(ctr, 1) == p.n_splits - 1) ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  const size_t base = (static_cast<size_t>(b) * q_tiles + qt) * p.n_splits;
+  for (int idx = threadIdx.x; idx < kQT * 2; idx += blockDim.x) {
+    const int r = idx >> 1, half = idx & 1;
+    if (row0 + r >= R) continue;
+    float M = -INFINITY;
+    for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, __ldcg(p.part_ml + ((base + s) * kQT + r) * 2));
+    float wsum = 0.0f;
+    float acc[D / 2];
+#pragma unroll
+    for (int d = 0; d < D / 2; ++d) acc[d] = 0.0f;
+    for (int s = 0; s < p.n_splits; ++s) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((base + s) * kQT + r) * 2));
+      const float w = (ml.x == -INFINITY) ? 0.0f : exp2f(ml.x - M);
+      wsum += w * ml.y;
+      const float* src = p.part_o + ((base + s) * kQT + r) * D + half * (D / 2);
+#pragma unroll
+      for (int d = 0; d < D / 2; d += 4) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + d));
+        acc[d] += w * v.x;
+        acc[d + 1] += w * v.y;
+        acc[d + 2] += w * v.z;
+        acc[d + 3] += w * v.w;
+      }
+    }
+    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+    bf16* dst = p.out + (static_cast<size_t>(b) * R + row0 + r) * D + half * (D / 2);
+#pragma unroll
+    for (int d = 0; d < D / 2; d += 2)
+      *reinterpret_cast<__nv_bfloat162*>(dst + d) = __floats2bfloat162_rn(acc[d] * inv, acc[d + 1] * inv);
+  }
+  if (threadIdx.x == 0) *ctr = 0;
+}
+
+template <int D>
+static cudaError_t configure_d() {
+  return cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(AttnCfg<D>::SMEM));
+}
+
+cudaError_t configure_attention_kernels() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaSuccess) return done;
+  cudaError_t e;
+  if ((e = configure_d<32>()) != cudaSuccess) return e;
+  if ((e = configure_d<64>()) != cudaSuccess) return e;
+  if ((e = configure_d<128>()) != cudaSuccess) return e;
+  if ((e = configure_d<256>()) != cudaSuccess) return e;
+  done = cudaSuccess;
+  return done;
+}
+
+template <int D>
+static cudaError_t launch_d(const AttnParams& p, int batch, int q_tiles, cudaStream_t s, bool pdl) {
+  using C = AttnCfg<D>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q_tiles, p.n_splits, batch);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_kernel<D>, p);
+}
+
+cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
+                             cudaStream_t s, bool pdl) {
+  switch (head_dim) {
+    case 32: return launch_d<32>(p, batch, q_tiles, s, pdl);
+    case 64: return launch_d<64>(p, batch, q_tiles, s, pdl);
+    case 128: return launch_d<128>(p, batch, q_tiles, s, pdl);
+    case 256: return launch_d<256>(p, batch, q_tiles, s, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int attn_q_tile() { return kQT; }
+
+int attn_key_tile(int head_dim) {
+  switch (head_dim) {
+    case 32: return AttnCfg<32>::KT;
+    case 64: return AttnCfg<64>::KT;
+    case 128: return AttnCfg<128>::KT;
+    default: return AttnCfg<256>::KT;
+  }
+}
+
+}  // namespace vla

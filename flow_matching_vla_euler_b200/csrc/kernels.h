@@ -1,0 +1,148 @@
+// kernels.h -- internal launchers of the sm_100a kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vla {
+
+typedef __nv_bfloat16 bf16;
+
+// Device-side view of the cache partition, read by kernels at run time so that a
+// captured graph stays valid when the prefix or the ring changes.
+struct CacheDesc {
+  int n_static;   // valid keys in the static region
+  int n_ring;     // valid ring slots (0..n_sliding); slots [0, n_ring) are valid
+  int pos0;       // RoPE position of suffix token 0 = n_static + n_ring
+  int pad;
+};
+
+// ----------------------------------------------------------------------- GEMM
+// out[token][feature] = sum_k X[token][k] * Wt[feature][k], computed as
+// D[feature][token] in TMEM (weights are the 128-row MMA operand, tokens the N side).
+
+enum Epi : int {
+  EPI_RESID = 0,        // resid[m][n] += gate[n] * acc             (gate may be null: 1)
+  EPI_QKV = 1,          // rotary epilogue; Q -> out, K/V -> cache dynamic region
+  EPI_GEGLU = 2,        // rows interleaved (gate f, up f): out[m][f] = gelu(g) * u
+  EPI_SWISH_VEC = 3,    // out[m][n] = bf16(swish(acc + vec[n]))
+  EPI_BIAS_STORE = 4,   // resid[m][n] = acc + vec[n] (action rows only)
+  EPI_STORE = 5,        // resid[m][n] = acc (plain fp32 product)
+};
+
+struct GemmParams {
+  int n_feat;         // output rows of the (packed) weight, multiple of 128
+  int k_dim;          // reduction length, multiple of 64
+  int m_tok;          // valid tokens (rows of X)
+  int w_row0;         // first row of this weight in the stacked weight tensor map
+  int splits;         // K splits (grid.z)
+  int kb_per_split;   // 64-wide K blocks per split
+  float* resid;       // fp32 residual [m][ld_resid]
+  int ld_resid;
+  const float* vec;   // gate / bias / time vector, indexed by output feature
+  bf16* out;          // bf16 output [m][ld_out]
+  int ld_out;
+  bf16* kc;           // EPI_QKV: this layer's K cache [max_batch][kcap][D]
+  bf16* vc;
+  int kcap, dyn_off, seq, n_heads, head_dim;
+  const float* rope;  // [seq][D/2][2] (cos, sin) at positions pos0 + s
+  int has_state;      // EPI_BIAS_STORE: skip row s == 0 of each observation
+  float* ws;          // split-K partial tiles
+  int* counters;      // one arrival counter per output tile (left at 0)
+  int* err;           // device status word
+};
+
+// tn: token tile (64, 128 or 256). Returns cudaSuccess or the launch error.
+cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                        const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl);
+size_t gemm_smem_bytes(int tn);
+cudaError_t configure_gemm_kernels();
+int gemm_stages(int tn);
+
+// ------------------------------------------------------------------ attention
+
+struct AttnParams {
+  const bf16* q;        // [B][S][H][D] (rows (s, h) contiguous per observation)
+  const bf16* kc;       // this layer's K cache [max_batch][kcap][D]
+  const bf16* vc;
+  bf16* out;            // [B][S][H][D]
+  const CacheDesc* cache;
+  int seq, n_heads, kcap;
+  int ring_off;         // first ring slot row (= n_static_max)
+  int dyn_off;          // first dynamic row (= n_static_max + n_sliding)
+  int has_state;        // row s == 0 sees the prefix and itself only
+  int n_splits;         // key splits (grid.y)
+  float* part_o;        // split partials [B][q_tiles][n_splits][64][D] fp32
+  float* part_ml;       // [B][q_tiles][n_splits][64][2]
+  int* counters;        // [B][q_tiles], left at 0
+  float scale_log2;     // log2(e) / sqrt(D)
+  int* err;
+};
+
+cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
+                             cudaStream_t s, bool pdl);
+int attn_q_tile();                       // query rows per CTA
+cudaError_t configure_attention_kernels();
+int attn_key_tile(int head_dim);         // keys per pipeline stage
+
+// -------------------------------------------------------------- small kernels
+
+struct NormParams {
+  const float* x;       // [M][W]
+  bf16* y;              // [M][W]
+  const float* scale;   // AdaRMSNorm scale [W] (null for plain)
+  const float* shift;   // AdaRMSNorm shift [W]
+  const float* w;       // plain RMSNorm weight [W] (y = n * (1 + w))
+  int M, W;
+  float eps;
+};
+cudaError_t launch_norm(const NormParams& p, cudaStream_t s, bool pdl);
+
+struct EmbedParams {
+  const float* x;        // Euler state [B][C][A]
+  const float* state;    // [B][Sd] or null
+  const float* w_in;     // action_in [W][A] fp32
+  const float* b_in;     // [W]
+  const float* w_st;     // state_in [W][Sd]
+  const float* b_st;
+  float* resid;          // [B*S][W]
+  bf16* e_out;           // Pi0: bf16 action embedding [B*S][W] (state rows zeroed), else null
+  int B, C, A, S, Sd, W, has_state;
+};
+cudaError_t launch_embed(const EmbedParams& p, cudaStream_t s, bool pdl);
+
+struct FinalParams {
+  const float* resid;    // [B*S][W]
+  float* x;              // Euler state [B][C][A], updated in place
+  const float* scale;    // final AdaRMSNorm scale/shift, or null
+  const float* shift;
+  const float* w;        // plain final norm weight
+  const float* w_out;    // action_out [A][W] fp32
+  const float* b_out;    // [A]
+  int B, C, A, S, W, has_state;
+  float eps, dt;
+};
+cudaError_t launch_final(const FinalParams& p, cudaStream_t s, bool pdl);
+
+// Time tables: temb[k][Td] for t_k = 1 - k/steps.
+cudaError_t launch_temb(float* temb, int steps, int time_dim, cudaStream_t s);
+// y[r][o] = act(sum_i x[r][i] * w[o * ldw + i] + b[o]), r < rows, o < n_out.
+cudaError_t launch_rowgemv(const float* x, int rows, int n_in, const bf16* w, long ldw,
+                           const bf16* b, int n_out, float* y, int act_swish, cudaStream_t s);
+
+// Cache maintenance.
+cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L,
+                              int D, int max_batch, int kcap, int n_static_max, bf16* kc,
+                              bf16* vc, cudaStream_t s);
+cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, int D,
+                               int max_batch, int kcap, int slot_row, bf16* kc, bf16* vc,
+                               cudaStream_t s);
+// Writes the cache descriptor and the rotary table [seq][D/2][2] for pos0 = n_static+n_ring.
+cudaError_t launch_cache_update(CacheDesc* desc, int n_static, int n_ring, float* rope,
+                                int seq, int head_dim, float rope_base, cudaStream_t s);
+cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch,
+                               int kcap, int rows, int D, cudaStream_t s);
+
+}  // namespace vla

@@ -1,0 +1,333 @@
+// small_kernels.cu -- the non-GEMM steps of the denoise loop and cache maintenance.
+//
+//  norm        (Ada)RMSNorm of the fp32 residual rows -> bf16 GEMM operand
+//              (Reflex abstract: AdaRMSNorm gated on flow phase)
+//  embed       action / state embeddings into the residual stream
+//  final       final norm, action projection and the Euler update x <- x + dt v
+//              (FlowEdge README "euler 10"; realtime-vla "10 flow steps")
+//  temb/rowgemv  per-step time tables: t-embedding, time MLP, AdaRMSNorm modulation
+//  prefix_set / ring_append / cache_update / copy_region: the static / sliding regions
+//              (Reflex abstract: O(1) incremental cache updates)
+#include <cmath>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace vla {
+
+static inline cudaLaunchConfig_t make_cfg(dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                          cudaLaunchAttribute* attr, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cfg;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ------------------------------------------------------------------------- norm
+// One warp per token row; W is a multiple of 128 so each lane moves float4s.
+__global__ void __launch_bounds__(128) norm_kernel(const NormParams p) {
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + warp;
+  if (row >= p.M) return;
+  const float* x = p.x + static_cast<size_t>(row) * p.W;
+  float ss = 0.0f;
+  for (int i = lane * 4; i < p.W; i += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / static_cast<float>(p.W) + p.eps);
+  bf16* y = p.y + static_cast<size_t>(row) * p.W;
+  for (int i = lane * 4; i < p.W; i += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    float o[4] = {v.x * r, v.y * r, v.z * r, v.w * r};
+    if (p.scale) {
+      const float4 sc = *reinterpret_cast<const float4*>(p.scale + i);
+      const float4 sh = *reinterpret_cast<const float4*>(p.shift + i);
+      o[0] = fmaf(o[0], 1.0f + sc.x, sh.x);
+      o[1] = fmaf(o[1], 1.0f + sc.y, sh.y);
+      o[2] = fmaf(o[2], 1.0f + sc.z, sh.z);
+      o[3] = fmaf(o[3], 1.0f + sc.w, sh.w);
+    } else {
+      const float4 w = *reinterpret_cast<const float4*>(p.w + i);
+      o[0] *= 1.0f + w.x;
+      o[1] *= 1.0f + w.y;
+      o[2] *= 1.0f + w.z;
+      o[3] *= 1.0f + w.w;
+    }
+    __nv_bfloat162 a = __floats2bfloat162_rn(o[0], o[1]);
+    __nv_bfloat162 c = __floats2bfloat162_rn(o[2], o[3]);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&a);
+    pk.y = *reinterpret_cast<uint32_t*>(&c);
+    *reinterpret_cast<uint2*>(y + i) = pk;
+  }
+}
+
+cudaError_t launch_norm(const NormParams& p, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3((p.M + 3) / 4), dim3(128), 0, s, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, norm_kernel, p);
+}
+
+// ------------------------------------------------------------------------ embed
+// One CTA per suffix row. State row: state_in(state); action rows: action_in(x), both
+// fp32. Pi0 routes the action embedding (bf16) into the action-time MLP instead.
+__global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
+  __shared__ float vin[256];
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int m = blockIdx.x;
+  const int b = m / p.S, s = m - b * p.S;
+  const bool st = p.has_state && s == 0;
+  const int len = st ? p.Sd : p.A;
+  const float* src = st ? p.state + static_cast<size_t>(b) * p.Sd
+                        : p.x + (static_cast<size_t>(b) * p.C + (s - p.has_state)) * p.A;
+  const float* w = st ? p.w_st : p.w_in;
+  const float* bias = st ? p.b_st : p.b_in;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) vin[i] = src[i];
+  __syncthreads();
+  for (int n = threadIdx.x; n < p.W; n += blockDim.x) {
+    const float* wr = w + static_cast<size_t>(n) * len;
+    float acc = bias[n];
+    for (int a = 0; a < len; ++a) acc = fmaf(wr[a], vin[a], acc);
+    if (p.e_out && !st) {
+      p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(acc);
+    } else {
+      p.resid[static_cast<size_t>(m) * p.W + n] = acc;
+      if (p.e_out) p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(0.0f);
+    }
+  }
+}
+
+cudaError_t launch_embed(const EmbedParams& p, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = make_cfg(dim3(p.B * p.S), dim3(256), 0, s, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, embed_kernel, p);
+}
+
+// ------------------------------------------------------------------------ final
+// One CTA per action row: norm in fp32, v = W_out y + b_out (fp32), x += dt * v.
+__global__ void __launch_bounds__(256) final_kernel(const FinalParams p) {
+  extern __shared__ float y[];   // [W]
+  __shared__ float red[8];
+  if (threadIdx.x == 0) pdl_trigger();
+  pdl_wait();
+  const int bc = blockIdx.x;
+  const int b = bc / p.C, c = bc - b * p.C;
+  const float* xr = p.resid + (static_cast<size_t>(b) * p.S + p.has_state + c) * p.W;
+  float ss = 0.0f;
+  for (int i = threadIdx.x; i < p.W; i += blockDim.x) {
+    const float v = xr[i];
+    y[i] = v;
+    ss += v * v;
+  }
+  ss = warp_sum(ss);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += red[i];
+  const float r = 1.0f / sqrtf(tot / static_cast<float>(p.W) + p.eps);
+  for (int i = threadIdx.x; i < p.W; i += blockDim.x) {
+    const float n = y[i] * r;
+    y[i] = p.scale ? fmaf(n, 1.0f + p.scale[i], p.shift[i]) : n * (1.0f + p.w[i]);
+  }
+  __syncthreads();
+  for (int a = warp; a < p.A; a += 8) {
+    const float* wr = p.w_out + static_cast<size_t>(a) * p.W;
+    float acc = 0.0f;
+    for (int i = lane; i < p.W; i += 32) acc = fmaf(wr[i], y[i], acc);
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      float* xo = p.x + (static_cast<size_t>(b) * p.C + c) * p.A + a;
+      *xo = fmaf(p.dt, acc + p.b_out[a], *xo);
+    }
+  }
+}
+
+cudaError_t launch_final(const FinalParams& p, cudaStream_t s, bool pdl) {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg =
+      make_cfg(dim3(p.B * p.C), dim3(256), static_cast<size_t>(p.W) * sizeof(float), s, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, final_kernel, p);
+}
+
+// ------------------------------------------------------------------- time tables
+// t_k = 1 - k/steps; sinusoidal embedding with periods 4e-3 .. 4, sin half first.
+__global__ void temb_kernel(float* temb, int steps, int dim) {
+  const int k = blockIdx.x;
+  const int half = dim / 2;
+  const double t = 1.0 - static_cast<double>(k) / steps;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double frac = static_cast<double>(i) / (half - 1);
+    const double period = 4e-3 * pow(4.0 / 4e-3, frac);
+    const double ang = 2.0 * 3.14159265358979323846 * t / period;
+    temb[static_cast<size_t>(k) * dim + i] = static_cast<float>(sin(ang));
+    temb[static_cast<size_t>(k) * dim + half + i] = static_cast<float>(cos(ang));
+  }
+}
+
+cudaError_t launch_temb(float* temb, int steps, int time_dim, cudaStream_t s) {
+  temb_kernel<<<steps, 128, 0, s>>>(temb, steps, time_dim);
+  return cudaGetLastError();
+}
+
+// One warp per output feature, 8 rows (time steps) at a time.
+__global__ void __launch_bounds__(256) rowgemv_kernel(const float* x, int rows, int n_in,
+                                                      const bf16* w, long ldw, const bf16* bvec,
+                                                      int n_out, float* y, int act_swish) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * 8 + warp;
+  if (o >= n_out) return;
+  const bf16* wr = w + static_cast<size_t>(o) * ldw;
+  const float bias = bvec ? __bfloat162float(bvec[o]) : 0.0f;
+  for (int r0 = 0; r0 < rows; r0 += 8) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    for (int i = lane; i < n_in; i += 32) {
+      const float wv = __bfloat162float(wr[i]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r0 + j < rows) acc[j] = fmaf(wv, x[static_cast<size_t>(r0 + j) * n_in + i], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float v = warp_sum(acc[j]) + bias;
+      if (lane == 0 && r0 + j < rows)
+        y[static_cast<size_t>(r0 + j) * n_out + o] = act_swish ? swishf(v) : v;
+    }
+  }
+}
+
+cudaError_t launch_rowgemv(const float* x, int rows, int n_in, const bf16* w, long ldw,
+                           const bf16* b, int n_out, float* y, int act_swish, cudaStream_t s) {
+  rowgemv_kernel<<<(n_out + 7) / 8, 256, 0, s>>>(x, rows, n_in, w, ldw, b, n_out, y, act_swish);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------- cache upkeep
+// K, V [L][batch][n][D] -> cache rows [0, n) of each (layer, observation): the static
+// region, then the ring slots 0.. (the ring starts right after the static capacity).
+__global__ void prefix_set_kernel(const uint4* K, const uint4* V, int n, int batch, int L, int D8,
+                                  int max_batch, int kcap, uint4* kc, uint4* vc) {
+  const size_t total = static_cast<size_t>(L) * batch * n * D8;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % D8);
+    size_t r = i / D8;
+    const int j = static_cast<int>(r % n);
+    r /= n;
+    const int b = static_cast<int>(r % batch);
+    const int l = static_cast<int>(r / batch);
+    const size_t dst = ((static_cast<size_t>(l) * max_batch + b) * kcap + j) * D8 + c;
+    kc[dst] = K[i];
+    vc[dst] = V[i];
+  }
+}
+
+cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L, int D,
+                              int max_batch, int kcap, int, bf16* kc, bf16* vc, cudaStream_t s) {
+  const size_t total = static_cast<size_t>(L) * batch * n_tokens * (D / 8);
+  if (total == 0) return cudaSuccess;
+  const int blocks = static_cast<int>((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
+  prefix_set_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(K),
+                                           reinterpret_cast<const uint4*>(V), n_tokens, batch, L,
+                                           D / 8, max_batch, kcap, reinterpret_cast<uint4*>(kc),
+                                           reinterpret_cast<uint4*>(vc));
+  return cudaGetLastError();
+}
+
+// One token of K/V per (layer, observation) into cache row slot_row.
+__global__ void ring_append_kernel(const uint4* K, const uint4* V, int batch, int L, int D8,
+                                   int max_batch, int kcap, int slot_row, uint4* kc, uint4* vc) {
+  const int total = L * batch * D8;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int c = i % D8, lb = i / D8;
+    const int b = lb % batch, l = lb / batch;
+    const size_t dst = ((static_cast<size_t>(l) * max_batch + b) * kcap + slot_row) * D8 + c;
+    kc[dst] = K[i];
+    vc[dst] = V[i];
+  }
+}
+
+cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, int D, int max_batch,
+                               int kcap, int slot_row, bf16* kc, bf16* vc, cudaStream_t s) {
+  const int total = L * batch * (D / 8);
+  const int blocks = (total + 255) / 256;
+  ring_append_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(K),
+                                            reinterpret_cast<const uint4*>(V), batch, L, D / 8,
+                                            max_batch, kcap, slot_row, reinterpret_cast<uint4*>(kc),
+                                            reinterpret_cast<uint4*>(vc));
+  return cudaGetLastError();
+}
+
+// Descriptor + rotary table [seq][D/2] of (cos, sin) at positions pos0 + s, in double.
+__global__ void cache_update_kernel(CacheDesc* desc, int n_static, int n_ring, float* rope, int seq,
+                                    int D, double base) {
+  const int pos0 = n_static + n_ring;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    desc->n_static = n_static;
+    desc->n_ring = n_ring;
+    desc->pos0 = pos0;
+  }
+  const int half = D / 2;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < seq * half; idx += gridDim.x * blockDim.x) {
+    const int s = idx / half, i = idx % half;
+    const double ang = static_cast<double>(pos0 + s) * pow(base, -2.0 * i / D);
+    rope[2 * idx] = static_cast<float>(cos(ang));
+    rope[2 * idx + 1] = static_cast<float>(sin(ang));
+  }
+}
+
+cudaError_t launch_cache_update(CacheDesc* desc, int n_static, int n_ring, float* rope, int seq,
+                                int head_dim, float rope_base, cudaStream_t s) {
+  const int n = seq * head_dim / 2;
+  cache_update_kernel<<<(n + 255) / 256, 256, 0, s>>>(desc, n_static, n_ring, rope, seq, head_dim,
+                                                       static_cast<double>(rope_base));
+  return cudaGetLastError();
+}
+
+__global__ void copy_region_kernel(const uint4* kc, uint4* out, int L, int batch, int max_batch,
+                                   int kcap, int rows, int D8) {
+  const size_t total = static_cast<size_t>(L) * batch * rows * D8;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % D8);
+    size_t r = i / D8;
+    const int j = static_cast<int>(r % rows);
+    r /= rows;
+    const int b = static_cast<int>(r % batch);
+    const int l = static_cast<int>(r / batch);
+    out[i] = kc[((static_cast<size_t>(l) * max_batch + b) * kcap + j) * D8 + c];
+  }
+}
+
+cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch, int kcap,
+                               int rows, int D, cudaStream_t s) {
+  const size_t total = static_cast<size_t>(L) * batch * rows * (D / 8);
+  if (total == 0) return cudaSuccess;
+  const int blocks = static_cast<int>((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
+  copy_region_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(kc),
+                                            reinterpret_cast<uint4*>(out), L, batch, max_batch, kcap,
+                                            rows, D / 8);
+  return cudaGetLastError();
+}
+
+}  // namespace vla

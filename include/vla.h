@@ -1,0 +1,255 @@
+/*
+ * vla.h -- C ABI of the B200 (sm_100a) flow-matching action-expert library.
+ *
+ * The library runs the denoise loop of a Pi0/Pi05-style vision-language-action policy:
+ * a transformer "action expert" over the action chunk (plus an optional state token)
+ * that attends to a cached perception/prompt prefix K/V, integrated with explicit Euler
+ * steps from noise (t = 1) to actions (t = 0).
+ *
+ * Sources of the operations (web pages on the subject):
+ *  - realtime-vla write-up (dexmal), "The problem is a policy that thinks too long":
+ *    three components (vision encoder, LLM, action expert), the graph flattened to
+ *    GEMM-like ops plus scalar ops; "The latency table, and what it assumes": 10 flow
+ *    steps, chunk 50; "Copying an inference file into your own project": forward(images,
+ *    state (32,), noise (traj_len, 32)).
+ *  - Reflex abstract: perception K/V is independent of the denoise loop and is reused;
+ *    static / sliding / dynamic partition of the attention context with O(1) updates;
+ *    AdaRMSNorm gated on flow phase; operator fusion.
+ *  - FlowEdge README, "Installation" (flow sampling with "euler 10") and "Overview"
+ *    (pre-sized arena, no allocation after warm-up).
+ *
+ * Conventions for every entry point:
+ *  - Return value: VLA_OK (0) or a vla_status error code. On error, vla_last_error()
+ *    returns a message for the calling thread; no state of the handle has changed
+ *    unless the message says so. Nothing is ever printed.
+ *  - bf16 values are passed as uint16_t bit patterns. Matrices are row-major
+ *    [out][in] ("K-major"); stacked per-layer tensors put the layer index first.
+ *  - "device" pointers are CUDA device (or managed) memory on the current device;
+ *    "host" pointers are ordinary host memory. The caller owns every buffer it passes
+ *    and may free it once the call (and, for stream-ordered calls, the stream work)
+ *    is done; the library never keeps a caller pointer.
+ *  - cuda_stream is a cudaStream_t (NULL = legacy default stream). Stream-ordered calls
+ *    return as soon as the work is enqueued.
+ *  - A handle is used by one host thread and one stream at a time (not thread-safe per
+ *    handle); distinct handles are independent.
+ */
+#ifndef VLA_H_
+#define VLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VLA_API __attribute__((visibility("default")))
+#else
+#define VLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vla_status {
+  VLA_OK = 0,
+  VLA_ERR_ARG = 1,          /* null pointer, bad enum, negative size */
+  VLA_ERR_SHAPE = 2,        /* a size exceeds the capacity set at create, or breaks a
+                               divisibility rule of the kernels */
+  VLA_ERR_STATE = 3,        /* call out of order (e.g. denoise before any prefix) */
+  VLA_ERR_OOM = 4,          /* device allocation failed during create */
+  VLA_ERR_CUDA = 5,         /* a CUDA runtime call failed; message has the CUDA error */
+  VLA_ERR_TIMEOUT = 6,      /* a bounded wait inside a kernel gave up (device status) */
+  VLA_ERR_UNSUPPORTED = 7   /* device is not sm_100 or a feature is not built */
+} vla_status;
+
+typedef enum vla_time_kind {
+  /* Pi0: time enters through an MLP over concat(action embedding, sin/cos t-emb):
+     h = Linear2(swish(Linear1([e ; temb]))); blocks use plain RMSNorm with (1 + w). */
+  VLA_TIME_PI0_MLP = 0,
+  /* AdaRMSNorm whose (scale, shift, gate) are a linear map of the raw t-emb. */
+  VLA_TIME_ADA_SINCOS = 1,
+  /* Pi05: AdaRMSNorm conditioned on cond = swish(L2(swish(L1(temb)))). */
+  VLA_TIME_ADA_MLP = 2
+} vla_time_kind;
+
+/* Option bits for vla_config.flags. */
+#define VLA_FLAG_NO_PDL 1u      /* launch without programmatic dependent launch edges */
+
+typedef struct vla_config {
+  int n_layers;      /* L */
+  int width;         /* W, multiple of 128 */
+  int n_heads;       /* H query heads */
+  int n_kv_heads;    /* must be 1 (all query heads share one K/V head, GQA) */
+  int head_dim;      /* D in {32, 64, 128, 256} */
+  int mlp_dim;       /* F, multiple of 64 (GeGLU hidden width) */
+  int action_dim;    /* A <= 64 */
+  int chunk;         /* C action tokens per observation */
+  int state_dim;     /* 0 = no state token; else the state vector width (<= 256) */
+  int time_kind;     /* vla_time_kind */
+  int time_dim;      /* width of the sinusoidal t-embedding (even, >= 4) */
+  int n_static_max;  /* capacity of the static prefix region (keys per layer per obs) */
+  int n_sliding;     /* ring slots of the sliding region (0 = none) */
+  int max_batch;     /* observations per call, upper bound */
+  int max_steps;     /* Euler steps per call, upper bound (<= 64) */
+  float eps;         /* RMSNorm epsilon (1e-6 in the shipped workloads) */
+  float rope_base;   /* RoPE base (10000) */
+  unsigned flags;    /* VLA_FLAG_* */
+} vla_config;
+
+/*
+ * Parameters, all HOST pointers to bf16 bit patterns, copied (and repacked) by
+ * vla_expert_create. Shapes ([out][in] matrices; L layers stacked first):
+ *   action_in_w [W][A], action_in_b [W], action_out_w [A][W], action_out_b [A]
+ *   wq [L][H*D][W], wk [L][D][W], wv [L][D][W], wo [L][W][H*D]
+ *   w_gate [L][F][W], w_up [L][F][W], w_down [L][W][F]
+ *   state_dim > 0:      state_in_w [W][state_dim], state_in_b [W]
+ *   VLA_TIME_PI0_MLP:   time_mlp_in_w [W][W + time_dim] (action half first),
+ *                       time_mlp_in_b [W], time_mlp_out_w [W][W], time_mlp_out_b [W],
+ *                       norm1_w [L][W], norm2_w [L][W], final_norm_w [W]
+ *   VLA_TIME_ADA_MLP:   time_cond1_w [W][time_dim], time_cond1_b [W],
+ *                       time_cond2_w [W][W], time_cond2_b [W]
+ *   VLA_TIME_ADA_*:     norm1_mod_w [L][3W][Cd], norm1_mod_b [L][3W], norm2_mod_w,
+ *                       norm2_mod_b (same), final_norm_mod_w [3W][Cd],
+ *                       final_norm_mod_b [3W]; Cd = W (ADA_MLP) or time_dim (ADA_SINCOS);
+ *                       the 3W outputs split as [scale | shift | gate].
+ * Pointers a configuration does not use may be NULL.
+ */
+typedef struct vla_weights {
+  const uint16_t *action_in_w, *action_in_b, *action_out_w, *action_out_b;
+  const uint16_t *state_in_w, *state_in_b;
+  const uint16_t *time_mlp_in_w, *time_mlp_in_b, *time_mlp_out_w, *time_mlp_out_b;
+  const uint16_t *time_cond1_w, *time_cond1_b, *time_cond2_w, *time_cond2_b;
+  const uint16_t *norm1_w, *norm2_w, *final_norm_w;
+  const uint16_t *norm1_mod_w, *norm1_mod_b, *norm2_mod_w, *norm2_mod_b;
+  const uint16_t *final_norm_mod_w, *final_norm_mod_b;
+  const uint16_t *wq, *wk, *wv, *wo, *w_gate, *w_up, *w_down;
+} vla_weights;
+
+typedef struct vla_expert vla_expert;   /* opaque, owned by the library */
+
+/*
+ * vla_expert_create -- validate cfg, allocate every device buffer for cfg->max_batch
+ * observations (weights, the K/V cache regions, activations, time tables, split
+ * workspaces: nothing is allocated after this call, FlowEdge's "warmup (malloc 0)"),
+ * copy and repack the weights, and compute the time tables for cfg->max_steps steps.
+ * Synchronous on the current device. *out receives the handle.
+ * Errors: VLA_ERR_ARG (null), VLA_ERR_SHAPE (sizes break the rules in vla_config),
+ * VLA_ERR_UNSUPPORTED (device is not compute capability 10.0), VLA_ERR_OOM, VLA_ERR_CUDA.
+ */
+VLA_API int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** out);
+
+/* vla_expert_destroy -- synchronize the device, free everything. NULL is a no-op. */
+VLA_API void vla_expert_destroy(vla_expert* h);
+
+/*
+ * vla_cache_set_prefix -- load the cached context K/V (Reflex abstract: the perception
+ * and prompt K/V do not depend on the denoise loop, so they are computed once and
+ * reused by every Euler step). K and V are DEVICE bf16 [L][batch][n_tokens][D], keys
+ * already rotated by RoPE. The first min(n_tokens, n_static_max) tokens fill the static
+ * region; the remaining n_tokens - n_static_max (at most n_sliding) fill ring slots
+ * 0.. in order, and the ring head is set to the next slot. Suffix RoPE positions become
+ * n_static + n_ring. Stream-ordered. Errors: VLA_ERR_ARG, VLA_ERR_SHAPE
+ * (batch > max_batch, n_tokens < 0 or > n_static_max + n_sliding).
+ */
+VLA_API int vla_cache_set_prefix(vla_expert* h, const uint16_t* K, const uint16_t* V, int n_tokens,
+                         int batch, void* cuda_stream);
+
+/*
+ * vla_cache_append_sliding -- O(1) update of the sliding region (Reflex abstract): the
+ * DEVICE bf16 K_tok, V_tok [L][batch][D] of one new token overwrite ring slot `head`
+ * (the oldest entry once the ring is full) in every layer, and head advances by one
+ * modulo n_sliding. Only the 2 * L * batch * D values are written (a bit copy).
+ * Stream-ordered. Errors: VLA_ERR_STATE (no sliding region, or no prefix set),
+ * VLA_ERR_SHAPE (batch > max_batch or batch differs from the prefix batch), VLA_ERR_ARG.
+ */
+VLA_API int vla_cache_append_sliding(vla_expert* h, const uint16_t* K_tok, const uint16_t* V_tok,
+                             int batch, void* cuda_stream);
+
+/*
+ * vla_denoise -- the hot path: `steps` explicit Euler steps x <- x + dt * v(x, t),
+ * t_k = 1 - k/steps, dt = -1/steps, from x = noise to out_actions, every step running
+ * the action expert over the suffix tokens against the cached prefix.
+ * noise: DEVICE fp32 [batch][C][A] (not modified); state: DEVICE fp32
+ * [batch][state_dim], required iff state_dim > 0, else ignored; out_actions: DEVICE
+ * fp32 [batch][C][A], must not overlap noise. The first call for a (batch, steps) pair
+ * captures a CUDA graph of the whole loop; later calls replay it. Stream-ordered.
+ * Errors: VLA_ERR_ARG, VLA_ERR_SHAPE (batch or steps out of range), VLA_ERR_STATE (no
+ * prefix set, or prefix batch < batch), VLA_ERR_CUDA.
+ */
+VLA_API int vla_denoise(vla_expert* h, const float* noise, const float* state, int steps,
+                float* out_actions, int batch, void* cuda_stream);
+
+/*
+ * vla_denoise_host -- vla_denoise on HOST buffers with the same shapes: copies noise and
+ * state to the device on cuda_stream, runs the loop, copies the actions back and
+ * synchronizes the stream before returning (so out_actions is ready on return).
+ */
+VLA_API int vla_denoise_host(vla_expert* h, const float* noise, const float* state, int steps,
+                     float* out_actions, int batch, void* cuda_stream);
+
+/*
+ * vla_cache_export -- copy the static and sliding regions, DEVICE bf16
+ * [L][batch][n_static_max + n_sliding][D] each (ring slots in physical order, stale or
+ * never-written slots included), into caller buffers, and write the ring head and the
+ * valid counts to the HOST ints (any may be NULL). Stream-ordered. For tests and tools.
+ */
+VLA_API int vla_cache_export(vla_expert* h, uint16_t* K_out, uint16_t* V_out, int batch,
+                     int* head, int* n_static, int* n_ring, void* cuda_stream);
+
+/*
+ * vla_device_status -- synchronize cuda_stream and read the handle's device status word,
+ * which kernels set instead of trapping when a bounded wait gives up. Returns VLA_OK,
+ * VLA_ERR_TIMEOUT (status word set; it is then cleared) or VLA_ERR_CUDA.
+ */
+VLA_API int vla_device_status(vla_expert* h, void* cuda_stream);
+
+/* Kinds of kernels, for vla_profile_kernels. */
+typedef enum vla_kernel_kind {
+  VLA_K_GEMM_QKV = 0, VLA_K_ATTN = 1, VLA_K_GEMM_O = 2, VLA_K_GEMM_GATEUP = 3,
+  VLA_K_GEMM_DOWN = 4, VLA_K_NORM = 5, VLA_K_EMBED = 6, VLA_K_FINAL = 7,
+  VLA_K_TIME_MLP = 8, VLA_K_COUNT = 9
+} vla_kernel_kind;
+
+typedef struct vla_kernel_times {
+  float total_ms[VLA_K_COUNT];   /* summed device time of each kind over one denoise */
+  int launches[VLA_K_COUNT];     /* launches of each kind in one denoise */
+  double bytes[VLA_K_COUNT];     /* algorithmic DRAM bytes of each kind in one denoise */
+  double flops[VLA_K_COUNT];     /* algorithmic FLOPs (2 x MAC) of each kind */
+} vla_kernel_times;
+
+/*
+ * vla_profile_kernels -- run one denoise of the same (batch, steps) as vla_denoise, from
+ * a second graph that brackets every kernel with CUDA event records, and fill *times
+ * (host struct) with per-kind device time, launch counts and the algorithmic byte and
+ * FLOP counts. Synchronizes the stream. The events serialise the kernels, so use it for
+ * per-kernel shares, not for the end-to-end time.
+ */
+VLA_API int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, int steps,
+                        float* out_actions, int batch, vla_kernel_times* times,
+                        void* cuda_stream);
+
+/*
+ * vla_gemm_bf16 -- one launch of the library's tensor-core projection kernel on its own
+ * (the kernel behind every dense projection of vla_denoise; realtime-vla write-up: the
+ * expert reduces to GEMM-like ops), with a plain fp32 store epilogue:
+ *     Y[m][n] = sum_k X[m][k] * W[n][k],  m < m_tok, n < n_feat.
+ * W: DEVICE bf16 [n_feat][k_dim]; X: DEVICE bf16 [m_tok][k_dim]; Y: DEVICE fp32
+ * [m_tok][n_feat] (overwritten). n_feat % 128 == 0, k_dim % 64 == 0, m_tok >= 1; W and
+ * X 16-byte aligned. split_k = 0 picks the split-K factor the denoise loop would use;
+ * split_k > 0 forces (at most) that many K splits. The split-K partial tiles live in a
+ * workspace this call allocates and frees stream-ordered (cudaMallocAsync / cudaFreeAsync).
+ * Stream-ordered. Errors: VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_UNSUPPORTED, VLA_ERR_CUDA.
+ */
+VLA_API int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim,
+                          int m_tok, int split_k, void* cuda_stream);
+
+/* Message of the last failed call on this thread ("" if none). Valid until the next call. */
+VLA_API const char* vla_last_error(void);
+
+/* Library version string. */
+VLA_API const char* vla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VLA_H_ */

@@ -1,0 +1,120 @@
+"""The CUDA denoise path (through the C ABI) against the fp64 oracle on the same seeded
+inputs, element by element, for every workload shape; plus the exact special cases."""
+import numpy as np
+import pytest
+
+from tests._helpers import (check_actions, get, golden_actions, load_prefix, make_expert,
+                            make_inputs, oracle_actions, run)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid_pi0_b3", "mid_ada_b2", "mid_d128"])
+def test_small_workloads_match_oracle(name):
+    wl = get(name)
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    check_actions(got, golden_actions(name), name)
+    ex.device_status()
+
+
+@pytest.mark.parametrize("name", ["pi0_1view", "pi05_3view"])
+def test_full_size_batch1_matches_oracle(name):
+    wl = get(name)
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    check_actions(got, oracle_actions(wl, inp), name)
+    ex.device_status()
+
+
+def test_batch64_sampled_observations_match_oracle():
+    """64 independent observations in one call; the oracle checks a sample of them."""
+    wl = get("pi05_3view_b64")
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    idx = [0, 37, 63]
+    check_actions(got[idx], oracle_actions(wl, inp, batch_idx=idx), "b64 sample")
+    assert np.all(np.isfinite(got))
+    ex.device_status()
+
+
+def test_zero_velocity_is_bit_exact():
+    """v == 0 (zero action projection) leaves the noise untouched: x + dt * 0 == x."""
+    wl = get("mid_ada_b2")
+    inp = make_inputs(wl)
+    inp["params"]["action_out.w"][:] = 0
+    inp["params"]["action_out.b"][:] = 0
+    ex, _ = make_expert(wl, inp)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    assert np.array_equal(got.astype(np.float32), inp["noise"])
+
+
+def test_repeat_calls_are_bit_identical_and_pdl_free_equal():
+    import flow_matching_vla_euler_b200 as V
+    wl = get("mid_pi0_b3")
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    a = run(ex, inp, wl.steps)
+    b = run(ex, inp, wl.steps)
+    assert np.array_equal(a, b)
+    ex2, _ = make_expert(wl, inp, flags=V.VLA_FLAG_NO_PDL)
+    load_prefix(ex2, inp)
+    c = run(ex2, inp, wl.steps)
+    assert np.array_equal(a, c)
+
+
+def test_batch_rows_match_single_observation_runs():
+    wl = get("mid_ada_b2")
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    full = run(ex, inp, wl.steps)
+    for b in range(wl.batch):
+        one = {k: v for k, v in inp.items()}
+        one["noise"] = inp["noise"][b:b + 1]
+        one["prefix_k"] = inp["prefix_k"][:, b:b + 1]
+        one["prefix_v"] = inp["prefix_v"][:, b:b + 1]
+        load_prefix(ex, one)
+        got = run(ex, one, wl.steps)
+        np.testing.assert_allclose(got[0], full[b], rtol=0, atol=2e-3)
+
+
+def test_step_counts_and_host_entry_point():
+    """Other step counts use their own time tables; vla_denoise_host equals vla_denoise."""
+    wl = get("mid_ada_b2")
+    ex, inp = make_expert(wl, max_steps=8)
+    load_prefix(ex, inp)
+    for steps in (1, 2, 4, 8):
+        got = run(ex, inp, steps)
+        from dataclasses import replace
+        ref = oracle_actions(replace(wl, steps=steps), inp)
+        check_actions(got, ref, f"steps={steps}")
+    host = ex.denoise_host(inp["noise"], inp["state"], 4).astype(np.float64)
+    assert np.array_equal(host, run(ex, inp, 4))
+
+
+def test_error_paths_on_device():
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    wl = get("tiny")
+    ex, inp = make_expert(wl)
+    noise = torch.from_numpy(inp["noise"]).cuda()
+    state = torch.from_numpy(inp["state"]).cuda()
+    with pytest.raises(V.VlaError) as e:
+        ex.denoise(noise, state, 4)
+    assert e.value.code == V.VLA_ERR_STATE
+    load_prefix(ex, inp)
+    with pytest.raises(V.VlaError) as e:
+        ex.denoise(noise, state, 5)          # beyond max_steps
+    assert e.value.code == V.VLA_ERR_SHAPE
+    with pytest.raises(V.VlaError) as e:
+        ex.denoise(noise, None, 4)           # state required
+    assert e.value.code == V.VLA_ERR_ARG
+    kt = torch.zeros((wl.expert.n_layers, 1, wl.expert.head_dim), dtype=torch.int16, device="cuda")
+    with pytest.raises(V.VlaError) as e:
+        ex.append_sliding(kt, kt)            # no sliding region
+    assert e.value.code == V.VLA_ERR_STATE
+    ex.device_status()
