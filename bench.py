@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the flow-matching action-expert denoise loop on B200.
+
+One "step" is one whole denoise: N = 10 Euler steps of the Pi05-style expert (18 layers,
+width 1024, 8 query heads over one 256-d K/V head, GeGLU 4096) over a 50-action chunk,
+attending to a 788-key cached prefix (3 views x 256 image tokens + 20 prompt tokens), at
+batch 1 -- the workload the pages time end to end (realtime-vla write-up, "The latency
+table, and what it assumes": 10 flow steps, chunk 50, 3 views, 20-token prompt). The
+same expert at batch 64 is reported as a secondary line (chunks/s, tensor-core bound).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0. Multi-GPU (torchrun, one process per GPU): every rank
+runs an independent replica (the path has no cross-observation exchange), timing is the
+max over ranks, and the value is whole-job ms per denoise.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms per 10-step chunk-50 denoise (batch 1) & chunks/s @batch 64; % HBM/TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="pi05_3view")
+    p.add_argument("--secondary", default="pi05_3view_b64")
+    p.add_argument("--secondary-steps", type=int, default=40)
+    p.add_argument("--no-secondary", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-profile", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "gemm": ["flow_matching_vla_euler_b200/csrc/gemm_tc.cu", "flow_matching_vla_euler_b200/csrc/ptx.cuh",
+             "flow_matching_vla_euler_b200/csrc/kernels.h"],
+    "attention": ["flow_matching_vla_euler_b200/csrc/attention.cu", "flow_matching_vla_euler_b200/csrc/ptx.cuh",
+                  "flow_matching_vla_euler_b200/csrc/kernels.h"],
+}
+
+
+def ncu_traffic(kind: str, workload: str):
+    """DRAM bytes per launch of `kind` on `workload` from a committed ncu summary, or None
+    when no capture exists or the kernel source changed since it was taken. Summary lines:
+    ``traffic <kind> <workload> <source_sha> <bytes_per_launch>``."""
+    fam = "attention" if kind == "attention" else "gemm"
+    want = source_sha(KERNEL_SOURCES[fam])
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
+        return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(pdir, fn)) as f:
+            for line in f:
+                m = re.match(r"^\s*traffic\s+(\S+)\s+(\S+)\s+(\S+)\s+([0-9.eE+]+)\s*$", line)
+                if m and m.group(1) == kind and m.group(2) == workload and m.group(3) == want:
+                    return float(m.group(4))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, enabled: bool = True):
+        self.index, self.enabled, self.proc = index, enabled, None
+
+    def __enter__(self):
+        if self.enabled:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                     "-lms", "200"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            except OSError:
+                self.proc = None
+            time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            rows = [r for r in csv.reader(f) if len(r) >= 9]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int, device=None) -> float:
+    """Largest value of x over all ranks (all-reduce MAX); x itself at one rank."""
+    if ws <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    if device is None:
+        device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- workload set-up
+
+def build_expert(wl, inp):
+    import numpy as np
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    ex = V.Expert(wl.expert, inp["params"], n_static_max=wl.n_static, n_sliding=wl.n_sliding,
+                  max_batch=wl.batch, max_steps=wl.steps)
+    bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+    ex.set_prefix(bits(inp["prefix_k"]), bits(inp["prefix_v"]))
+    noise = torch.from_numpy(inp["noise"]).cuda()
+    state = None if inp["state"] is None else torch.from_numpy(inp["state"]).cuda()
+    return ex, noise, state
+
+
+def time_device(ex, noise, state, steps, K, W, ws):
+    """K denoises back to back on the current stream, CUDA events, max over ranks."""
+    import torch
+    out = torch.empty_like(noise)
+    for _ in range(W):
+        ex.denoise(noise, state, steps, out)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    ev[0].record(s)
+    for i in range(K):
+        ex.denoise(noise, state, steps, out)
+        ev[i + 1].record(s)
+    torch.cuda.synchronize()
+    barrier(ws)
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+    total = ev[0].elapsed_time(ev[K])
+    return total, per, out
+
+
+def time_e2e(ex, inp, steps, K, W, ws):
+    """Same metric through vla_denoise_host: pinned host noise/state in, actions out,
+    host<->device copies inside the timed region every step."""
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    noise = torch.from_numpy(inp["noise"]).pin_memory()
+    state = None if inp["state"] is None else torch.from_numpy(inp["state"]).pin_memory()
+    out = torch.empty_like(noise).pin_memory()
+    B = noise.shape[0]
+    sp = None if state is None else state.data_ptr()
+    stream = torch.cuda.current_stream().cuda_stream
+    for _ in range(W):
+        V.vla_denoise_host(ex.handle, noise.data_ptr(), sp, steps, out.data_ptr(), B, stream)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(K):
+        V.vla_denoise_host(ex.handle, noise.data_ptr(), sp, steps, out.data_ptr(), B, stream)
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(ws)
+    h2d = noise.numel() * 4 + (0 if state is None else state.numel() * 4)
+    return e0.elapsed_time(e1), h2d, out.numel() * 4
+
+
+def roofline(ex, noise, state, steps, peaks, peak_src, workload, bound, reps=3):
+    """Per-kernel device time from event-bracketed launches (vla_profile_kernels) on the
+    launching stream; the dominant kernel's algorithmic bytes (or FLOPs) per launch over
+    its mean launch duration."""
+    prof = None
+    acc = {}
+    for _ in range(reps):
+        _, prof = ex.profile_kernels(noise, state, steps)
+        for k, v in prof.items():
+            a = acc.setdefault(k, {"ms": 0.0, "launches": 0, "bytes": v["bytes"], "flops": v["flops"]})
+            a["ms"] += v["ms"] / reps
+            a["launches"] = v["launches"]
+    dom = max(acc, key=lambda k: acc[k]["ms"])
+    d = acc[dom]
+    per_launch_ms = d["ms"] / max(1, d["launches"])
+    shares = {k: round(v["ms"] / sum(x["ms"] for x in acc.values()), 4) for k, v in acc.items() if v["ms"] > 0}
+    if bound == "hbm":
+        achieved = d["bytes"] / max(1, d["launches"]) / (per_launch_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = d["flops"] / max(1, d["launches"]) / (per_launch_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    tr = ncu_traffic(dom, workload)
+    return {"kernel": dom, "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": tr,
+            "algorithmic_per_launch": d["bytes"] / max(1, d["launches"]) if bound == "hbm"
+            else d["flops"] / max(1, d["launches"]),
+            "mean_launch_us": round(per_launch_ms * 1e3, 2), "launches_per_denoise": d["launches"],
+            "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+            "time_shares": shares}, acc
+
+
+class OracleRunner:
+    """The fp64 oracle as it stands, on the host cores. Inputs are widened once; each
+    call times `euler_steps` Euler steps (expert velocity + update) of `n_obs`
+    observations."""
+
+    def __init__(self, wl, inp, n_obs=1):
+        import numpy as np
+        import oracle as O
+        self.O, self.wl, self.n_obs = O, wl, n_obs
+        self.P = O.decode_params(inp["params"])
+        self.pk = O.bf16_to_f64(inp["prefix_k"][:, :n_obs])
+        self.pv = O.bf16_to_f64(inp["prefix_v"][:, :n_obs])
+        self.noise = inp["noise"][:n_obs].astype(np.float64)
+        self.st = None if inp["state"] is None else inp["state"][:n_obs].astype(np.float64)
+
+    def ms(self, euler_steps=None):
+        steps = self.wl.steps
+        n = steps if euler_steps is None else euler_steps
+        t0 = time.perf_counter()
+        for b in range(self.n_obs):
+            x = self.noise[b]
+            for k in range(n):
+                t = 1.0 - k / steps
+                v = self.O.expert_velocity(self.wl.expert, self.P, x, t,
+                                           None if self.st is None else self.st[b],
+                                           self.pk[:, b], self.pv[:, b])
+                x = x + (-1.0 / steps) * v
+        return (time.perf_counter() - t0) * 1e3
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [os.cpu_count()])
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    """The oracle on the host cores, on this arm's config and metric: each timed step is
+    a bounded sample (one Euler step of the batch-1 denoise), scaled to ms per denoise."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from vla_inputs import get, make_inputs
+    wl = get(args.workload)
+    inp = make_inputs(wl)
+    runner = OracleRunner(wl, inp, 1)
+    for _ in range(min(args.warmup, 1)):
+        runner.ms(1)
+    est = runner.ms(1)
+    k = max(1, min(args.steps, int(150_000 / max(est, 1.0))))
+    samples = [runner.ms(1) for _ in range(k)]
+    per_step = statistics.mean(samples)
+    value = per_step * wl.steps
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "ms",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(value, 3), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "euler_steps": wl.steps,
+                       "chunk": wl.expert.chunk, "cached_keys": wl.n_cached},
+            "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": cores, "kind": "oracle",
+                             "sample": f"{k} timed samples of one Euler step (expert velocity + update) "
+                                       f"of the batch-1 denoise, mean x {wl.steps} steps"},
+            "e2e": {"value": round(value, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    from vla_inputs import get, make_inputs
+    ws, rank, local = dist_setup(args)
+    peaks, peak_src = load_peaks()
+    wl = get(args.workload)
+    inp = make_inputs(wl, seed=wl.seed + rank)
+    ex, noise, state = build_expert(wl, inp)
+    steps = wl.steps
+    with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clk:
+        total_ms, per, _ = time_device(ex, noise, state, steps, args.steps, args.warmup, ws)
+    clocks = clk.summary()
+    ex.device_status()
+    t_max = max_over_ranks(total_ms, ws)
+    ms_per_step = t_max / args.steps
+    value = t_max / (args.steps * ws)
+    e2e = None
+    if not args.no_e2e:
+        k_e = max(10, args.steps // 4)
+        e_ms, h2d, d2h = time_e2e(ex, inp, steps, k_e, 3, ws)
+        e_ms = max_over_ranks(e_ms, ws)
+        e2e = {"value": round(e_ms / (k_e * ws), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": k_e}
+    roof, acc = (None, None)
+    if not args.no_profile:
+        roof, acc = roofline(ex, noise, state, steps, peaks, peak_src, wl.name, "hbm")
+    launches_per_denoise = sum(v["launches"] for v in acc.values()) if acc else None
+    # whole-denoise roofline: weights once per Euler step + K/V reads, at measured HBM rate
+    bytes_denoise = sum(v["bytes"] for v in acc.values()) if acc else None
+    ex.close()
+    del ex
+    torch.cuda.empty_cache()
+
+    secondary = None
+    if not args.no_secondary:
+        wl2 = get(args.secondary)
+        inp2 = make_inputs(wl2, seed=wl2.seed + rank)
+        ex2, n2, s2 = build_expert(wl2, inp2)
+        k2 = args.secondary_steps
+        t2, per2, _ = time_device(ex2, n2, s2, wl2.steps, k2, min(args.warmup, 5), ws)
+        ex2.device_status()
+        t2 = max_over_ranks(t2, ws)
+        ms2 = t2 / k2
+        r2 = None
+        if not args.no_profile:
+            r2, acc2 = roofline(ex2, n2, s2, wl2.steps, peaks, peak_src, wl2.name, "tensor", reps=1)
+            fl = sum(v["flops"] for v in acc2.values())
+            r2["denoise_tflops_achieved"] = round(fl / (ms2 * 1e-3) / 1e12, 1)
+            r2["denoise_frac_of_burst_peak"] = round(fl / (ms2 * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)
+        secondary = {"workload": wl2.name, "metric": "chunks/s @batch 64", "unit": "chunks/s",
+                     "value": round(wl2.batch * k2 * ws / (t2 * 1e-3), 1),
+                     "ms_per_denoise": round(ms2, 3), "steps": k2, "roofline": r2}
+        ex2.close()
+        del ex2
+        del inp2
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        ms_cpu = OracleRunner(wl, inp, 1).ms()
+        cpu = {"value": round(ms_cpu, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"one full {wl.steps}-step denoise of one observation of {wl.name} "
+                         f"(fp64 numpy, BLAS on all host cores)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "ms", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "euler_steps": steps,
+                       "chunk": wl.expert.chunk, "action_dim": wl.expert.action_dim,
+                       "layers": wl.expert.n_layers, "width": wl.expert.width, "mlp": wl.expert.mlp_dim,
+                       "heads": f"{wl.expert.n_heads}q/{wl.expert.n_kv_heads}kv x {wl.expert.head_dim}",
+                       "cached_keys": wl.n_cached, "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                       "l2": "inputs larger than L2: 623 MB of weights streamed per Euler step"},
+            "latency_ms": {"median": round(statistics.median(per), 4),
+                           "p10": round(float(np.percentile(per, 10)), 4),
+                           "p90": round(float(np.percentile(per, 90)), 4)},
+            "roofline": roof,
+            "denoise_roofline": None if bytes_denoise is None else {
+                "algorithmic_bytes": bytes_denoise,
+                "roofline_ms": round(bytes_denoise / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
+                "frac": round(bytes_denoise / (peaks["hbm_gbs"] * 1e9) * 1e3 / ms_per_step, 4),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": peak_src},
+            "secondary": secondary,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": None if launches_per_denoise is None else launches_per_denoise * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        barrier(ws)
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -7,8 +7,8 @@ from collections import deque
 import numpy as np
 import pytest
 
-from tests._helpers import (check_actions, get, make_expert, make_inputs, oracle_actions, run,
-                            to_cuda_bits)
+from tests._helpers import (MAX_ABS, MEAN_ABS, check_actions, get, make_expert, make_inputs,
+                            oracle_actions, run, to_cuda_bits)
 from vla_inputs import make_ring_token
 
 pytestmark = pytest.mark.gpu
@@ -55,9 +55,13 @@ def _stream(name, ticks, oracle_ticks):
         lv = np.concatenate([pv[:, :, :ns], np.stack(list(ring_v), axis=2)], axis=2)
         full.set_prefix(to_cuda_bits(lk), to_cuda_bits(lv))
         ref = run(full, inp, wl.steps)
-        d = float(np.abs(got - ref).max())
+        # both sides approximate the same exact value (keys summed in a different order),
+        # so they must agree within the acceptance tolerance used against the oracle
+        diff = np.abs(got - ref)
+        d = float(diff.max())
         worst = max(worst, d)
-        assert d <= 2e-3, f"tick {tick}: incremental vs recompute {d:.3e}"
+        assert d <= MAX_ABS and float(diff.mean()) <= MEAN_ABS, \
+            f"tick {tick}: incremental vs recompute max {d:.3e} mean {float(diff.mean()):.3e}"
         if tick in oracle_ticks:
             check_actions(got, oracle_actions(wl, inp, prefix_k=lk, prefix_v=lv), f"tick {tick}")
     ex.device_status()
