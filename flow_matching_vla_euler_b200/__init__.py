@@ -75,6 +75,7 @@ _SIGNATURES = {
     "vla_device_status": (_I, [_P, _P]),
     "vla_profile_kernels": (_I, [_P, _P, _P, _I, _P, _I, ctypes.POINTER(vla_kernel_times), _P]),
     "vla_gemm_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "vla_gemm_bf16_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "vla_last_error": (ctypes.c_char_p, []),
     "vla_version": (ctypes.c_char_p, []),
 }
@@ -156,6 +157,11 @@ def vla_profile_kernels(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream) 
 
 def vla_gemm_bf16(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, stream):
     _check(load_library().vla_gemm_bf16(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, stream))
+
+
+def vla_gemm_bf16_noalloc(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, stream):
+    _check(load_library().vla_gemm_bf16_noalloc(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k,
+                                                stream))
 
 
 def gemm(W, X, split_k: int = 0):

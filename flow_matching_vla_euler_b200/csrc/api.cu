@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -1028,3 +1029,92 @@ int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free variant of vla_gemm_bf16 for callers that may not allocate device
+// memory while they run. Its scratch is this one static array: split-K partial tiles
+// (8 MiB) followed by 4096 ints (tile arrival counters, then the status word).
+namespace {
+
+constexpr size_t kNoAllocPartialBytes = size_t(8) << 20;
+constexpr int kNoAllocCounters = 4096;   // 4095 tile counters + 1 status word
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartialBytes / 4 + kNoAllocCounters];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on device `dev` (which is current). In host code
+// the array's name is only a host-side handle, so the address is looked up once per
+// device and cached.
+int noalloc_scratch(int dev, float** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(VLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(VLA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
+    g_noalloc_addr[dev] = p;
+  }
+  *out = static_cast<float*>(g_noalloc_addr[dev]);
+  return VLA_OK;
+}
+
+}  // namespace
+
+extern "C" int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim,
+                                     int m_tok, int split_k, void* cuda_stream) {
+  g_err.clear();
+  if (!W || !X || !Y) return fail(VLA_ERR_ARG, "null W, X or Y");
+  if (n_feat < 128 || n_feat % 128 || k_dim < 64 || k_dim % 64 || m_tok < 1)
+    return fail(VLA_ERR_SHAPE, "need n_feat %% 128 == 0, k_dim %% 64 == 0, m_tok >= 1 (got %d, %d, %d)", n_feat,
+                k_dim, m_tok);
+  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(X)) & 15)
+    return fail(VLA_ERR_ARG, "W and X must be 16-byte aligned");
+  if (split_k < 0) return fail(VLA_ERR_ARG, "split_k must be >= 0");
+  int dev = 0, major = 0, sms = 148;
+  CU(cudaGetDevice(&dev));
+  CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  if (major != 10) return fail(VLA_ERR_UNSUPPORTED, "device is sm_%d0; this library is built for sm_100a", major);
+  CU(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  GemmPlan g = plan_gemm(n_feat, k_dim, m_tok, sms);
+  if (split_k > 0) {
+    const int nkb = k_dim / 64;
+    g.kb_per_split = cdiv(nkb, std::min(split_k, nkb));
+    g.splits = cdiv(nkb, g.kb_per_split);
+  }
+  const size_t tiles = static_cast<size_t>(g.n_tiles) * g.m_tiles;
+  const size_t need = g.splits > 1 ? tiles * g.splits * g.tn * 128 * sizeof(float) : 0;
+  if (need > kNoAllocPartialBytes || tiles > static_cast<size_t>(kNoAllocCounters - 1))
+    return fail(VLA_ERR_SHAPE,
+                "vla_gemm_bf16_noalloc: this shape needs %zu bytes of split-K scratch and %zu tile counters; "
+                "the static scratch holds %zu bytes and %d counters (use vla_gemm_bf16, or a smaller split_k)",
+                need, tiles, kNoAllocPartialBytes, kNoAllocCounters - 1);
+  float* scratch = nullptr;
+  int rc = noalloc_scratch(dev, &scratch);
+  if (rc) return rc;
+  CU(configure_gemm_kernels());
+  CUtensorMap tw, tx;
+  if ((rc = make_tmap(&tw, W, k_dim, n_feat, 128))) return rc;
+  if ((rc = make_tmap(&tx, X, k_dim, m_tok, g.tn))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  int* ctr = reinterpret_cast<int*>(scratch + kNoAllocPartialBytes / 4);
+  // counters and the status word must start at zero; the partial tiles are overwritten
+  CU(cudaMemsetAsync(ctr, 0, kNoAllocCounters * sizeof(int), s));
+  GemmParams p{};
+  p.n_feat = n_feat;
+  p.k_dim = k_dim;
+  p.m_tok = m_tok;
+  p.splits = g.splits;
+  p.kb_per_split = g.kb_per_split;
+  p.resid = Y;
+  p.ld_resid = n_feat;
+  p.ws = scratch;
+  p.counters = ctr;
+  p.err = ctr + kNoAllocCounters - 1;
+  CU(launch_gemm(g.tn, EPI_STORE, tw, tx, p, g.n_tiles, g.m_tiles, s, false));
+  return VLA_OK;
+}
+

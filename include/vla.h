@@ -242,6 +242,33 @@ VLA_API int vla_profile_kernels(vla_expert* h, const float* noise, const float* 
 VLA_API int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim,
                           int m_tok, int split_k, void* cuda_stream);
 
+/*
+ * vla_gemm_bf16_noalloc -- the same product as vla_gemm_bf16 (same kernel, same split-K
+ * plan, same arguments and layouts), for callers that must not allocate device memory
+ * while they run: a real-time control thread that is forbidden to enter cudaMalloc /
+ * cudaFree (those calls can take driver locks or synchronize the device, so their latency
+ * is unbounded), or a process whose device memory is fully owned by another allocator.
+ * The pages have no counterpart of this entry point; it exists only for such callers.
+ *
+ * Scratch: the split-K partial tiles, the per-tile arrival counters and a status word
+ * live in one file-scope static device array of 8 MiB + 16 KiB, which every GPU that
+ * loads this library holds until the process exits. A call whose plan needs more than
+ * 8 MiB of partial tiles, or more than 4095 output tiles, is rejected with VLA_ERR_SHAPE
+ * (the message gives the size it needed); nothing is launched then.
+ * Set-up: the first call on each device looks up the device address of that array (with
+ * that device current); with lazy module loading that is also when the driver backs the
+ * array with device memory, so the device's free memory drops once, at that first call.
+ * Make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array. Each call clears the counters and
+ * the status word (stream-ordered) before its kernel, so the contents left by the last
+ * call do not matter; but calls that can overlap on the GPU (other streams, other host
+ * threads) race on the array and must be serialized by the caller.
+ * The call allocates nothing: no cudaMalloc, cudaMallocAsync, cudaFree or allocating
+ * library routine. Stream-ordered. Errors: as vla_gemm_bf16, plus VLA_ERR_SHAPE above.
+ */
+VLA_API int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y, int n_feat,
+                                  int k_dim, int m_tok, int split_k, void* cuda_stream);
+
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VLA_API const char* vla_last_error(void);
 
