@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -80,17 +81,35 @@ GemmPlan plan_gemm(int n_feat, int k_dim, int m_tok, int sm_count) {
   return g;
 }
 
+// Denoise-path plan: the K splits of a tile form one cluster (power of two, at most
+// max_cluster), doubled until the grid covers the SMs, keeping >= 2 K blocks per split.
+GemmPlan plan_gemm_cluster(int n_feat, int k_dim, int m_tok, int sm_count, int max_cluster) {
+  GemmPlan g;
+  g.tn = m_tok <= 64 ? 64 : (m_tok <= 512 ? 128 : 256);
+  g.n_tiles = n_feat / 128;
+  g.m_tiles = cdiv(m_tok, g.tn);
+  const int nkb = k_dim / 64;
+  const int base = g.n_tiles * g.m_tiles;
+  int S = 1;
+  while (S * 2 <= max_cluster && base * S < sm_count && S * 4 <= nkb) S *= 2;
+  g.splits = S;
+  g.kb_per_split = cdiv(nkb, S);
+  return g;
+}
+
 struct AttnPlan {
   int q_tiles, splits;
 };
 
-AttnPlan plan_attn(int rows, int batch, int max_key_tiles, int sm_count) {
+// Key splits per query tile: a power of two (one cluster), doubled until the grid covers
+// the SMs, at most max_cluster and at most the number of key tiles.
+AttnPlan plan_attn(int rows, int batch, int max_key_tiles, int sm_count, int max_cluster) {
   AttnPlan a;
   a.q_tiles = cdiv(rows, attn_q_tile());
   const int base = a.q_tiles * batch;
-  int splits = 1;
-  if (base < sm_count) splits = std::min(cdiv(sm_count, base), std::max(1, max_key_tiles / 2));
-  a.splits = std::max(1, splits);
+  int ns = 1;
+  while (ns * 2 <= max_cluster && base * ns < sm_count && ns * 2 <= max_key_tiles) ns *= 2;
+  a.splits = ns;
   return a;
 }
 
@@ -129,6 +148,8 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 struct vla_expert {
   vla_config cfg;
   int dev = 0, sm_count = 148;
+  int gemm_cluster[3] = {1, 1, 1};   // largest split cluster for token tiles 64 / 128 / 256
+  int attn_cluster = 1;
   int L, W, H, D, F, A, C, Sd, S, hs, HD, Td, Cd, qkv_rows, kcap, ring_off, dyn_off, max_M;
   bool ada, pi0;
 
@@ -145,6 +166,7 @@ struct vla_expert {
 
   // time tables
   float* tables[kTableSlots] = {};
+  float* ctables[kTableSlots] = {};   // W * shift of the folded norms (AdaRMSNorm only)
   int table_steps[kTableSlots] = {};
   int table_age[kTableSlots] = {};
   int table_clock = 0;
@@ -156,9 +178,11 @@ struct vla_expert {
   bf16 *hb = nullptr, *qb = nullptr, *ob = nullptr, *ub = nullptr, *eb = nullptr, *h1b = nullptr;
   bf16 *kc = nullptr, *vc = nullptr;
   CacheDesc* desc = nullptr;
-  float *ws = nullptr, *part_o = nullptr, *part_ml = nullptr;
-  int *ctr = nullptr, *attn_ctr = nullptr, *err = nullptr;
-  size_t ws_floats = 0, part_floats = 0, ctr_ints = 0, attn_ctr_ints = 0;
+  int* err = nullptr;
+  // per-token sum-of-squares partials of the residual, [rstat_rows][max_M]: rstat_a feeds
+  // the first norm of each layer, rstat_b the second (single 64-token tile path)
+  float *rstat_a = nullptr, *rstat_b = nullptr;
+  int rstat_rows = 0;
   float *hx = nullptr, *hstate = nullptr;   // staging for vla_denoise_host (device)
 
   // host mirror of the cache state
@@ -166,6 +190,10 @@ struct vla_expert {
   int prefix_batch = 0, n_static = 0, n_ring = 0, head = 0;
 
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
+
+  // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
+  unsigned long long* trace = nullptr;
+  std::string trace_file;
 
   struct GraphEntry {
     cudaGraph_t g = nullptr;
@@ -177,6 +205,10 @@ struct vla_expert {
 };
 
 namespace {
+
+int cluster_cap(const vla_expert* h, int tn) {
+  return h->gemm_cluster[tn == 64 ? 0 : (tn == 128 ? 1 : 2)];
+}
 
 template <typename T>
 int dalloc(vla_expert* h, T** p, size_t count) {
@@ -207,10 +239,21 @@ int upload_f32(vla_expert* h, float** dst, const uint16_t* src, size_t n) {
   return VLA_OK;
 }
 
+// bf16 [rows][cols] -> fp32 [cols][rows] on the device.
+int upload_f32_t(vla_expert* h, float** dst, const uint16_t* src, size_t rows, size_t cols) {
+  std::vector<float> tmp(rows * cols);
+  for (size_t r = 0; r < rows; ++r)
+    for (size_t c = 0; c < cols; ++c) tmp[c * rows + r] = bf16_to_f32(src[r * cols + c]);
+  int rc = dalloc(h, dst, rows * cols);
+  if (rc) return rc;
+  CU(cudaMemcpy(*dst, tmp.data(), rows * cols * 4, cudaMemcpyHostToDevice));
+  return VLA_OK;
+}
+
 int validate(const vla_config* c, const vla_weights* w) {
   if (!c || !w) return fail(VLA_ERR_ARG, "null config or weights");
-  if (c->n_layers < 1 || c->width < 128 || c->width % 128)
-    return fail(VLA_ERR_SHAPE, "width must be a positive multiple of 128 (got %d)", c->width);
+  if (c->n_layers < 1 || c->width < 128 || c->width % 128 || c->width > 2048)
+    return fail(VLA_ERR_SHAPE, "width must be a multiple of 128 in [128, 2048] (got %d)", c->width);
   if (c->n_kv_heads != 1) return fail(VLA_ERR_UNSUPPORTED, "only one K/V head is supported");
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
     return fail(VLA_ERR_SHAPE, "head_dim must be 32, 64, 128 or 256 (got %d)", c->head_dim);
@@ -255,15 +298,28 @@ int compute_tables(vla_expert* h, int slot, int steps, cudaStream_t s) {
   CU(launch_temb(h->temb, steps, h->Td, s));
   if (h->pi0) {
     // tau_k = time half of the first action-time MLP layer applied to temb_k, + bias
-    CU(launch_rowgemv(h->temb, steps, h->Td, h->tin_full + h->W, h->W + h->Td, h->tin_b, h->W, tbl, 0, s));
+    CU(launch_rowgemv(h->temb, steps, h->Td, h->Td, h->tin_full + h->W, h->W + h->Td, h->tin_b, h->W, tbl, h->W, 0, s));
   } else {
     const float* cond = h->temb;
     if (h->cfg.time_kind == VLA_TIME_ADA_MLP) {
-      CU(launch_rowgemv(h->temb, steps, h->Td, h->cond1_w, h->Td, h->cond1_b, h->W, h->tscr1, 1, s));
-      CU(launch_rowgemv(h->tscr1, steps, h->W, h->cond2_w, h->W, h->cond2_b, h->W, h->tscr2, 1, s));
+      CU(launch_rowgemv(h->temb, steps, h->Td, h->Td, h->cond1_w, h->Td, h->cond1_b, h->W, h->tscr1, h->W, 1, s));
+      CU(launch_rowgemv(h->tscr1, steps, h->W, h->W, h->cond2_w, h->W, h->cond2_b, h->W, h->tscr2, h->W, 1, s));
       cond = h->tscr2;
     }
-    CU(launch_rowgemv(cond, steps, h->Cd, h->mod_w, h->Cd, h->mod_b, (2 * h->L + 1) * 3 * h->W, tbl, 0, s));
+    CU(launch_rowgemv(cond, steps, h->Cd, h->Cd, h->mod_w, h->Cd, h->mod_b, (2 * h->L + 1) * 3 * h->W, tbl,
+                      h->table_stride, 0, s));
+    // folded norms: c = W * shift for the QKV (norm 1) and gate/up (norm 2) weights,
+    // [step][layer][qkv_rows + 2F]
+    const long cw = h->qkv_rows + 2L * h->F;
+    float* ct = h->ctables[slot];
+    for (int l = 0; l < h->L; ++l) {
+      CU(launch_rowgemv(tbl + (static_cast<long>(2 * l) * 3 + 1) * h->W, steps, h->W, h->table_stride,
+                        h->wqkv + static_cast<size_t>(l) * h->qkv_rows * h->W, h->W, nullptr, h->qkv_rows,
+                        ct + l * cw, h->L * cw, 0, s));
+      CU(launch_rowgemv(tbl + (static_cast<long>(2 * l + 1) * 3 + 1) * h->W, steps, h->W, h->table_stride,
+                        h->wgu + static_cast<size_t>(l) * 2 * h->F * h->W, h->W, nullptr, 2 * h->F,
+                        ct + l * cw + h->qkv_rows, h->L * cw, 0, s));
+    }
   }
   h->table_steps[slot] = steps;
   return VLA_OK;
@@ -327,19 +383,26 @@ struct Recorder {
   }
 };
 
+// Sum-of-squares contributor rows a push-mode residual epilogue writes for this plan.
+int contributors(const GemmPlan& g) { return g.n_tiles * g.m_tiles * g.splits * (g.splits == 1 ? 2 : 1); }
+
+GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
+  const int tn = plan_gemm(n_feat, k_dim, M, h->sm_count).tn;
+  return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, cluster_cap(h, tn));
+}
+
 int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensorMap& tw,
                  const CUtensorMap& tx, GemmParams p, int n_feat, int k_dim, int M, bool pdl) {
-  const GemmPlan g = plan_gemm(n_feat, k_dim, M, h->sm_count);
+  const GemmPlan g = denoise_plan(h, n_feat, k_dim, M);
   p.n_feat = n_feat;
   p.k_dim = k_dim;
   p.m_tok = M;
   p.splits = g.splits;
   p.kb_per_split = g.kb_per_split;
-  p.ws = h->ws;
-  p.counters = h->ctr;
   p.err = h->err;
+  p.ld_rstat = h->max_M;
   rec.begin(kind);
-  CU(launch_gemm(g.tn, epi, tw, tx, p, g.n_tiles, g.m_tiles, rec.s, pdl));
+  CU(launch_gemm(g.tn, epi, tw, tx, p, g.n_tiles, g.m_tiles, rec.s, pdl, true));
   return rec.end(kind);
 }
 
@@ -350,8 +413,21 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
   const float* tbl = h->tables[slot];
   const int key_tiles_max = cdiv(h->cfg.n_static_max, attn_key_tile(h->D)) +
                             cdiv(h->cfg.n_sliding, attn_key_tile(h->D)) + cdiv(h->S, attn_key_tile(h->D));
-  const AttnPlan ap = plan_attn(h->S * h->H, B, key_tiles_max, h->sm_count);
+  const AttnPlan ap = plan_attn(h->S * h->H, B, key_tiles_max, h->sm_count, h->attn_cluster);
   const float dt = -1.0f / static_cast<float>(steps);
+  // All suffix tokens in one 64-token tile: the norms are fused into the QKV and gate/up
+  // GEMMs, fed by per-token sum-of-squares partials from the residual writers.
+  const bool fused = M <= 64;
+  const long cw = h->qkv_rows + 2L * h->F;
+  // modulation the next norm applies to z: AdaRMSNorm (1 + scale_j) or RMSNorm (1 + w)
+  auto zmod = [&](const float* tk, int j) -> const float* {
+    if (j >= 2 * L) return nullptr;
+    if (h->ada) return tk + (static_cast<long>(j) * 3 + 0) * W;
+    return ((j & 1) ? h->n2_w : h->n1_w) + static_cast<long>(j / 2) * W;
+  };
+  const int n_mlp2 = contributors(denoise_plan(h, W, W, M));
+  const int n_o = contributors(denoise_plan(h, W, h->HD, M));
+  const int n_down = contributors(denoise_plan(h, W, h->F, M));
   for (int k = 0; k < steps; ++k) {
     const float* tk = tbl + static_cast<long>(k) * h->table_stride;
     EmbedParams e{};
@@ -370,6 +446,12 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
     e.Sd = h->Sd;
     e.W = W;
     e.has_state = h->hs;
+    e.rstat = fused ? h->rstat_a : nullptr;   // contributor row 0
+    if (fused) {
+      e.zout = h->hb;
+      e.zmod = zmod(tk, 0);
+    }
+    int n_a = 1;                               // contributor rows of rstat_a for norm 1
     rec.begin(VLA_K_EMBED);
     CU(launch_embed(e, rec.s, pdl));
     rec.end(VLA_K_EMBED);
@@ -386,10 +468,21 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
       q.ld_resid = W;
       q.has_state = h->hs;
       q.seq = h->S;
+      if (fused) {
+        q.rstat_out = h->rstat_a;
+        q.rstat_slot0 = 1;
+        q.zout = h->hb;
+        q.zmod = zmod(tk, 0);
+        n_a = 1 + n_mlp2;
+      }
       rc = enqueue_gemm(h, rec, VLA_K_TIME_MLP, EPI_BIAS_STORE, h->tm_w2, am.h1b, q, W, W, M, pdl);
       if (rc) return rc;
     }
     for (int l = 0; l < L; ++l) {
+      // trace regions: 0 QKV, 1 attention, 2 O, 3 gate/up, 4 down ([512 CTAs][16])
+      auto tr = [&](int region) -> unsigned long long* {
+        return (h->trace && k == 0 && l == 0) ? h->trace + static_cast<size_t>(region) * 512 * 16 : nullptr;
+      };
       for (int half = 0; half < 2; ++half) {
         const int j = 2 * l + half;
         NormParams n{};
@@ -404,9 +497,11 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
         n.M = M;
         n.W = W;
         n.eps = h->cfg.eps;
-        rec.begin(VLA_K_NORM);
-        CU(launch_norm(n, rec.s, pdl));
-        rec.end(VLA_K_NORM);
+        if (!fused) {
+          rec.begin(VLA_K_NORM);
+          CU(launch_norm(n, rec.s, pdl));
+          rec.end(VLA_K_NORM);
+        }
         const float* gate = h->ada ? tk + (static_cast<long>(j) * 3 + 2) * W : nullptr;
         if (half == 0) {
           GemmParams p{};
@@ -421,6 +516,13 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.n_heads = h->H;
           p.head_dim = h->D;
           p.rope = h->rope;
+          p.trace = tr(0);
+          if (fused) {
+            p.rstat_in = h->rstat_a;
+            p.rstat_n = n_a;
+            p.cvec = h->ada ? h->ctables[slot] + (static_cast<long>(k) * L + l) * cw : nullptr;
+            p.eps = h->cfg.eps;
+          }
           int rc = enqueue_gemm(h, rec, VLA_K_GEMM_QKV, EPI_QKV, h->tm_wqkv, am.hb, p, h->qkv_rows, W, M, pdl);
           if (rc) return rc;
           AttnParams a{};
@@ -436,11 +538,9 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           a.dyn_off = h->dyn_off;
           a.has_state = h->hs;
           a.n_splits = ap.splits;
-          a.part_o = h->part_o;
-          a.part_ml = h->part_ml;
-          a.counters = h->attn_ctr;
           a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h->D));
           a.err = h->err;
+          a.trace = tr(1);
           rec.begin(VLA_K_ATTN);
           CU(launch_attention(h->D, a, B, ap.q_tiles, rec.s, pdl));
           rec.end(VLA_K_ATTN);
@@ -449,6 +549,12 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           o.resid = h->resid;
           o.ld_resid = W;
           o.vec = gate;
+          o.trace = tr(2);
+          if (fused) {
+            o.rstat_out = h->rstat_b;
+            o.zout = h->hb;
+            o.zmod = zmod(tk, j + 1);
+          }
           rc = enqueue_gemm(h, rec, VLA_K_GEMM_O, EPI_RESID, h->tm_wo, am.ob, o, W, h->HD, M, pdl);
           if (rc) return rc;
         } else {
@@ -456,6 +562,13 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.w_row0 = l * 2 * h->F;
           p.out = h->ub;
           p.ld_out = h->F;
+          p.trace = tr(3);
+          if (fused) {
+            p.rstat_in = h->rstat_b;
+            p.rstat_n = n_o;
+            p.cvec = h->ada ? h->ctables[slot] + (static_cast<long>(k) * L + l) * cw + h->qkv_rows : nullptr;
+            p.eps = h->cfg.eps;
+          }
           int rc = enqueue_gemm(h, rec, VLA_K_GEMM_GATEUP, EPI_GEGLU, h->tm_wgu, am.hb, p, 2 * h->F, W, M, pdl);
           if (rc) return rc;
           GemmParams d{};
@@ -463,6 +576,13 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           d.resid = h->resid;
           d.ld_resid = W;
           d.vec = gate;
+          d.trace = tr(4);
+          if (fused) {
+            d.rstat_out = h->rstat_a;
+            d.zout = l + 1 < L ? h->hb : nullptr;
+            d.zmod = zmod(tk, j + 1);
+            n_a = n_down;
+          }
           rc = enqueue_gemm(h, rec, VLA_K_GEMM_DOWN, EPI_RESID, h->tm_wdown, am.ub, d, W, h->F, M, pdl);
           if (rc) return rc;
         }
@@ -615,6 +735,10 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   h->dyn_off = cfg->n_static_max + cfg->n_sliding;
   h->kcap = h->dyn_off + h->S;
   h->max_M = cfg->max_batch * h->S;
+  h->gemm_cluster[0] = gemm_max_cluster(64);
+  h->gemm_cluster[1] = gemm_max_cluster(128);
+  h->gemm_cluster[2] = gemm_max_cluster(256);
+  h->attn_cluster = attn_max_cluster(h->D);
   const int L = h->L, W = h->W, H = h->H, D = h->D, F = h->F, DH = D / 2;
 
   auto cleanup = [&](int code) {
@@ -656,12 +780,12 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = upload_bf16(h, &h->wdown, w->w_down, static_cast<size_t>(L) * W * F))) return cleanup(rc);
 
   // ---- small fp32 parameters
-  if ((rc = upload_f32(h, &h->ain_w, w->action_in_w, static_cast<size_t>(W) * h->A))) return cleanup(rc);
+  if ((rc = upload_f32_t(h, &h->ain_w, w->action_in_w, W, h->A))) return cleanup(rc);
   if ((rc = upload_f32(h, &h->ain_b, w->action_in_b, W))) return cleanup(rc);
   if ((rc = upload_f32(h, &h->aout_w, w->action_out_w, static_cast<size_t>(h->A) * W))) return cleanup(rc);
   if ((rc = upload_f32(h, &h->aout_b, w->action_out_b, h->A))) return cleanup(rc);
   if (h->hs) {
-    if ((rc = upload_f32(h, &h->st_w, w->state_in_w, static_cast<size_t>(W) * h->Sd))) return cleanup(rc);
+    if ((rc = upload_f32_t(h, &h->st_w, w->state_in_w, W, h->Sd))) return cleanup(rc);
     if ((rc = upload_f32(h, &h->st_b, w->state_in_b, W))) return cleanup(rc);
   }
   if (h->pi0) {
@@ -722,36 +846,19 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = dalloc(h, &h->kc, cache_elems))) return cleanup(rc);
   if ((rc = dalloc(h, &h->vc, cache_elems))) return cleanup(rc);
   if ((rc = dalloc(h, &h->rope, static_cast<size_t>(h->S) * D))) return cleanup(rc);
+  h->rstat_rows = (W / 128) * 32 + 2;
+  if ((rc = dalloc(h, &h->rstat_a, static_cast<size_t>(h->rstat_rows) * h->max_M))) return cleanup(rc);
+  if ((rc = dalloc(h, &h->rstat_b, static_cast<size_t>(h->rstat_rows) * h->max_M))) return cleanup(rc);
   if ((rc = dalloc(h, &h->desc, 1))) return cleanup(rc);
   if ((rc = dalloc(h, &h->err, 1))) return cleanup(rc);
-
-  // workspace sizes: the largest plan over every batch size up to max_batch
-  {
-    const int shapes[6][2] = {{h->qkv_rows, W}, {W, h->HD}, {2 * F, W}, {W, F}, {W, W}, {W, W}};
-    const int key_tiles_max = cdiv(cfg->n_static_max, attn_key_tile(D)) + cdiv(cfg->n_sliding, attn_key_tile(D)) +
-                              cdiv(h->S, attn_key_tile(D));
-    for (int b = 1; b <= cfg->max_batch; ++b) {
-      for (auto& sh : shapes) {
-        const GemmPlan g = plan_gemm(sh[0], sh[1], b * h->S, h->sm_count);
-        h->ws_floats = std::max(h->ws_floats, static_cast<size_t>(g.n_tiles) * g.m_tiles * g.splits * g.tn * 128);
-        h->ctr_ints = std::max(h->ctr_ints, static_cast<size_t>(g.n_tiles) * g.m_tiles);
-      }
-      const AttnPlan a = plan_attn(h->S * H, b, key_tiles_max, h->sm_count);
-      if (a.splits > 1)
-        h->part_floats = std::max(h->part_floats, static_cast<size_t>(b) * a.q_tiles * a.splits * attn_q_tile() * D);
-      h->attn_ctr_ints = std::max(h->attn_ctr_ints, static_cast<size_t>(b) * a.q_tiles);
-    }
-  }
-  if ((rc = dalloc(h, &h->ws, h->ws_floats))) return cleanup(rc);
-  if ((rc = dalloc(h, &h->ctr, h->ctr_ints))) return cleanup(rc);
-  if ((rc = dalloc(h, &h->part_o, h->part_floats))) return cleanup(rc);
-  if ((rc = dalloc(h, &h->part_ml, h->part_floats / std::max(1, D) * 2 + 2))) return cleanup(rc);
-  if ((rc = dalloc(h, &h->attn_ctr, h->attn_ctr_ints))) return cleanup(rc);
 
   // ---- time tables
   h->table_stride = h->ada ? static_cast<long>(2 * L + 1) * 3 * W : W;
   for (int i = 0; i < kTableSlots; ++i) {
     if ((rc = dalloc(h, &h->tables[i], static_cast<size_t>(cfg->max_steps) * h->table_stride))) return cleanup(rc);
+    if (h->ada &&
+        (rc = dalloc(h, &h->ctables[i], static_cast<size_t>(cfg->max_steps) * L * (h->qkv_rows + 2 * static_cast<size_t>(F)))))
+      return cleanup(rc);
     h->table_steps[i] = 0;
   }
   if ((rc = dalloc(h, &h->temb, static_cast<size_t>(cfg->max_steps) * h->Td))) return cleanup(rc);
@@ -771,6 +878,11 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     h->tm_w2 = h->tm_wo;
   }
 
+  if (const char* tf = getenv("VLA_TRACE_FILE")) {
+    h->trace_file = tf;
+    if ((rc = dalloc(h, &h->trace, static_cast<size_t>(5) * 512 * 16))) return cleanup(rc);
+  }
+
   cudaError_t e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cleanup(fail(VLA_ERR_CUDA, "stream create: %s", cudaGetErrorString(e)));
   int slot;
@@ -784,6 +896,21 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
 void vla_expert_destroy(vla_expert* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  if (h->trace && !h->trace_file.empty()) {
+    std::vector<unsigned long long> t(static_cast<size_t>(5) * 512 * 16);
+    if (cudaMemcpy(t.data(), h->trace, t.size() * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
+      if (FILE* f = fopen(h->trace_file.c_str(), "w")) {
+        static const char* names[5] = {"qkv", "attention", "o", "gateup", "down"};
+        for (int r = 0; r < 5; ++r)
+          for (int c = 0; c < 512; ++c)
+            for (int k = 0; k < 16; ++k) {
+              const unsigned long long v = t[(static_cast<size_t>(r) * 512 + c) * 16 + k];
+              if (v) fprintf(f, "%s,%d,%d,%llu\n", names[r], c, k, v);
+            }
+        fclose(f);
+      }
+    }
+  }
   for (auto& kv : h->graphs) {
     cudaGraphExecDestroy(kv.second.exec);
     cudaGraphDestroy(kv.second.g);
@@ -906,10 +1033,8 @@ int vla_device_status(vla_expert* h, void* cuda_stream) {
   CU(cudaMemcpy(&v, h->err, sizeof(int), cudaMemcpyDeviceToHost));
   if (v != 0) {
     cudaMemset(h->err, 0, sizeof(int));
-    cudaMemset(h->ctr, 0, h->ctr_ints * sizeof(int));
-    cudaMemset(h->attn_ctr, 0, h->attn_ctr_ints * sizeof(int));
     cudaDeviceSynchronize();
-    return fail(VLA_ERR_TIMEOUT, "a kernel wait timed out (device status %d); split counters were reset", v);
+    return fail(VLA_ERR_TIMEOUT, "a kernel wait timed out (device status %d); the status word was cleared", v);
   }
   return VLA_OK;
 }

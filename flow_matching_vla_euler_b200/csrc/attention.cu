@@ -64,7 +64,12 @@ struct AttnCfg {
   static constexpr int KT = D >= 256 ? 32 : 64;            // keys per stage
   static constexpr int CPR = D / 8;                        // 16-byte chunks per row
   static constexpr int SWZ = (CPR >= 8 ? 8 : CPR) - 1;     // XOR mask for chunk swizzle
-  static constexpr size_t SMEM = (size_t)(kQT + 4 * KT) * D * 2;
+  static constexpr size_t MAIN = (size_t)(kQT + 4 * KT) * D * 2;   // Q + 2 K/V stages
+  // split merge: each CTA receives, from every split of its cluster, the unnormalised O
+  // rows it owns ([splits][64/splits][D], 64 rows in total) and their (m, l)
+  static constexpr size_t RECV_O = (size_t)kQT * D * 4;
+  static constexpr size_t RECV_ML = (size_t)kQT * 8;
+  static constexpr size_t SMEM = MAIN + RECV_O + RECV_ML + 16;
 };
 
 // byte offset of (row, chunk) in a swizzled [rows][D] bf16 tile
@@ -106,6 +111,44 @@ __device__ __forceinline__ void load_kv_tile(const bf16* kbase, const bf16* vbas
   }
 }
 
+// CTA rank r of the cluster owns rows [r*64/NS, (r+1)*64/NS) of the query tile; every
+// split has pushed its unnormalised O rows and (m, l) for them into r's receive buffers
+// (slot = sender rank). The owner merges the NS slots in rank order (deterministic).
+template <int D, int NS>
+__device__ __forceinline__ void merge_received(const AttnParams& p, const float* ro, const float* rml, int b,
+                                               int R, int row0, int r0) {
+  constexpr int ROWS = kQT / NS, D4 = D / 4;
+  for (int it = threadIdx.x; it < ROWS * D4; it += blockDim.x) {
+    const int rr = it / D4, d = (it % D4) * 4;
+    if (row0 + r0 + rr >= R) continue;
+    float2 ml[NS];
+    float4 v[NS];
+#pragma unroll
+    for (int q = 0; q < NS; ++q) {
+      ml[q] = *reinterpret_cast<const float2*>(rml + (q * ROWS + rr) * 2);
+      v[q] = *reinterpret_cast<const float4*>(ro + (q * ROWS + rr) * D + d);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < NS; ++q) M = fmaxf(M, ml[q].x);
+    float wsum = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int q = 0; q < NS; ++q) {
+      const float w = (ml[q].x == -INFINITY) ? 0.0f : exp2f(ml[q].x - M);
+      wsum += w * ml[q].y;
+      acc.x += w * v[q].x;
+      acc.y += w * v[q].y;
+      acc.z += w * v[q].z;
+      acc.w += w * v[q].w;
+    }
+    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+    bf16* dst = p.out + (static_cast<size_t>(b) * R + row0 + r0 + rr) * D + d;
+    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
   using C = AttnCfg<D>;
@@ -122,8 +165,24 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
   const int H = p.n_heads, R = p.seq * H;
   const int row0 = qt * kQT;
 
-  if (threadIdx.x == 0) pdl_trigger();
+  float* recv_o = reinterpret_cast<float*>(sm + C::MAIN);
+  float* recv_ml = reinterpret_cast<float*>(sm + C::MAIN + C::RECV_O);
+  const uint32_t recv_bar = smem_u32(sm + C::MAIN + C::RECV_O + C::RECV_ML);
+  if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 0);
+    if (p.n_splits > 1) {
+      mbar_init(recv_bar, 1);
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(C::RECV_O + C::RECV_ML));
+      fence_mbar_init();
+    }
+    pdl_trigger();
+  }
+  if (p.n_splits > 1) {
+    __syncthreads();
+    cluster_sync_all();                      // every receive barrier of the cluster is armed
+  }
   pdl_wait();
+  if (threadIdx.x == 0) trace_stamp(p.trace, 1);
   const CacheDesc cd = *p.cache;
   Segs sg;
   sg.off[0] = 0;
@@ -263,6 +322,7 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
     __syncthreads();
   }
 
+  if (threadIdx.x == 0) trace_stamp(p.trace, 2);
   // quad-reduce the row sums
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
@@ -287,65 +347,57 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
     return;
   }
 
-  // split partials, then the last CTA of this query tile merges them in split order
-  const int q_tiles = gridDim.x;
-  const size_t slot = (static_cast<size_t>(b) * q_tiles + qt) * p.n_splits + split;
-  float* po = p.part_o + slot * kQT * D;
-  float* pml = p.part_ml + slot * kQT * 2;
+  // Split partials: the n_splits CTAs of this query tile are one cluster. Each writes its
+  // unnormalised O and (m, l) to its own shared memory (the Q/K/V buffers are idle now)
+  // and pushes the rows owned by CTA q to q's receive buffers with bulk copies.
+  __syncthreads();
+  float* po = reinterpret_cast<float*>(sm);                // [64][D]
+  float* pml = po + kQT * D;                               // [64][2]
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
     for (int i = 0; i < OB; ++i)
-      __stcg(reinterpret_cast<float2*>(po + rloc[h2] * D + i * 8 + qd * 2),
-             make_float2(o[i][2 * h2], o[i][2 * h2 + 1]));
-    if (qd == 0) __stcg(reinterpret_cast<float2*>(pml + rloc[h2] * 2), make_float2(m_run[h2], l_run[h2]));
+      *reinterpret_cast<float2*>(po + rloc[h2] * D + i * 8 + qd * 2) =
+          make_float2(o[i][2 * h2], o[i][2 * h2 + 1]);
+    if (qd == 0) *reinterpret_cast<float2*>(pml + rloc[h2] * 2) = make_float2(m_run[h2], l_run[h2]);
   }
-  __threadfence();
+  fence_proxy_async_smem();
   __syncthreads();
-  __shared__ int s_last;
-  int* ctr = p.counters + static_cast<size_t>(b) * q_tiles + qt;
-  if (threadIdx.x == 0) s_last = (atomicAdd(ctr, 1) == p.n_splits - 1) ? 1 : 0;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  const size_t base = (static_cast<size_t>(b) * q_tiles + qt) * p.n_splits;
-  for (int idx = threadIdx.x; idx < kQT * 2; idx += blockDim.x) {
-    const int r = idx >> 1, half = idx & 1;
-    if (row0 + r >= R) continue;
-    float M = -INFINITY;
-    for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, __ldcg(p.part_ml + ((base + s) * kQT + r) * 2));
-    float wsum = 0.0f;
-    float acc[D / 2];
-#pragma unroll
-    for (int d = 0; d < D / 2; ++d) acc[d] = 0.0f;
-    for (int s = 0; s < p.n_splits; ++s) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((base + s) * kQT + r) * 2));
-      const float w = (ml.x == -INFINITY) ? 0.0f : exp2f(ml.x - M);
-      wsum += w * ml.y;
-      const float* src = p.part_o + ((base + s) * kQT + r) * D + half * (D / 2);
-#pragma unroll
-      for (int d = 0; d < D / 2; d += 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + d));
-        acc[d] += w * v.x;
-        acc[d + 1] += w * v.y;
-        acc[d + 2] += w * v.z;
-        acc[d + 3] += w * v.w;
-      }
+  const int ns = p.n_splits, rows = kQT / ns;
+  const uint32_t rank = cluster_ctarank();
+  if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 3);
+    const uint32_t so = static_cast<uint32_t>(rows * D * 4), sml = static_cast<uint32_t>(rows * 8);
+    const uint32_t po_s = smem_u32(po), pml_s = smem_u32(pml);
+    const uint32_t ro_s = smem_u32(recv_o) + rank * so, rml_s = smem_u32(recv_ml) + rank * sml;
+    for (int q = 0; q < ns; ++q) {
+      const uint32_t rb = mapa_shared(recv_bar, q);
+      bulk_copy_to_peer(mapa_shared(ro_s, q), po_s + q * so, so, rb);
+      bulk_copy_to_peer(mapa_shared(rml_s, q), pml_s + q * sml, sml, rb);
     }
-    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
-    bf16* dst = p.out + (static_cast<size_t>(b) * R + row0 + r) * D + half * (D / 2);
-#pragma unroll
-    for (int d = 0; d < D / 2; d += 2)
-      *reinterpret_cast<__nv_bfloat162*>(dst + d) = __floats2bfloat162_rn(acc[d] * inv, acc[d + 1] * inv);
+    bulk_commit();
   }
-  if (threadIdx.x == 0) *ctr = 0;
+  mbar_wait(recv_bar, 0, p.err);
+  if (threadIdx.x == 0) trace_stamp(p.trace, 4);
+  const int r0 = static_cast<int>(rank) * rows;
+  switch (ns) {
+    case 2: merge_received<D, 2>(p, recv_o, recv_ml, b, R, row0, r0); break;
+    case 4: merge_received<D, 4>(p, recv_o, recv_ml, b, R, row0, r0); break;
+    case 8: merge_received<D, 8>(p, recv_o, recv_ml, b, R, row0, r0); break;
+    default: merge_received<D, 16>(p, recv_o, recv_ml, b, R, row0, r0); break;
+  }
+  if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 5);
+    bulk_wait_all();                         // own outgoing copies finished before exit
+  }
 }
 
 template <int D>
 static cudaError_t configure_d() {
-  return cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(AttnCfg<D>::SMEM));
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(AttnCfg<D>::SMEM));
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
 cudaError_t configure_attention_kernels() {
@@ -368,16 +420,28 @@ static cudaError_t launch_d(const AttnParams& p, int batch, int q_tiles, cudaStr
   cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (p.n_splits > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = p.n_splits;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, attn_kernel<D>, p);
 }
 
 cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
                              cudaStream_t s, bool pdl) {
+  if (p.n_splits < 1 || p.n_splits > 16 || (p.n_splits & (p.n_splits - 1))) return cudaErrorInvalidValue;
   switch (head_dim) {
     case 32: return launch_d<32>(p, batch, q_tiles, s, pdl);
     case 64: return launch_d<64>(p, batch, q_tiles, s, pdl);
@@ -388,6 +452,37 @@ cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q
 }
 
 int attn_q_tile() { return kQT; }
+
+template <int D>
+static int max_cluster_d() {
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = AttnCfg<D>::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  for (int c = 16; c >= 2; c >>= 1) {
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = c;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(1, c, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_kernel<D>, &cfg) == cudaSuccess && n > 0) return c;
+    cudaGetLastError();
+  }
+  return 1;
+}
+
+int attn_max_cluster(int head_dim) {
+  if (configure_attention_kernels() != cudaSuccess) return 1;
+  switch (head_dim) {
+    case 32: return max_cluster_d<32>();
+    case 64: return max_cluster_d<64>();
+    case 128: return max_cluster_d<128>();
+    default: return max_cluster_d<256>();
+  }
+}
 
 int attn_key_tile(int head_dim) {
   switch (head_dim) {

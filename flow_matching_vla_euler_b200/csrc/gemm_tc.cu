@@ -24,16 +24,20 @@
 
 namespace vla {
 
-template <int TN>
+template <int TN, bool CL>
 struct GemmCfg {
   static constexpr int BM = 128;                  // weight rows per tile (MMA M)
   static constexpr int BK = 64;                   // K per stage: one 128-byte swizzle row
   static constexpr int A_BYTES = BM * BK * 2;     // 16 KB
   static constexpr int B_BYTES = TN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 4;
+  // token tile 64 with cluster splits: partial tiles are pushed to their owners' receive
+  // buffers (32 KB); three stages keep two CTAs per SM
+  static constexpr bool PUSH = CL && TN == 64;
+  static constexpr int STAGES = PUSH ? 3 : 4;
+  static constexpr int RECV_BYTES = PUSH ? 128 * TN * 4 : 0;
   static constexpr int TMEM_COLS = TN;            // fp32 accumulator columns (power of 2)
-  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + RECV_BYTES + 1024;   // + barriers, rinv
 };
 
 template <int EPI>
@@ -124,39 +128,234 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
   }
 }
 
-template <int TN, int EPI>
+// Epilogue on one pair of adjacent output rows (2i, 2i + 1) at one token, used by the
+// cluster reduction; the pair is the unit the GeGLU and rotary epilogues need.
+template <int EPI>
+__device__ __forceinline__ void epi_pair(const GemmParams& p, int fn0, int m, float v0, float v1) {
+  if (m >= p.m_tok) return;
+  if constexpr (EPI == EPI_RESID) {
+    float2* dst = reinterpret_cast<float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0);
+    const float g0 = p.vec ? p.vec[fn0] : 1.0f, g1 = p.vec ? p.vec[fn0 + 1] : 1.0f;
+    float2 r = *dst;
+    r.x += g0 * v0;
+    r.y += g1 * v1;
+    *dst = r;
+  } else if constexpr (EPI == EPI_STORE) {
+    *reinterpret_cast<float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0) = make_float2(v0, v1);
+  } else if constexpr (EPI == EPI_BIAS_STORE) {
+    if (p.has_state && (m % p.seq) == 0) return;
+    *reinterpret_cast<float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0) =
+        make_float2(v0 + p.vec[fn0], v1 + p.vec[fn0 + 1]);
+  } else if constexpr (EPI == EPI_SWISH_VEC) {
+    *reinterpret_cast<__nv_bfloat162*>(p.out + static_cast<size_t>(m) * p.ld_out + fn0) =
+        __floats2bfloat162_rn(swishf(v0 + p.vec[fn0]), swishf(v1 + p.vec[fn0 + 1]));
+  } else if constexpr (EPI == EPI_GEGLU) {
+    p.out[static_cast<size_t>(m) * p.ld_out + (fn0 >> 1)] = __float2bfloat16_rn(gelu_tanhf(v0) * v1);
+  } else if constexpr (EPI == EPI_QKV) {
+    const int D = p.head_dim, DH = D >> 1, H = p.n_heads;
+    const int pr = fn0 >> 1;
+    if (pr >= (H + 2) * DH) return;   // padding rows
+    const int b = m / p.seq, s = m - b * p.seq;
+    int kind, head = 0, i;
+    if (pr < H * DH) {
+      kind = 0;
+      head = pr / DH;
+      i = pr - head * DH;
+    } else if (pr < (H + 1) * DH) {
+      kind = 1;
+      i = pr - H * DH;
+    } else {
+      kind = 2;
+      i = pr - (H + 1) * DH;
+    }
+    float o0 = v0, o1 = v1;
+    if (kind < 2) {
+      const float2 cs = reinterpret_cast<const float2*>(p.rope)[s * DH + i];
+      o0 = fmaf(v0, cs.x, -v1 * cs.y);
+      o1 = fmaf(v1, cs.x, v0 * cs.y);
+    }
+    bf16* dst;
+    if (kind == 0)
+      dst = p.out + static_cast<size_t>(m) * p.ld_out + head * D;
+    else
+      dst = (kind == 1 ? p.kc : p.vc) + (static_cast<size_t>(b) * p.kcap + p.dyn_off + s) * D;
+    dst[i] = __float2bfloat16_rn(o0);
+    dst[i + DH] = __float2bfloat16_rn(o1);
+  }
+}
+
+// Sum of rows [row0, row0 + 128/S) of the S partial tiles of this cluster (rank order,
+// so the result does not depend on timing), then the epilogue on row pairs. Loads of
+// G items x S ranks are issued before any add so the distributed-shared-memory latency
+// is paid once per group, not once per rank.
+template <int EPI, int TN, int S>
+__device__ __forceinline__ void cluster_reduce(const GemmParams& p, uint32_t part, int etid, int row0,
+                                               int fbase, int m0) {
+  constexpr int HALF = 64 / S;                 // row pairs per rank
+  constexpr int ITEMS = HALF * TN;             // (row pair, token) items per rank
+  constexpr int G = S >= 16 ? 1 : 16 / S;      // items per group
+  uint32_t peer[S];
+#pragma unroll
+  for (int q = 0; q < S; ++q) peer[q] = mapa_shared(part, q);
+  for (int base = etid; base < ITEMS; base += 128 * G) {
+    float2 t[G][S];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int it = base + g * 128;
+      const int rp = it % HALF, c = it / HALF;
+      const uint32_t off = static_cast<uint32_t>((c * 128 + row0 + 2 * rp) * 4);
+#pragma unroll
+      for (int q = 0; q < S; ++q)
+        t[g][q] = it < ITEMS ? ld_dsmem_f2(peer[q] + off) : make_float2(0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int it = base + g * 128;
+      if (it >= ITEMS) break;
+      float v0 = 0.0f, v1 = 0.0f;
+#pragma unroll
+      for (int q = 0; q < S; ++q) {
+        v0 += t[g][q].x;
+        v1 += t[g][q].y;
+      }
+      const int rp = it % HALF, c = it / HALF;
+      epi_pair<EPI>(p, fbase + 2 * rp, m0 + c, v0, v1);
+    }
+  }
+}
+
+// Push-mode reduction, token tile 64: every CTA of the cluster has sent rows
+// [q*128/S, (q+1)*128/S) of its partial tile to CTA q (receive slot = sender rank); the
+// owner sums its S slots in rank order (deterministic) and runs the epilogue on row pairs.
+// Partial rows are stored with their 16-byte chunks XOR-swizzled by (global row & 15).
+template <int EPI, int S>
+__device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, const float* s_rinv, int etid,
+                                            int row0, int fbase, int m0, int contrib) {
+  constexpr int RS = 128 / S, HALF = RS / 2, ITEMS = HALF * 64;
+  constexpr bool RESID = EPI == EPI_RESID || EPI == EPI_BIAS_STORE;
+  for (int it = etid; it < ITEMS; it += 128) {
+    const int rp = it % HALF, c = it / HALF;
+    const int lr0 = 2 * rp, lr1 = lr0 + 1;
+    const int i0 = lr0 * 64 + ((((c >> 2) ^ ((row0 + lr0) & 15))) << 2) + (c & 3);
+    const int i1 = lr1 * 64 + ((((c >> 2) ^ ((row0 + lr1) & 15))) << 2) + (c & 3);
+    float v0 = 0.0f, v1 = 0.0f;
+#pragma unroll
+    for (int q = 0; q < S; ++q) {
+      v0 += recv[q * RS * 64 + i0];
+      v1 += recv[q * RS * 64 + i1];
+    }
+    const int m = m0 + c;
+    const int fn0 = fbase + lr0;
+    if constexpr (RESID) {
+      // new residual values (+ z for the next GEMM) -> per-token sum of squares
+      float ss = 0.0f;
+      if (m < p.m_tok) {
+        const size_t off = static_cast<size_t>(m) * p.ld_resid + fn0;
+        float2* dst = reinterpret_cast<float2*>(p.resid + off);
+        float2 r = make_float2(0.0f, 0.0f);
+        bool wrote = true;
+        if constexpr (EPI == EPI_RESID) {
+          const float g0 = p.vec ? p.vec[fn0] : 1.0f, g1 = p.vec ? p.vec[fn0 + 1] : 1.0f;
+          r = *dst;
+          r.x += g0 * v0;
+          r.y += g1 * v1;
+          *dst = r;
+        } else {
+          wrote = !(p.has_state && (m % p.seq) == 0);
+          if (wrote) {
+            r = make_float2(v0 + p.vec[fn0], v1 + p.vec[fn0 + 1]);
+            *dst = r;
+          }
+        }
+        if (wrote) {
+          ss = r.x * r.x + r.y * r.y;
+          if (p.zout)
+            *reinterpret_cast<__nv_bfloat162*>(p.zout + off) =
+                __floats2bfloat162_rn(r.x * (1.0f + p.zmod[fn0]), r.y * (1.0f + p.zmod[fn0 + 1]));
+        }
+      }
+      if (p.rstat_out) {
+        // one contributor row per 32 row pairs of this owner (a warp's worth of lanes)
+        constexpr int SUB = (HALF + 31) / 32;
+#pragma unroll
+        for (int o = 1; o < HALF && o < 32; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if ((rp & 31) == 0 && m < p.m_tok)
+          p.rstat_out[static_cast<size_t>(p.rstat_slot0 + contrib * SUB + (rp >> 5)) * p.ld_rstat + m] = ss;
+      }
+    } else {
+      if (s_rinv) {
+        // folded norm: out = rinv[m] * (W z) + W shift
+        const float rv = s_rinv[c];
+        v0 = fmaf(rv, v0, p.cvec ? p.cvec[fn0] : 0.0f);
+        v1 = fmaf(rv, v1, p.cvec ? p.cvec[fn0 + 1] : 0.0f);
+      }
+      epi_pair<EPI>(p, fn0, m, v0, v1);
+    }
+  }
+}
+
+// CL = false: one CTA per (tile, split); split partials, if any, go through the global
+// workspace p.ws and the last CTA of a tile to arrive sums them (any split count).
+// CL = true: the p.splits CTAs of a tile are one thread-block cluster; each leaves its
+// partial tile in its own shared memory and CTA rank r sums rows [r*128/S, (r+1)*128/S)
+// over all ranks through distributed shared memory, in rank order (deterministic).
+template <int TN, int EPI, bool CL>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                    const GemmParams p) {
-  using G = GemmCfg<TN>;
+  using G = GemmCfg<TN, CL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + G::STAGES * G::A_BYTES;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2 * G::STAGES + 1);
+  float* recv = reinterpret_cast<float*>(smem + G::STAGES * G::STAGE_BYTES);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES + G::RECV_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2 * G::STAGES + 2);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
-  const int kb0 = split * p.kb_per_split;
-  const int nkb = min(p.kb_per_split, p.k_dim / G::BK - kb0);
+  const int nkb_total = p.k_dim / G::BK;
+  int kb0, nkb;
+  if constexpr (CL) {
+    kb0 = (split * nkb_total) / p.splits;
+    nkb = ((split + 1) * nkb_total) / p.splits - kb0;
+  } else {
+    kb0 = split * p.kb_per_split;
+    nkb = min(p.kb_per_split, nkb_total - kb0);
+  }
+  const bool cluster_red = CL && p.splits > 1;
+  const bool push = G::PUSH;                 // token tile 64: always through the receive buffer
 
   const uint32_t full0 = smem_u32(&bar[0]);
   const uint32_t empty0 = smem_u32(&bar[G::STAGES]);
   const uint32_t accf = smem_u32(&bar[2 * G::STAGES]);
+  const uint32_t recv_bar = smem_u32(&bar[2 * G::STAGES + 1]);
+  const int npre = min(nkb, G::STAGES);
 
   if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 0);
     for (int s = 0; s < G::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     mbar_init(accf, 1);
+    if (push) {
+      mbar_init(recv_bar, 1);
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(128 * TN * 4));   // S slices
+    }
     *s_last = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
+    // Weights are never written by earlier kernels: stream them right away.
+    const uint64_t pol_w = policy_evict_first();
+    const int y_w = p.w_row0 + n_tile * G::BM;
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect_tx(full0 + 8 * i, G::STAGE_BYTES);
+      tma_load_2d(smem_u32(sA + i * G::A_BYTES), &tm_w, full0 + 8 * i, (kb0 + i) * G::BK, y_w, pol_w);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), G::TMEM_COLS);
@@ -166,7 +365,11 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) pdl_trigger();
+  if (push) cluster_sync_all();              // every receive barrier of the cluster is armed
+  if (threadIdx.x == 0) {
+    pdl_trigger();
+    trace_stamp(p.trace, 1);
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -174,17 +377,10 @@ __global__ void __launch_bounds__(192, 1)
       const uint64_t pol_x = policy_evict_last();
       const int y_w = p.w_row0 + n_tile * G::BM;
       const int y_x = m_tile * TN;
-      const int npre = min(nkb, G::STAGES);
-      // Weights are never written by earlier kernels: stream them before the wait.
-      for (int i = 0; i < npre; ++i) {
-        mbar_arrive_expect_tx(full0 + 8 * i, G::STAGE_BYTES);
-        tma_load_2d(smem_u32(sA + i * G::A_BYTES), &tm_w, full0 + 8 * i, (kb0 + i) * G::BK, y_w,
-                    pol_w);
-      }
       pdl_wait();
+      trace_stamp(p.trace, 2);
       for (int i = 0; i < npre; ++i)
-        tma_load_2d(smem_u32(sB + i * G::B_BYTES), &tm_x, full0 + 8 * i, (kb0 + i) * G::BK, y_x,
-                    pol_x);
+        tma_load_2d(smem_u32(sB + i * G::B_BYTES), &tm_x, full0 + 8 * i, (kb0 + i) * G::BK, y_x, pol_x);
       int issued = npre;
       for (int i = npre; i < nkb; ++i) {
         const int s = i % G::STAGES;
@@ -209,6 +405,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = 0; i < nkb; ++i) {
         const int s = i % G::STAGES;
         if (!mbar_wait(full0 + 8 * s, (i / G::STAGES) & 1, p.err)) break;
+        if (i == 0) trace_stamp(p.trace, 3);
         tc_fence_after();
         const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * G::A_BYTES));
         const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * G::B_BYTES));
@@ -218,6 +415,7 @@ __global__ void __launch_bounds__(192, 1)
         umma_commit(empty0 + 8 * s);
       }
       umma_commit(accf);   // always signalled, so the epilogue never waits forever
+      trace_stamp(p.trace, 4);
     }
     __syncwarp();
   } else {
@@ -229,50 +427,156 @@ __global__ void __launch_bounds__(192, 1)
     const int tile = m_tile * gridDim.x + n_tile;
     const int fn = n_tile * G::BM + r;
     const int m0 = m_tile * TN;
+    float* s_rinv = reinterpret_cast<float*>(tmem_slot + 4);
+    if (p.rstat_in) {
+      // rinv per token from the residual producers' sum-of-squares partials, computed while
+      // the main loop runs (two threads per token, loads unrolled)
+      const int tok = etid & 63, par = etid >> 6;
+      const int m = m0 + tok;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (m < p.m_tok) {
+        int c = par;
+        for (; c + 14 < p.rstat_n; c += 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[u] += p.rstat_in[static_cast<size_t>(c + 2 * u) * p.ld_rstat + m];
+        }
+        for (; c < p.rstat_n; c += 2) acc[0] += p.rstat_in[static_cast<size_t>(c) * p.ld_rstat + m];
+      }
+      float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      if (par == 1) s_rinv[64 + tok] = ss;
+      named_bar_sync(1, 128);
+      if (par == 0)
+        s_rinv[tok] = m < p.m_tok ? 1.0f / sqrtf((ss + s_rinv[64 + tok]) / static_cast<float>(p.k_dim) + p.eps) : 0.0f;
+      named_bar_sync(1, 128);
+    }
     mbar_wait(accf, 0, p.err);
     tc_fence_after();
+    if (etid == 0) trace_stamp(p.trace, 5);
 
-    bool last = true;
-    if (p.splits > 1) {
-      float* mine = p.ws + static_cast<size_t>(tile * p.splits + split) * TN * 128;
+    if (push) {
+      // partial tile -> own shared memory as [row][64 tokens] fp32, 16-byte chunks
+      // swizzled by (row & 15); the pipeline buffers are idle once the MMAs completed
+      float* part = reinterpret_cast<float*>(smem);
       for (int c = 0; c < TN; c += 16) {
         float v[16];
         tmem_ld16(taddr + c, v);
+        if (nkb == 0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) __stcg(mine + (c + j) * 128 + r, v[j]);
-      }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (etid == 0) *s_last = (atomicAdd(p.counters + tile, 1) == p.splits - 1) ? 1 : 0;
-      named_bar_sync(1, 128);
-      last = *s_last != 0;
-      if (last) __threadfence();
-    }
-    if (last) {
-      for (int c = 0; c < TN; c += 16) {
-        float v[16];
-        tmem_ld16(taddr + c, v);
-        if (p.splits > 1) {
-          float acc[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-          for (int s = 0; s < p.splits; ++s) {
-            if (s == split) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] += v[j];
-            } else {
-              const float* part = p.ws + static_cast<size_t>(tile * p.splits + s) * TN * 128;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] += __ldcg(part + (c + j) * 128 + r);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = acc[j];
+          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
         }
-        epi_apply<EPI>(p, v, fn, m0 + c, lane);
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const int chunk = ((c >> 2) + j4) ^ (r & 15);
+          *reinterpret_cast<float4*>(part + r * 64 + chunk * 4) =
+              make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+        }
       }
-      if (p.splits > 1 && etid == 0) p.counters[tile] = 0;
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      const int S = p.splits, RS = 128 / S;
+      const uint32_t rank = cluster_ctarank();
+      if (etid == 0) {
+        trace_stamp(p.trace, 6);
+        const uint32_t slice = static_cast<uint32_t>(RS * 64 * 4);
+        const uint32_t src = smem_u32(part), dst = smem_u32(recv) + rank * slice;
+        for (int q = 0; q < S; ++q)
+          bulk_copy_to_peer(mapa_shared(dst, q), src + q * slice, slice, mapa_shared(recv_bar, q));
+        bulk_commit();
+      }
+      mbar_wait(recv_bar, 0, p.err);
+      if (etid == 0) trace_stamp(p.trace, 7);
+      const int row0 = static_cast<int>(rank) * RS;
+      const int fbase = n_tile * G::BM + row0;
+      const int contrib = n_tile * S + static_cast<int>(rank);
+      const float* rv = p.rstat_in ? s_rinv : nullptr;
+      switch (S) {
+        case 1: push_reduce<EPI, 1>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+        case 2: push_reduce<EPI, 2>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+        case 4: push_reduce<EPI, 4>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+        case 8: push_reduce<EPI, 8>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+        default: push_reduce<EPI, 16>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+      }
+      if (etid == 0) {
+        trace_stamp(p.trace, 8);
+        bulk_wait_all();                     // own outgoing copies finished before exit
+      }
+    } else if (cluster_red) {
+      // partial tile -> own shared memory, [token][row] fp32 (the pipeline buffers are idle)
+      float* part = reinterpret_cast<float*>(smem);
+      for (int c = 0; c < TN; c += 16) {
+        float v[16];
+        tmem_ld16(taddr + c, v);
+        if (nkb == 0) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) part[(c + j) * 128 + r] = v[j];
+      }
+    } else {
+      bool last = true;
+      if (p.splits > 1) {
+        float* mine = p.ws + static_cast<size_t>(tile * p.splits + split) * TN * 128;
+        for (int c = 0; c < TN; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(mine + (c + j) * 128 + r, v[j]);
+        }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (etid == 0) *s_last = (atomicAdd(p.counters + tile, 1) == p.splits - 1) ? 1 : 0;
+        named_bar_sync(1, 128);
+        last = *s_last != 0;
+        if (last) __threadfence();
+      }
+      if (last) {
+        for (int c = 0; c < TN; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + c, v);
+          if (p.splits > 1) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+            for (int s = 0; s < p.splits; ++s) {
+              if (s == split) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] += v[j];
+              } else {
+                const float* prt = p.ws + static_cast<size_t>(tile * p.splits + s) * TN * 128;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] += __ldcg(prt + (c + j) * 128 + r);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = acc[j];
+          }
+          epi_apply<EPI>(p, v, fn, m0 + c, lane);
+        }
+        if (p.splits > 1 && etid == 0) p.counters[tile] = 0;
+      }
     }
+  }
+
+  if (cluster_red && !push) {
+    if (threadIdx.x == 64) trace_stamp(p.trace, 6);
+    cluster_sync_all();                      // every partial tile is in its CTA's smem
+    if (threadIdx.x == 64) trace_stamp(p.trace, 7);
+    if (warp >= 2) {
+      const int etid = (warp - 2) * 32 + lane;
+      const int row0 = static_cast<int>(cluster_ctarank()) * (128 / p.splits);
+      const uint32_t part = smem_u32(smem);
+      const int m0 = m_tile * TN, fbase = n_tile * G::BM + row0;
+      switch (p.splits) {
+        case 2: cluster_reduce<EPI, TN, 2>(p, part, etid, row0, fbase, m0); break;
+        case 4: cluster_reduce<EPI, TN, 4>(p, part, etid, row0, fbase, m0); break;
+        case 8: cluster_reduce<EPI, TN, 8>(p, part, etid, row0, fbase, m0); break;
+        default: cluster_reduce<EPI, TN, 16>(p, part, etid, row0, fbase, m0); break;
+      }
+    }
+    if (threadIdx.x == 64) trace_stamp(p.trace, 8);
+    cluster_sync_all();                      // peers finished reading this CTA's smem
+    if (threadIdx.x == 64) trace_stamp(p.trace, 9);
   }
 
   tc_fence_before();
@@ -281,86 +585,154 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem, G::TMEM_COLS);
   }
+  if (threadIdx.x == 0) trace_stamp(p.trace, 10);
 }
 
-template <int TN, int EPI>
+template <int TN, int EPI, bool CL>
 static cudaError_t configure_one() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(GemmCfg<TN>::SMEM));
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(GemmCfg<TN, CL>::SMEM));
+  if (e == cudaSuccess && CL)
+    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
-template <int TN>
+template <int TN, bool CL>
 static cudaError_t configure_tn() {
   cudaError_t e;
-  if ((e = configure_one<TN, EPI_RESID>()) != cudaSuccess) return e;
-  if ((e = configure_one<TN, EPI_QKV>()) != cudaSuccess) return e;
-  if ((e = configure_one<TN, EPI_GEGLU>()) != cudaSuccess) return e;
-  if ((e = configure_one<TN, EPI_SWISH_VEC>()) != cudaSuccess) return e;
-  if ((e = configure_one<TN, EPI_BIAS_STORE>()) != cudaSuccess) return e;
-  return configure_one<TN, EPI_STORE>();
+  if ((e = configure_one<TN, EPI_RESID, CL>()) != cudaSuccess) return e;
+  if ((e = configure_one<TN, EPI_QKV, CL>()) != cudaSuccess) return e;
+  if ((e = configure_one<TN, EPI_GEGLU, CL>()) != cudaSuccess) return e;
+  if ((e = configure_one<TN, EPI_SWISH_VEC, CL>()) != cudaSuccess) return e;
+  if ((e = configure_one<TN, EPI_BIAS_STORE, CL>()) != cudaSuccess) return e;
+  return configure_one<TN, EPI_STORE, CL>();
 }
 
-// Sets the shared-memory carve-out of every instantiation once, outside any capture.
+// Sets the shared-memory carve-out (and the non-portable cluster size) of every
+// instantiation once, outside any capture.
 cudaError_t configure_gemm_kernels() {
   static cudaError_t done = cudaErrorNotReady;
   if (done == cudaSuccess) return done;
   cudaError_t e;
-  if ((e = configure_tn<64>()) != cudaSuccess) return e;
-  if ((e = configure_tn<128>()) != cudaSuccess) return e;
-  if ((e = configure_tn<256>()) != cudaSuccess) return e;
+  if ((e = configure_tn<64, false>()) != cudaSuccess) return e;
+  if ((e = configure_tn<128, false>()) != cudaSuccess) return e;
+  if ((e = configure_tn<256, false>()) != cudaSuccess) return e;
+  if ((e = configure_tn<64, true>()) != cudaSuccess) return e;
+  if ((e = configure_tn<128, true>()) != cudaSuccess) return e;
+  if ((e = configure_tn<256, true>()) != cudaSuccess) return e;
   done = cudaSuccess;
   return done;
 }
 
-template <int TN, int EPI>
+// Largest cluster (power of two <= 16) that the device can co-schedule for the
+// TN-token kernel.
+int gemm_max_cluster(int tn) {
+  if (configure_gemm_kernels() != cudaSuccess) return 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(192, 1, 1);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int best = 1;
+  for (int c = 16; c >= 2; c >>= 1) {
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = c;
+    cfg.gridDim = dim3(1, 1, c);
+    int n = 0;
+    cudaError_t e;
+    switch (tn) {
+      case 64:
+        cfg.dynamicSmemBytes = GemmCfg<64, true>::SMEM;
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<64, EPI_RESID, true>, &cfg);
+        break;
+      case 128:
+        cfg.dynamicSmemBytes = GemmCfg<128, true>::SMEM;
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<128, EPI_RESID, true>, &cfg);
+        break;
+      default:
+        cfg.dynamicSmemBytes = GemmCfg<256, true>::SMEM;
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<256, EPI_RESID, true>, &cfg);
+        break;
+    }
+    if (e == cudaSuccess && n > 0) {
+      best = c;
+      break;
+    }
+    cudaGetLastError();
+  }
+  return best;
+}
+
+template <int TN, int EPI, bool CL>
 static cudaError_t launch_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
                               int n_tiles, int m_tiles, cudaStream_t s, bool pdl) {
-  using G = GemmCfg<TN>;
+  using G = GemmCfg<TN, CL>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles, m_tiles, p.splits);
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = G::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (CL) {
+    // always an explicit cluster (also of size 1): the cluster-mode code paths use
+    // cluster-scope instructions (barrier.cluster, mapa, bulk copies to shared::cluster)
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = p.splits;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI>, tm_w, tm_x, p);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI, CL>, tm_w, tm_x, p);
 }
 
-template <int TN>
+template <int TN, bool CL>
 static cudaError_t launch_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                              const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s,
                              bool pdl) {
   switch (epi) {
-    case EPI_RESID: return launch_one<TN, EPI_RESID>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case EPI_QKV: return launch_one<TN, EPI_QKV>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case EPI_GEGLU: return launch_one<TN, EPI_GEGLU>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case EPI_SWISH_VEC:
-      return launch_one<TN, EPI_SWISH_VEC>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case EPI_BIAS_STORE:
-      return launch_one<TN, EPI_BIAS_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case EPI_STORE: return launch_one<TN, EPI_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_RESID: return launch_one<TN, EPI_RESID, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_QKV: return launch_one<TN, EPI_QKV, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_GEGLU: return launch_one<TN, EPI_GEGLU, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_SWISH_VEC: return launch_one<TN, EPI_SWISH_VEC, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_BIAS_STORE: return launch_one<TN, EPI_BIAS_STORE, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case EPI_STORE: return launch_one<TN, EPI_STORE, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                        const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl) {
+                        const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl,
+                        bool cluster) {
+  if (cluster && (p.splits & (p.splits - 1))) return cudaErrorInvalidValue;   // power of two
   switch (tn) {
-    case 64: return launch_tn<64>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case 128: return launch_tn<128>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case 256: return launch_tn<256>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 64:
+      return cluster ? launch_tn<64, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
+                     : launch_tn<64, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 128:
+      return cluster ? launch_tn<128, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
+                     : launch_tn<128, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 256:
+      return cluster ? launch_tn<256, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
+                     : launch_tn<256, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
 
 size_t gemm_smem_bytes(int tn) {
   switch (tn) {
-    case 64: return GemmCfg<64>::SMEM;
-    case 128: return GemmCfg<128>::SMEM;
-    case 256: return GemmCfg<256>::SMEM;
+    case 64: return GemmCfg<64, false>::SMEM;
+    case 128: return GemmCfg<128, false>::SMEM;
+    case 256: return GemmCfg<256, false>::SMEM;
     default: return 0;
   }
 }

@@ -49,14 +49,35 @@ struct GemmParams {
   int kcap, dyn_off, seq, n_heads, head_dim;
   const float* rope;  // [seq][D/2][2] (cos, sin) at positions pos0 + s
   int has_state;      // EPI_BIAS_STORE: skip row s == 0 of each observation
+  // Single 64-token tile path (cluster mode), norms folded into the neighbouring GEMMs:
+  //  residual writers (EPI_RESID / EPI_BIAS_STORE) also write z = bf16(resid * (1 + zmod))
+  //  ([m][ld_resid]; zmod = AdaRMSNorm scale or RMSNorm weight of the next norm, null: no
+  //  z) and per-token sums of squares to rstat_out[(rstat_slot0 + contributor) * ld_rstat + m];
+  //  z consumers (EPI_QKV / EPI_GEGLU) scale their product by
+  //  rinv = 1/sqrt(sum of rstat_n rows of rstat_in / k_dim + eps), then add cvec[n] (the
+  //  weights times the AdaRMSNorm shift; null: 0).
+  float* rstat_out;
+  int rstat_slot0, ld_rstat;
+  bf16* zout;
+  const float* zmod;
+  const float* rstat_in;
+  int rstat_n;
+  const float* cvec;
+  float eps;
   float* ws;          // split-K partial tiles
   int* counters;      // one arrival counter per output tile (left at 0)
   int* err;           // device status word
+  unsigned long long* trace;   // optional: [ctas][16] %globaltimer stamps, or null
 };
 
-// tn: token tile (64, 128 or 256). Returns cudaSuccess or the launch error.
+// tn: token tile (64, 128 or 256). cluster = false: split partials through p.ws /
+// p.counters (any split count); cluster = true: the splits (a power of two, at most
+// gemm_max_cluster(tn)) of a tile form a cluster and reduce in distributed shared memory.
 cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                        const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl);
+                        const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl,
+                        bool cluster = false);
+
+int gemm_max_cluster(int tn);
 size_t gemm_smem_bytes(int tn);
 cudaError_t configure_gemm_kernels();
 int gemm_stages(int tn);
@@ -73,12 +94,11 @@ struct AttnParams {
   int ring_off;         // first ring slot row (= n_static_max)
   int dyn_off;          // first dynamic row (= n_static_max + n_sliding)
   int has_state;        // row s == 0 sees the prefix and itself only
-  int n_splits;         // key splits (grid.y)
-  float* part_o;        // split partials [B][q_tiles][n_splits][64][D] fp32
-  float* part_ml;       // [B][q_tiles][n_splits][64][2]
-  int* counters;        // [B][q_tiles], left at 0
+  int n_splits;         // key splits (grid.y): 1, or a power of two <= 16 forming one
+                        // cluster per query tile (partials merged in shared memory)
   float scale_log2;     // log2(e) / sqrt(D)
   int* err;
+  unsigned long long* trace;   // optional: [ctas][16] %globaltimer stamps, or null
 };
 
 cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
@@ -86,11 +106,12 @@ cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q
 int attn_q_tile();                       // query rows per CTA
 cudaError_t configure_attention_kernels();
 int attn_key_tile(int head_dim);         // keys per pipeline stage
+int attn_max_cluster(int head_dim);      // largest co-schedulable split cluster
 
 // -------------------------------------------------------------- small kernels
 
 struct NormParams {
-  const float* x;       // [M][W]
+  const float* x;       // [M][W], W a multiple of 128 and <= 2048
   bf16* y;              // [M][W]
   const float* scale;   // AdaRMSNorm scale [W] (null for plain)
   const float* shift;   // AdaRMSNorm shift [W]
@@ -103,13 +124,16 @@ cudaError_t launch_norm(const NormParams& p, cudaStream_t s, bool pdl);
 struct EmbedParams {
   const float* x;        // Euler state [B][C][A]
   const float* state;    // [B][Sd] or null
-  const float* w_in;     // action_in [W][A] fp32
+  const float* w_in;     // action_in, transposed: [A][W] fp32
   const float* b_in;     // [W]
-  const float* w_st;     // state_in [W][Sd]
+  const float* w_st;     // state_in, transposed: [Sd][W]
   const float* b_st;
   float* resid;          // [B*S][W]
   bf16* e_out;           // Pi0: bf16 action embedding [B*S][W] (state rows zeroed), else null
   int B, C, A, S, Sd, W, has_state;
+  float* rstat;          // optional: per-row sum of squares of the residual rows written
+  bf16* zout;            // optional: z = bf16(resid * (1 + zmod)) for the rows written
+  const float* zmod;
 };
 cudaError_t launch_embed(const EmbedParams& p, cudaStream_t s, bool pdl);
 
@@ -128,9 +152,9 @@ cudaError_t launch_final(const FinalParams& p, cudaStream_t s, bool pdl);
 
 // Time tables: temb[k][Td] for t_k = 1 - k/steps.
 cudaError_t launch_temb(float* temb, int steps, int time_dim, cudaStream_t s);
-// y[r][o] = act(sum_i x[r][i] * w[o * ldw + i] + b[o]), r < rows, o < n_out.
-cudaError_t launch_rowgemv(const float* x, int rows, int n_in, const bf16* w, long ldw,
-                           const bf16* b, int n_out, float* y, int act_swish, cudaStream_t s);
+// y[r * ldy + o] = act(sum_i x[r * ldx + i] * w[o * ldw + i] + b[o]), r < rows, o < n_out.
+cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const bf16* w, long ldw,
+                           const bf16* b, int n_out, float* y, long ldy, int act_swish, cudaStream_t s);
 
 // Cache maintenance.
 cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L,

@@ -36,7 +36,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // ------------------------------------------------------------------------- norm
-// One warp per token row; W is a multiple of 128 so each lane moves float4s.
+// One warp per token row. The whole row (W <= 128 * NV floats) is loaded into registers
+// with all loads in flight at once, reduced with shuffles, then modulated and stored.
+template <int NV>
 __global__ void __launch_bounds__(128) norm_kernel(const NormParams p) {
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
@@ -44,17 +46,23 @@ __global__ void __launch_bounds__(128) norm_kernel(const NormParams p) {
   const int row = blockIdx.x * 4 + warp;
   if (row >= p.M) return;
   const float* x = p.x + static_cast<size_t>(row) * p.W;
+  const int nv = p.W / 128;
+  float4 v[NV];
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+    if (k < nv) v[k] = *reinterpret_cast<const float4*>(x + k * 128 + lane * 4);
   float ss = 0.0f;
-  for (int i = lane * 4; i < p.W; i += 128) {
-    const float4 v = *reinterpret_cast<const float4*>(x + i);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
+#pragma unroll
+  for (int k = 0; k < NV; ++k)
+    if (k < nv) ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / static_cast<float>(p.W) + p.eps);
   bf16* y = p.y + static_cast<size_t>(row) * p.W;
-  for (int i = lane * 4; i < p.W; i += 128) {
-    const float4 v = *reinterpret_cast<const float4*>(x + i);
-    float o[4] = {v.x * r, v.y * r, v.z * r, v.w * r};
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    if (k >= nv) break;
+    const int i = k * 128 + lane * 4;
+    float o[4] = {v[k].x * r, v[k].y * r, v[k].z * r, v[k].w * r};
     if (p.scale) {
       const float4 sc = *reinterpret_cast<const float4*>(p.scale + i);
       const float4 sh = *reinterpret_cast<const float4*>(p.shift + i);
@@ -81,12 +89,18 @@ __global__ void __launch_bounds__(128) norm_kernel(const NormParams p) {
 cudaError_t launch_norm(const NormParams& p, cudaStream_t s, bool pdl) {
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3((p.M + 3) / 4), dim3(128), 0, s, attr, pdl);
-  return cudaLaunchKernelEx(&cfg, norm_kernel, p);
+  if (p.W <= 256) return cudaLaunchKernelEx(&cfg, norm_kernel<2>, p);
+  if (p.W <= 512) return cudaLaunchKernelEx(&cfg, norm_kernel<4>, p);
+  if (p.W <= 1024) return cudaLaunchKernelEx(&cfg, norm_kernel<8>, p);
+  if (p.W <= 2048) return cudaLaunchKernelEx(&cfg, norm_kernel<16>, p);
+  return cudaErrorInvalidValue;
 }
 
 // ------------------------------------------------------------------------ embed
 // One CTA per suffix row. State row: state_in(state); action rows: action_in(x), both
-// fp32. Pi0 routes the action embedding (bf16) into the action-time MLP instead.
+// fp32, with the maps stored transposed ([in][W]) so a warp reads 32 consecutive output
+// features per input element. Pi0 routes the action embedding (bf16) into the
+// action-time MLP instead of the residual.
 __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
   __shared__ float vin[256];
   if (threadIdx.x == 0) pdl_trigger();
@@ -97,19 +111,34 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
   const int len = st ? p.Sd : p.A;
   const float* src = st ? p.state + static_cast<size_t>(b) * p.Sd
                         : p.x + (static_cast<size_t>(b) * p.C + (s - p.has_state)) * p.A;
-  const float* w = st ? p.w_st : p.w_in;
+  const float* wt = st ? p.w_st : p.w_in;     // [len][W]
   const float* bias = st ? p.b_st : p.b_in;
   for (int i = threadIdx.x; i < len; i += blockDim.x) vin[i] = src[i];
   __syncthreads();
+  float ss = 0.0f;
   for (int n = threadIdx.x; n < p.W; n += blockDim.x) {
-    const float* wr = w + static_cast<size_t>(n) * len;
     float acc = bias[n];
-    for (int a = 0; a < len; ++a) acc = fmaf(wr[a], vin[a], acc);
+#pragma unroll 8
+    for (int a = 0; a < len; ++a) acc = fmaf(wt[static_cast<size_t>(a) * p.W + n], vin[a], acc);
     if (p.e_out && !st) {
       p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(acc);
     } else {
       p.resid[static_cast<size_t>(m) * p.W + n] = acc;
+      ss += acc * acc;
+      if (p.zout) p.zout[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(acc * (1.0f + p.zmod[n]));
       if (p.e_out) p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(0.0f);
+    }
+  }
+  if (p.rstat) {
+    // sum of squares of the residual row written here (0 for rows left to the time MLP)
+    __shared__ float red[8];
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.0f;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+      p.rstat[m] = t;
     }
   }
 }
@@ -131,6 +160,7 @@ __global__ void __launch_bounds__(256) final_kernel(const FinalParams p) {
   const int b = bc / p.C, c = bc - b * p.C;
   const float* xr = p.resid + (static_cast<size_t>(b) * p.S + p.has_state + c) * p.W;
   float ss = 0.0f;
+#pragma unroll 4
   for (int i = threadIdx.x; i < p.W; i += blockDim.x) {
     const float v = xr[i];
     y[i] = v;
@@ -152,6 +182,7 @@ __global__ void __launch_bounds__(256) final_kernel(const FinalParams p) {
   for (int a = warp; a < p.A; a += 8) {
     const float* wr = p.w_out + static_cast<size_t>(a) * p.W;
     float acc = 0.0f;
+#pragma unroll 8
     for (int i = lane; i < p.W; i += 32) acc = fmaf(wr[i], y[i], acc);
     acc = warp_sum(acc);
     if (lane == 0) {
@@ -189,9 +220,9 @@ cudaError_t launch_temb(float* temb, int steps, int time_dim, cudaStream_t s) {
 }
 
 // One warp per output feature, 8 rows (time steps) at a time.
-__global__ void __launch_bounds__(256) rowgemv_kernel(const float* x, int rows, int n_in,
+__global__ void __launch_bounds__(256) rowgemv_kernel(const float* x, int rows, int n_in, long ldx,
                                                       const bf16* w, long ldw, const bf16* bvec,
-                                                      int n_out, float* y, int act_swish) {
+                                                      int n_out, float* y, long ldy, int act_swish) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o = blockIdx.x * 8 + warp;
   if (o >= n_out) return;
@@ -205,20 +236,20 @@ __global__ void __launch_bounds__(256) rowgemv_kernel(const float* x, int rows, 
       const float wv = __bfloat162float(wr[i]);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (r0 + j < rows) acc[j] = fmaf(wv, x[static_cast<size_t>(r0 + j) * n_in + i], acc[j]);
+        if (r0 + j < rows) acc[j] = fmaf(wv, x[static_cast<size_t>(r0 + j) * ldx + i], acc[j]);
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float v = warp_sum(acc[j]) + bias;
       if (lane == 0 && r0 + j < rows)
-        y[static_cast<size_t>(r0 + j) * n_out + o] = act_swish ? swishf(v) : v;
+        y[static_cast<size_t>(r0 + j) * ldy + o] = act_swish ? swishf(v) : v;
     }
   }
 }
 
-cudaError_t launch_rowgemv(const float* x, int rows, int n_in, const bf16* w, long ldw,
-                           const bf16* b, int n_out, float* y, int act_swish, cudaStream_t s) {
-  rowgemv_kernel<<<(n_out + 7) / 8, 256, 0, s>>>(x, rows, n_in, w, ldw, b, n_out, y, act_swish);
+cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const bf16* w, long ldw,
+                           const bf16* b, int n_out, float* y, long ldy, int act_swish, cudaStream_t s) {
+  rowgemv_kernel<<<(n_out + 7) / 8, 256, 0, s>>>(x, rows, n_in, ldx, w, ldw, b, n_out, y, ldy, act_swish);
   return cudaGetLastError();
 }
 
