@@ -393,12 +393,29 @@ GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
 
 int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensorMap& tw,
                  const CUtensorMap& tx, GemmParams p, int n_feat, int k_dim, int M, bool pdl) {
+  if (M > 64) {
+    // several token tiles: persistent kernel, one CTA per SM, no K split
+    const GemmPlan g0 = plan_gemm(n_feat, k_dim, M, h->sm_count);
+    p.n_feat = n_feat;
+    p.k_dim = k_dim;
+    p.m_tok = M;
+    p.splits = 1;
+    p.kb_per_split = k_dim / 64;
+    p.w_stream = 0;
+    p.err = h->err;
+    const int total = g0.n_tiles * g0.m_tiles;
+    rec.begin(kind);
+    CU(launch_gemm_persistent(g0.tn, epi, tw, tx, p, g0.n_tiles, g0.m_tiles, std::min(total, h->sm_count), rec.s,
+                              pdl));
+    return rec.end(kind);
+  }
   const GemmPlan g = denoise_plan(h, n_feat, k_dim, M);
   p.n_feat = n_feat;
   p.k_dim = k_dim;
   p.m_tok = M;
   p.splits = g.splits;
   p.kb_per_split = g.kb_per_split;
+  p.w_stream = g.m_tiles == 1 ? 1 : 0;   // weights reused by every token tile stay in L2
   p.err = h->err;
   p.ld_rstat = h->max_M;
   rec.begin(kind);
@@ -1141,6 +1158,7 @@ int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, in
   p.m_tok = m_tok;
   p.splits = g.splits;
   p.kb_per_split = g.kb_per_split;
+  p.w_stream = g.m_tiles == 1 ? 1 : 0;
   p.resid = Y;
   p.ld_resid = n_feat;
   p.ws = static_cast<float*>(scratch);
@@ -1234,6 +1252,7 @@ extern "C" int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float
   p.m_tok = m_tok;
   p.splits = g.splits;
   p.kb_per_split = g.kb_per_split;
+  p.w_stream = g.m_tiles == 1 ? 1 : 0;
   p.resid = Y;
   p.ld_resid = n_feat;
   p.ws = scratch;

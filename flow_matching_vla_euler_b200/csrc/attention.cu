@@ -418,7 +418,7 @@ static cudaError_t launch_d(const AttnParams& p, int batch, int q_tiles, cudaStr
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(q_tiles, p.n_splits, batch);
   cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.dynamicSmemBytes = p.n_splits > 1 ? C::SMEM : C::MAIN;   // receive buffers only when merging
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   int na = 0;

@@ -44,15 +44,15 @@ template <int EPI>
 __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], int fn, int mb,
                                           int lane) {
   if constexpr (EPI == EPI_RESID) {
+    // all 16 residual values are loaded before any store (no load-store serialisation)
     const float g = p.vec ? p.vec[fn] : 1.0f;
+    float* base = p.resid + static_cast<size_t>(mb) * p.ld_resid + fn;
+    float old[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int m = mb + j;
-      if (m < p.m_tok) {
-        float* dst = p.resid + static_cast<size_t>(m) * p.ld_resid + fn;
-        *dst = *dst + g * v[j];
-      }
-    }
+    for (int j = 0; j < 16; ++j) old[j] = (mb + j < p.m_tok) ? base[static_cast<size_t>(j) * p.ld_resid] : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (mb + j < p.m_tok) base[static_cast<size_t>(j) * p.ld_resid] = fmaf(g, v[j], old[j]);
   } else if constexpr (EPI == EPI_BIAS_STORE) {
     const float b = p.vec[fn];
 #pragma unroll
@@ -76,14 +76,19 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
         p.out[static_cast<size_t>(m) * p.ld_out + fn] = __float2bfloat16_rn(swishf(v[j] + b));
     }
   } else if constexpr (EPI == EPI_GEGLU) {
-    // packed rows: 2f = gate feature f, 2f + 1 = up feature f
+    // packed rows: 2f = gate feature f (even lane), 2f + 1 = up feature f (odd lane).
+    // The two lanes of a pair split the 16 tokens: the even lane finishes tokens 0..7,
+    // the odd lane tokens 8..15, each after swapping the halves it lacks.
+    const bool odd = lane & 1;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float up = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      const int m = mb + j;
-      if (!(lane & 1) && m < p.m_tok)
-        p.out[static_cast<size_t>(m) * p.ld_out + (fn >> 1)] =
-            __float2bfloat16_rn(gelu_tanhf(v[j]) * up);
+    for (int j = 0; j < 8; ++j) {
+      const float send = odd ? v[j] : v[j + 8];        // up[0..7] to even, gate[8..15] to odd
+      const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+      const float g = odd ? got : v[j];
+      const float u = odd ? v[j + 8] : got;
+      const int m = mb + j + (odd ? 8 : 0);
+      if (m < p.m_tok)
+        p.out[static_cast<size_t>(m) * p.ld_out + (fn >> 1)] = __float2bfloat16_rn(gelu_tanhf(g) * u);
     }
   } else if constexpr (EPI == EPI_QKV) {
     // packed rows: 2i / 2i+1 = dims (i, i + D/2) of one head of Q, then K, then V
@@ -105,31 +110,43 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
       i = 0;
     }
     const int dim = i + second * DH;
+    // token mb + j -> (observation, suffix position), stepped without a division per token
+    int b0 = mb / p.seq, s0 = mb - b0 * p.seq;
+    int bj[16], sj[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      bj[j] = b0;
+      sj[j] = s0;
+      if (++s0 == p.seq) {
+        s0 = 0;
+        ++b0;
+      }
+    }
+    float2 cs[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      cs[j] = (kind < 2 && mb + j < p.m_tok) ? reinterpret_cast<const float2*>(p.rope)[sj[j] * DH + i]
+                                              : make_float2(1.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
       const int m = mb + j;
       if (m >= p.m_tok || kind == 3) continue;
-      const int b = m / p.seq, s = m - b * p.seq;
-      float val = v[j];
-      if (kind < 2) {
-        const float2 cs = reinterpret_cast<const float2*>(p.rope)[s * DH + i];
-        // first half: x1 c - x2 s; second half: x2 c + x1 s (own value first)
-        val = second ? fmaf(v[j], cs.x, other * cs.y) : fmaf(v[j], cs.x, -other * cs.y);
-      }
+      // first half: x1 c - x2 s; second half: x2 c + x1 s (own value first); V unrotated
+      const float val = kind == 2 ? v[j]
+                                  : (second ? fmaf(v[j], cs[j].x, other * cs[j].y)
+                                            : fmaf(v[j], cs[j].x, -other * cs[j].y));
       const bf16 o = __float2bfloat16_rn(val);
       if (kind == 0)
         p.out[static_cast<size_t>(m) * p.ld_out + head * D + dim] = o;
       else if (kind == 1)
-        p.kc[(static_cast<size_t>(b) * p.kcap + p.dyn_off + s) * D + dim] = o;
+        p.kc[(static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j]) * D + dim] = o;
       else
-        p.vc[(static_cast<size_t>(b) * p.kcap + p.dyn_off + s) * D + dim] = o;
+        p.vc[(static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j]) * D + dim] = o;
     }
   }
 }
 
-// Epilogue on one pair of adjacent output rows (2i, 2i + 1) at one token, used by the
-// cluster reduction; the pair is the unit the GeGLU and rotary epilogues need.
 template <int EPI>
 __device__ __forceinline__ void epi_pair(const GemmParams& p, int fn0, int m, float v0, float v1) {
   if (m >= p.m_tok) return;
@@ -350,7 +367,7 @@ __global__ void __launch_bounds__(192, 1)
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
     // Weights are never written by earlier kernels: stream them right away.
-    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_w = p.w_stream ? policy_evict_first() : policy_evict_last();
     const int y_w = p.w_row0 + n_tile * G::BM;
     for (int i = 0; i < npre; ++i) {
       mbar_arrive_expect_tx(full0 + 8 * i, G::STAGE_BYTES);
@@ -373,7 +390,7 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_w = p.w_stream ? policy_evict_first() : policy_evict_last();
       const uint64_t pol_x = policy_evict_last();
       const int y_w = p.w_row0 + n_tile * G::BM;
       const int y_x = m_tile * TN;
@@ -588,6 +605,204 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) trace_stamp(p.trace, 10);
 }
 
+// ---------------------------------------------------------------------------------
+// Persistent variant for several token tiles (no K split): one CTA per SM walks the
+// output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... with the token tile varying
+// fastest (the weight tile stays hot in L2 across token tiles). TMA keeps a 4-stage ring
+// streaming across tile boundaries; the MMA warp alternates between two TMEM
+// accumulators, so the epilogue of one tile overlaps the main loop of the next.
+template <int TN>
+struct PersistCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = TN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = TN == 256 ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * TN;       // two accumulators
+  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+};
+
+template <int TN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        const GemmParams p, int n_tiles, int m_tiles) {
+  using G = PersistCfg<TN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + G::STAGES * G::A_BYTES;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2 * G::STAGES + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = p.k_dim / G::BK;
+  const int total = n_tiles * m_tiles;
+  const uint32_t full0 = smem_u32(&bar[0]);
+  const uint32_t empty0 = smem_u32(&bar[G::STAGES]);
+  const uint32_t tfull0 = smem_u32(&bar[2 * G::STAGES]);       // accumulator b filled
+  const uint32_t tempty0 = smem_u32(&bar[2 * G::STAGES + 2]);  // accumulator b drained
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < G::STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 1);
+    }
+    fence_mbar_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), G::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) pdl_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_last(), pol_x = policy_evict_last();
+      pdl_wait();
+      int g = 0;   // global k-block counter of this CTA (ring position)
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int m_tile = t % m_tiles, n_tile = t / m_tiles;
+        const int y_w = p.w_row0 + n_tile * G::BM, y_x = m_tile * TN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % G::STAGES;
+          if (g >= G::STAGES && !mbar_wait(empty0 + 8 * s, ((g / G::STAGES) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full0 + 8 * s, G::STAGE_BYTES);
+          tma_load_2d(smem_u32(sA + s * G::A_BYTES), &tm_w, full0 + 8 * s, kb * G::BK, y_w, pol_w);
+          tma_load_2d(smem_u32(sB + s * G::B_BYTES), &tm_x, full0 + 8 * s, kb * G::BK, y_x, pol_x);
+        }
+      }
+      // no copies left in flight: the last load of each used stage has landed
+      for (int s = 0; s < G::STAGES && s < g; ++s) {
+        const int last = s + ((g - 1 - s) / G::STAGES) * G::STAGES;
+        mbar_wait(full0 + 8 * s, (last / G::STAGES) & 1, p.err);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, TN);
+      int g = 0, lt = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++lt) {
+        const int b = lt & 1;
+        if (lt >= 2 && !mbar_wait(tempty0 + 8 * b, ((lt >> 1) - 1) & 1, p.err)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * TN);
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % G::STAGES;
+          if (!mbar_wait(full0 + 8 * s, (g / G::STAGES) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * G::A_BYTES));
+          const uint64_t db = sdesc_k_sw128(smem_u32(sB + s * G::B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < G::BK / 16; ++kk)
+            umma_bf16(acc, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(empty0 + 8 * s);
+        }
+        umma_commit(tfull0 + 8 * b);   // signalled even after a timeout: no waiter hangs
+      }
+    }
+    __syncwarp();
+  } else {
+    pdl_wait();
+    const int q = warp & 3, r = q * 32 + lane, etid = (warp - 2) * 32 + lane;
+    int lt = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      const int m_tile = t % m_tiles, n_tile = t / m_tiles;
+      if (!mbar_wait(tfull0 + 8 * b, (lt >> 1) & 1, p.err)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * TN);
+      const int fn = n_tile * G::BM + r, m0 = m_tile * TN;
+      for (int c = 0; c < TN; c += 32) {
+        float v[32];
+        tmem_ld32(taddr + c, v);
+        epi_apply<EPI>(p, *reinterpret_cast<float(*)[16]>(&v[0]), fn, m0 + c, lane);
+        epi_apply<EPI>(p, *reinterpret_cast<float(*)[16]>(&v[16]), fn, m0 + c + 16, lane);
+      }
+      tc_fence_before();
+      named_bar_sync(1, 128);
+      if (etid == 0) mbar_arrive(tempty0 + 8 * b);   // accumulator b may be overwritten
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G::TMEM_COLS);
+  }
+}
+
+template <int TN, int EPI>
+static cudaError_t launch_persist_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
+                                      int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = PersistCfg<TN>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_persist_kernel<TN, EPI>, tm_w, tm_x, p, n_tiles, m_tiles);
+}
+
+template <int TN>
+static cudaError_t launch_persist_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
+                                     int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+  switch (epi) {
+    case EPI_RESID: return launch_persist_one<TN, EPI_RESID>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_QKV: return launch_persist_one<TN, EPI_QKV>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_GEGLU: return launch_persist_one<TN, EPI_GEGLU>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_SWISH_VEC: return launch_persist_one<TN, EPI_SWISH_VEC>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_BIAS_STORE: return launch_persist_one<TN, EPI_BIAS_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_STORE: return launch_persist_one<TN, EPI_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                                   const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+  if (p.splits != 1) return cudaErrorInvalidValue;
+  switch (tn) {
+    case 128: return launch_persist_tn<128>(epi, tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case 256: return launch_persist_tn<256>(epi, tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int TN>
+static cudaError_t configure_persist_tn() {
+  cudaError_t e;
+  for (auto fn : {gemm_persist_kernel<TN, EPI_RESID>, gemm_persist_kernel<TN, EPI_QKV>,
+                  gemm_persist_kernel<TN, EPI_GEGLU>, gemm_persist_kernel<TN, EPI_SWISH_VEC>,
+                  gemm_persist_kernel<TN, EPI_BIAS_STORE>, gemm_persist_kernel<TN, EPI_STORE>})
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(PersistCfg<TN>::SMEM))) != cudaSuccess)
+      return e;
+  return cudaSuccess;
+}
+
 template <int TN, int EPI, bool CL>
 static cudaError_t configure_one() {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -620,6 +835,8 @@ cudaError_t configure_gemm_kernels() {
   if ((e = configure_tn<64, true>()) != cudaSuccess) return e;
   if ((e = configure_tn<128, true>()) != cudaSuccess) return e;
   if ((e = configure_tn<256, true>()) != cudaSuccess) return e;
+  if ((e = configure_persist_tn<128>()) != cudaSuccess) return e;
+  if ((e = configure_persist_tn<256>()) != cudaSuccess) return e;
   done = cudaSuccess;
   return done;
 }

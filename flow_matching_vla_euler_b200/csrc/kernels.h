@@ -39,6 +39,7 @@ struct GemmParams {
   int w_row0;         // first row of this weight in the stacked weight tensor map
   int splits;         // K splits (grid.z)
   int kb_per_split;   // 64-wide K blocks per split
+  int w_stream;       // 1: each weight tile is read once (L2 evict-first), 0: reused
   float* resid;       // fp32 residual [m][ld_resid]
   int ld_resid;
   const float* vec;   // gate / bias / time vector, indexed by output feature
@@ -78,6 +79,10 @@ cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensor
                         bool cluster = false);
 
 int gemm_max_cluster(int tn);
+// Persistent launch over n_tiles x m_tiles output tiles (splits must be 1), grid CTAs;
+// tn 128 or 256, two TMEM accumulators so epilogues overlap the next tile's main loop.
+cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                                   const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl);
 size_t gemm_smem_bytes(int tn);
 cudaError_t configure_gemm_kernels();
 int gemm_stages(int tn);
