@@ -177,6 +177,7 @@ struct vla_expert {
   float *x = nullptr, *state = nullptr, *resid = nullptr, *rope = nullptr;
   bf16 *hb = nullptr, *qb = nullptr, *ob = nullptr, *ub = nullptr, *eb = nullptr, *h1b = nullptr;
   bf16 *kc = nullptr, *vc = nullptr;
+  bf16* vtc = nullptr;   // transposed V cache [L][max_batch][D][kcap] (head_dim 256)
   CacheDesc* desc = nullptr;
   int* err = nullptr;
   // per-token sum-of-squares partials of the residual, [rstat_rows][max_M]: rstat_a feeds
@@ -190,6 +191,7 @@ struct vla_expert {
   int prefix_batch = 0, n_static = 0, n_ring = 0, head = 0;
 
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
+  CUtensorMap tm_q, tm_kc, tm_vt;   // tensor-core attention operands (head_dim 256)
 
   // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
   unsigned long long* trace = nullptr;
@@ -431,6 +433,8 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
   const int key_tiles_max = cdiv(h->cfg.n_static_max, attn_key_tile(h->D)) +
                             cdiv(h->cfg.n_sliding, attn_key_tile(h->D)) + cdiv(h->S, attn_key_tile(h->D));
   const AttnPlan ap = plan_attn(h->S * h->H, B, key_tiles_max, h->sm_count, h->attn_cluster);
+  // tensor-core attention once every 128-row query tile has a CTA of its own
+  const bool use_tc_attn = h->vtc && B * cdiv(h->S * h->H, attn_tc_q_tile()) >= h->sm_count;
   const float dt = -1.0f / static_cast<float>(steps);
   // All suffix tokens in one 64-token tile: the norms are fused into the QKV and gate/up
   // GEMMs, fed by per-token sum-of-squares partials from the residual writers.
@@ -527,6 +531,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.ld_out = h->HD;
           p.kc = h->kc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
           p.vc = h->vc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
+          p.vtc = h->vtc ? h->vtc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D : nullptr;
           p.kcap = h->kcap;
           p.dyn_off = h->dyn_off;
           p.seq = h->S;
@@ -559,7 +564,25 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           a.err = h->err;
           a.trace = tr(1);
           rec.begin(VLA_K_ATTN);
-          CU(launch_attention(h->D, a, B, ap.q_tiles, rec.s, pdl));
+          if (use_tc_attn) {
+            AttnTcParams t{};
+            t.out = h->ob;
+            t.cache = h->desc;
+            t.layer = l;
+            t.max_batch = h->cfg.max_batch;
+            t.kcap = h->kcap;
+            t.ring_off = h->ring_off;
+            t.dyn_off = h->dyn_off;
+            t.seq = h->S;
+            t.n_heads = h->H;
+            t.has_state = h->hs;
+            t.scale_log2 = a.scale_log2;
+            t.err = h->err;
+            t.trace = tr(1);
+            CU(launch_attention_tc(h->tm_q, h->tm_kc, h->tm_vt, t, B, rec.s, pdl));
+          } else {
+            CU(launch_attention(h->D, a, B, ap.q_tiles, rec.s, pdl));
+          }
           rec.end(VLA_K_ATTN);
           GemmParams o{};
           o.w_row0 = l * W;
@@ -748,9 +771,12 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   h->pi0 = !h->ada;
   h->Cd = cfg->time_kind == VLA_TIME_ADA_MLP ? h->W : h->Td;
   h->qkv_rows = cdiv((h->H + 2) * h->D, 128) * 128;
-  h->ring_off = cfg->n_static_max;
-  h->dyn_off = cfg->n_static_max + cfg->n_sliding;
-  h->kcap = h->dyn_off + h->S;
+  // cache rows per (layer, observation): static | ring | dynamic, each region starting on
+  // a 64-row boundary (tensor-core attention reads the transposed V cache with TMA, whose
+  // inner coordinate must be 16-byte aligned)
+  h->ring_off = cdiv(cfg->n_static_max, 64) * 64;
+  h->dyn_off = h->ring_off + cdiv(cfg->n_sliding, 64) * 64;
+  h->kcap = cdiv(h->dyn_off + h->S, 64) * 64;
   h->max_M = cfg->max_batch * h->S;
   h->gemm_cluster[0] = gemm_max_cluster(64);
   h->gemm_cluster[1] = gemm_max_cluster(128);
@@ -862,6 +888,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   const size_t cache_elems = static_cast<size_t>(L) * cfg->max_batch * h->kcap * D;
   if ((rc = dalloc(h, &h->kc, cache_elems))) return cleanup(rc);
   if ((rc = dalloc(h, &h->vc, cache_elems))) return cleanup(rc);
+  if (D == 256 && (rc = dalloc(h, &h->vtc, cache_elems))) return cleanup(rc);
   if ((rc = dalloc(h, &h->rope, static_cast<size_t>(h->S) * D))) return cleanup(rc);
   h->rstat_rows = (W / 128) * 32 + 2;
   if ((rc = dalloc(h, &h->rstat_a, static_cast<size_t>(h->rstat_rows) * h->max_M))) return cleanup(rc);
@@ -887,6 +914,13 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  if (h->vtc) {
+    const uint64_t rows = static_cast<uint64_t>(L) * cfg->max_batch;
+    if ((rc = make_tmap(&h->tm_q, h->qb, D, static_cast<uint64_t>(h->max_M) * H, 128))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_kc, h->kc, D, rows * h->kcap, 64))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_vt, h->vtc, h->kcap, rows * D, 256))) return cleanup(rc);
+    CU(configure_attention_tc_kernel());
+  }
   if (h->pi0) {
     if ((rc = make_tmap(&h->tm_w1a, h->w1a, W, W, 128))) return cleanup(rc);
     if ((rc = make_tmap(&h->tm_w2, h->w2, W, W, 128))) return cleanup(rc);
@@ -948,7 +982,7 @@ int vla_cache_set_prefix(vla_expert* h, const uint16_t* K, const uint16_t* V, in
     return fail(VLA_ERR_SHAPE, "n_tokens %d outside [0, %d]", n_tokens, h->cfg.n_static_max + h->cfg.n_sliding);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   CU(launch_prefix_set(reinterpret_cast<const bf16*>(K), reinterpret_cast<const bf16*>(V), n_tokens, batch, h->L,
-                       h->D, h->cfg.max_batch, h->kcap, h->cfg.n_static_max, h->kc, h->vc, s));
+                       h->D, h->cfg.max_batch, h->kcap, h->cfg.n_static_max, h->ring_off, h->kc, h->vc, h->vtc, s));
   const int n_static = std::min(n_tokens, h->cfg.n_static_max);
   const int n_ring = n_tokens - n_static;
   CU(launch_cache_update(h->desc, n_static, n_ring, h->rope, h->S, h->D, h->cfg.rope_base, s));
@@ -971,7 +1005,7 @@ int vla_cache_append_sliding(vla_expert* h, const uint16_t* K_tok, const uint16_
     return fail(VLA_ERR_SHAPE, "batch %d must equal the prefix batch %d", batch, h->prefix_batch);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   CU(launch_ring_append(reinterpret_cast<const bf16*>(K_tok), reinterpret_cast<const bf16*>(V_tok), batch, h->L,
-                        h->D, h->cfg.max_batch, h->kcap, h->ring_off + h->head, h->kc, h->vc, s));
+                        h->D, h->cfg.max_batch, h->kcap, h->ring_off + h->head, h->kc, h->vc, h->vtc, s));
   const int n_ring = std::min(h->n_ring + 1, h->cfg.n_sliding);
   if (n_ring != h->n_ring)
     CU(launch_cache_update(h->desc, h->n_static, n_ring, h->rope, h->S, h->D, h->cfg.rope_base, s));
@@ -1033,8 +1067,12 @@ int vla_cache_export(vla_expert* h, uint16_t* K_out, uint16_t* V_out, int batch,
     return fail(VLA_ERR_SHAPE, "batch %d outside [1, %d]", batch, h->cfg.max_batch);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   const int rows = h->cfg.n_static_max + h->cfg.n_sliding;
-  if (K_out) CU(launch_copy_region(h->kc, reinterpret_cast<bf16*>(K_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D, s));
-  if (V_out) CU(launch_copy_region(h->vc, reinterpret_cast<bf16*>(V_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D, s));
+  if (K_out)
+    CU(launch_copy_region(h->kc, reinterpret_cast<bf16*>(K_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D,
+                          h->cfg.n_static_max, h->ring_off, s));
+  if (V_out)
+    CU(launch_copy_region(h->vc, reinterpret_cast<bf16*>(V_out), h->L, batch, h->cfg.max_batch, h->kcap, rows, h->D,
+                          h->cfg.n_static_max, h->ring_off, s));
   if (head) *head = h->head;
   if (n_static) *n_static = h->n_static;
   if (n_ring) *n_ring = h->n_ring;

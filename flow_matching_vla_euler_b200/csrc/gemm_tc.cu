@@ -15,7 +15,8 @@
 // epilogue.
 //
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2..5 drain TMEM (tcgen05.ld) and run the epilogue. Every wait is
+// tcgen05.mma, warps 2..5 drain TMEM (tcgen05.ld) and run the epilogue (the persistent
+// variant below uses eight epilogue warps). Every wait is
 // bounded: on timeout the kernel sets the status word and winds down.
 #include <cstdio>
 
@@ -91,7 +92,9 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
         p.out[static_cast<size_t>(m) * p.ld_out + (fn >> 1)] = __float2bfloat16_rn(gelu_tanhf(g) * u);
     }
   } else if constexpr (EPI == EPI_QKV) {
-    // packed rows: 2i / 2i+1 = dims (i, i + D/2) of one head of Q, then K, then V
+    // packed rows: 2i / 2i+1 = dims (i, i + D/2) of one head of Q, then K, then V. A warp
+    // covers 16 consecutive pairs, which lie in one head region (D/2 is a multiple of 16),
+    // so the row kind below is the same for the whole warp.
     const int D = p.head_dim, DH = D >> 1, H = p.n_heads;
     const int pr = fn >> 1, second = fn & 1;
     int kind, head = 0, i;
@@ -106,8 +109,7 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
       kind = 2;
       i = pr - (H + 1) * DH;
     } else {
-      kind = 3;   // padding row
-      i = 0;
+      return;   // padding rows (whole warps)
     }
     const int dim = i + second * DH;
     // token mb + j -> (observation, suffix position), stepped without a division per token
@@ -122,27 +124,40 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
         ++b0;
       }
     }
+    if (kind == 2) {   // V: no rotation; cache row and transposed cache column
+      bf16* vrow = p.vc + dim;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (mb + j >= p.m_tok) break;
+        const size_t row = static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j];
+        const bf16 o = __float2bfloat16_rn(v[j]);
+        vrow[row * D] = o;
+        if (p.vtc) p.vtc[(static_cast<size_t>(bj[j]) * D + dim) * p.kcap + p.dyn_off + sj[j]] = o;
+      }
+      return;
+    }
+    const float2* rope = reinterpret_cast<const float2*>(p.rope) + i;
     float2 cs[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      cs[j] = (kind < 2 && mb + j < p.m_tok) ? reinterpret_cast<const float2*>(p.rope)[sj[j] * DH + i]
-                                              : make_float2(1.0f, 0.0f);
+    for (int j = 0; j < 16; ++j) cs[j] = mb + j < p.m_tok ? rope[sj[j] * DH] : make_float2(1.0f, 0.0f);
+    float o[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      const int m = mb + j;
-      if (m >= p.m_tok || kind == 3) continue;
-      // first half: x1 c - x2 s; second half: x2 c + x1 s (own value first); V unrotated
-      const float val = kind == 2 ? v[j]
-                                  : (second ? fmaf(v[j], cs[j].x, other * cs[j].y)
-                                            : fmaf(v[j], cs[j].x, -other * cs[j].y));
-      const bf16 o = __float2bfloat16_rn(val);
-      if (kind == 0)
-        p.out[static_cast<size_t>(m) * p.ld_out + head * D + dim] = o;
-      else if (kind == 1)
-        p.kc[(static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j]) * D + dim] = o;
-      else
-        p.vc[(static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j]) * D + dim] = o;
+      // first half: x1 c - x2 s; second half: x2 c + x1 s (own value first)
+      o[j] = second ? fmaf(v[j], cs[j].x, other * cs[j].y) : fmaf(v[j], cs[j].x, -other * cs[j].y);
+    }
+    if (kind == 0) {
+      bf16* dst = p.out + static_cast<size_t>(mb) * p.ld_out + head * D + dim;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (mb + j < p.m_tok) dst[static_cast<size_t>(j) * p.ld_out] = __float2bfloat16_rn(o[j]);
+    } else {
+      bf16* krow = p.kc + dim;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (mb + j < p.m_tok)
+          krow[(static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j]) * D] = __float2bfloat16_rn(o[j]);
     }
   }
 }
@@ -198,6 +213,11 @@ __device__ __forceinline__ void epi_pair(const GemmParams& p, int fn0, int m, fl
       dst = (kind == 1 ? p.kc : p.vc) + (static_cast<size_t>(b) * p.kcap + p.dyn_off + s) * D;
     dst[i] = __float2bfloat16_rn(o0);
     dst[i + DH] = __float2bfloat16_rn(o1);
+    if (kind == 2 && p.vtc) {
+      bf16* vt = p.vtc + static_cast<size_t>(b) * D * p.kcap + p.dyn_off + s;
+      vt[static_cast<size_t>(i) * p.kcap] = __float2bfloat16_rn(o0);
+      vt[static_cast<size_t>(i + DH) * p.kcap] = __float2bfloat16_rn(o1);
+    }
   }
 }
 
@@ -623,7 +643,7 @@ struct PersistCfg {
 };
 
 template <int TN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const GemmParams p, int n_tiles, int m_tiles) {
   using G = PersistCfg<TN>;
@@ -721,8 +741,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
+    // eight epilogue warps: two per TMEM lane quarter, each draining half of the columns
     pdl_wait();
-    const int q = warp & 3, r = q * 32 + lane, etid = (warp - 2) * 32 + lane;
+    const int ew = warp - 2, q = warp & 3, r = q * 32 + lane, etid = ew * 32 + lane;
+    const int c_begin = (ew >> 2) * (TN / 2);
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       const int b = lt & 1;
@@ -731,14 +753,14 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * TN);
       const int fn = n_tile * G::BM + r, m0 = m_tile * TN;
-      for (int c = 0; c < TN; c += 32) {
-        float v[32];
-        tmem_ld32(taddr + c, v);
-        epi_apply<EPI>(p, *reinterpret_cast<float(*)[16]>(&v[0]), fn, m0 + c, lane);
-        epi_apply<EPI>(p, *reinterpret_cast<float(*)[16]>(&v[16]), fn, m0 + c + 16, lane);
+#pragma unroll 1
+      for (int c = c_begin; c < c_begin + TN / 2; c += 16) {   // rolled: keeps the code small
+        float v[16];
+        tmem_ld16(taddr + c, v);
+        epi_apply<EPI>(p, v, fn, m0 + c, lane);
       }
       tc_fence_before();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 256);
       if (etid == 0) mbar_arrive(tempty0 + 8 * b);   // accumulator b may be overwritten
     }
   }
@@ -756,7 +778,7 @@ static cudaError_t launch_persist_one(const CUtensorMap& tm_w, const CUtensorMap
                                       int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
   cfg.dynamicSmemBytes = PersistCfg<TN>::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -47,6 +47,7 @@ struct GemmParams {
   int ld_out;
   bf16* kc;           // EPI_QKV: this layer's K cache [max_batch][kcap][D]
   bf16* vc;
+  bf16* vtc;          // EPI_QKV: this layer's transposed V cache [max_batch][D][kcap], or null
   int kcap, dyn_off, seq, n_heads, head_dim;
   const float* rope;  // [seq][D/2][2] (cos, sin) at positions pos0 + s
   int has_state;      // EPI_BIAS_STORE: skip row s == 0 of each observation
@@ -113,6 +114,22 @@ cudaError_t configure_attention_kernels();
 int attn_key_tile(int head_dim);         // keys per pipeline stage
 int attn_max_cluster(int head_dim);      // largest co-schedulable split cluster
 
+// Tensor-core attention (head_dim 256): one CTA per (128 query rows, observation), all
+// keys, no splits. tm_q over the query rows [rows][256], tm_k over the K cache
+// [L*max_batch*kcap][256], tm_vt over the transposed V cache [L*max_batch*256][kcap].
+struct AttnTcParams {
+  bf16* out;               // [B][S][H][256]
+  const CacheDesc* cache;
+  int layer, max_batch, kcap, ring_off, dyn_off, seq, n_heads, has_state;
+  float scale_log2;        // log2(e) / sqrt(D)
+  int* err;
+  unsigned long long* trace;   // optional: [ctas][16] %globaltimer stamps, or null
+};
+cudaError_t launch_attention_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vt,
+                                const AttnTcParams& p, int batch, cudaStream_t s, bool pdl);
+cudaError_t configure_attention_tc_kernel();
+int attn_tc_q_tile();
+
 // -------------------------------------------------------------- small kernels
 
 struct NormParams {
@@ -162,16 +179,17 @@ cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const b
                            const bf16* b, int n_out, float* y, long ldy, int act_swish, cudaStream_t s);
 
 // Cache maintenance.
-cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L,
-                              int D, int max_batch, int kcap, int n_static_max, bf16* kc,
-                              bf16* vc, cudaStream_t s);
+// vt: optional transposed V cache [L][max_batch][D][kcap] (null: none).
+cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L, int D, int max_batch,
+                              int kcap, int n_static_max, int ring_off, bf16* kc, bf16* vc, bf16* vt,
+                              cudaStream_t s);
 cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, int D,
-                               int max_batch, int kcap, int slot_row, bf16* kc, bf16* vc,
+                               int max_batch, int kcap, int slot_row, bf16* kc, bf16* vc, bf16* vt,
                                cudaStream_t s);
 // Writes the cache descriptor and the rotary table [seq][D/2][2] for pos0 = n_static+n_ring.
 cudaError_t launch_cache_update(CacheDesc* desc, int n_static, int n_ring, float* rope,
                                 int seq, int head_dim, float rope_base, cudaStream_t s);
 cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch,
-                               int kcap, int rows, int D, cudaStream_t s);
+                               int kcap, int rows, int D, int n_static_max, int ring_off, cudaStream_t s);
 
 }  // namespace vla

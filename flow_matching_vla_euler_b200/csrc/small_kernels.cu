@@ -254,10 +254,12 @@ cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const b
 }
 
 // ------------------------------------------------------------------- cache upkeep
-// K, V [L][batch][n][D] -> cache rows [0, n) of each (layer, observation): the static
-// region, then the ring slots 0.. (the ring starts right after the static capacity).
+// K, V [L][batch][n][D] -> cache rows of each (layer, observation): token j < n_static_max
+// goes to static row j, the rest to ring rows ring_off + (j - n_static_max). With a
+// transposed V cache (vt, [L][max_batch][D][kcap]) the V values are also written there.
 __global__ void prefix_set_kernel(const uint4* K, const uint4* V, int n, int batch, int L, int D8,
-                                  int max_batch, int kcap, uint4* kc, uint4* vc) {
+                                  int max_batch, int kcap, int n_static_max, int ring_off, uint4* kc, uint4* vc,
+                                  bf16* vt) {
   const size_t total = static_cast<size_t>(L) * batch * n * D8;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -267,45 +269,60 @@ __global__ void prefix_set_kernel(const uint4* K, const uint4* V, int n, int bat
     r /= n;
     const int b = static_cast<int>(r % batch);
     const int l = static_cast<int>(r / batch);
-    const size_t dst = ((static_cast<size_t>(l) * max_batch + b) * kcap + j) * D8 + c;
+    const int row = j < n_static_max ? j : ring_off + (j - n_static_max);
+    const size_t dst = ((static_cast<size_t>(l) * max_batch + b) * kcap + row) * D8 + c;
     kc[dst] = K[i];
-    vc[dst] = V[i];
+    const uint4 v = V[i];
+    vc[dst] = v;
+    if (vt) {
+      const bf16* e = reinterpret_cast<const bf16*>(&v);
+      const size_t base = ((static_cast<size_t>(l) * max_batch + b) * (D8 * 8) + c * 8) * kcap + row;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) vt[base + static_cast<size_t>(k) * kcap] = e[k];
+    }
   }
 }
 
-cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L, int D,
-                              int max_batch, int kcap, int, bf16* kc, bf16* vc, cudaStream_t s) {
+cudaError_t launch_prefix_set(const bf16* K, const bf16* V, int n_tokens, int batch, int L, int D, int max_batch,
+                              int kcap, int n_static_max, int ring_off, bf16* kc, bf16* vc, bf16* vt,
+                              cudaStream_t s) {
   const size_t total = static_cast<size_t>(L) * batch * n_tokens * (D / 8);
   if (total == 0) return cudaSuccess;
   const int blocks = static_cast<int>((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
-  prefix_set_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(K),
-                                           reinterpret_cast<const uint4*>(V), n_tokens, batch, L,
-                                           D / 8, max_batch, kcap, reinterpret_cast<uint4*>(kc),
-                                           reinterpret_cast<uint4*>(vc));
+  prefix_set_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(K), reinterpret_cast<const uint4*>(V),
+                                           n_tokens, batch, L, D / 8, max_batch, kcap, n_static_max, ring_off,
+                                           reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc), vt);
   return cudaGetLastError();
 }
 
 // One token of K/V per (layer, observation) into cache row slot_row.
 __global__ void ring_append_kernel(const uint4* K, const uint4* V, int batch, int L, int D8,
-                                   int max_batch, int kcap, int slot_row, uint4* kc, uint4* vc) {
+                                   int max_batch, int kcap, int slot_row, uint4* kc, uint4* vc, bf16* vt) {
   const int total = L * batch * D8;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const int c = i % D8, lb = i / D8;
     const int b = lb % batch, l = lb / batch;
     const size_t dst = ((static_cast<size_t>(l) * max_batch + b) * kcap + slot_row) * D8 + c;
     kc[dst] = K[i];
-    vc[dst] = V[i];
+    const uint4 v = V[i];
+    vc[dst] = v;
+    if (vt) {
+      const bf16* e = reinterpret_cast<const bf16*>(&v);
+      const size_t base = ((static_cast<size_t>(l) * max_batch + b) * (D8 * 8) + c * 8) * kcap + slot_row;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) vt[base + static_cast<size_t>(k) * kcap] = e[k];
+    }
   }
 }
 
 cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, int D, int max_batch,
-                               int kcap, int slot_row, bf16* kc, bf16* vc, cudaStream_t s) {
+                               int kcap, int slot_row, bf16* kc, bf16* vc, bf16* vt, cudaStream_t s) {
   const int total = L * batch * (D / 8);
   const int blocks = (total + 255) / 256;
   ring_append_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(K),
                                             reinterpret_cast<const uint4*>(V), batch, L, D / 8,
                                             max_batch, kcap, slot_row, reinterpret_cast<uint4*>(kc),
-                                            reinterpret_cast<uint4*>(vc));
+                                            reinterpret_cast<uint4*>(vc), vt);
   return cudaGetLastError();
 }
 
@@ -335,8 +352,10 @@ cudaError_t launch_cache_update(CacheDesc* desc, int n_static, int n_ring, float
   return cudaGetLastError();
 }
 
+// Static rows [0, n_static_max) then ring rows [ring_off, ring_off + rows - n_static_max)
+// of each (layer, observation), packed.
 __global__ void copy_region_kernel(const uint4* kc, uint4* out, int L, int batch, int max_batch,
-                                   int kcap, int rows, int D8) {
+                                   int kcap, int rows, int D8, int n_static_max, int ring_off) {
   const size_t total = static_cast<size_t>(L) * batch * rows * D8;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -346,18 +365,19 @@ __global__ void copy_region_kernel(const uint4* kc, uint4* out, int L, int batch
     r /= rows;
     const int b = static_cast<int>(r % batch);
     const int l = static_cast<int>(r / batch);
-    out[i] = kc[((static_cast<size_t>(l) * max_batch + b) * kcap + j) * D8 + c];
+    const int row = j < n_static_max ? j : ring_off + (j - n_static_max);
+    out[i] = kc[((static_cast<size_t>(l) * max_batch + b) * kcap + row) * D8 + c];
   }
 }
 
 cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch, int kcap,
-                               int rows, int D, cudaStream_t s) {
+                               int rows, int D, int n_static_max, int ring_off, cudaStream_t s) {
   const size_t total = static_cast<size_t>(L) * batch * rows * (D / 8);
   if (total == 0) return cudaSuccess;
   const int blocks = static_cast<int>((total + 255) / 256 < 148 * 8 ? (total + 255) / 256 : 148 * 8);
   copy_region_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(kc),
                                             reinterpret_cast<uint4*>(out), L, batch, max_batch, kcap,
-                                            rows, D / 8);
+                                            rows, D / 8, n_static_max, ring_off);
   return cudaGetLastError();
 }
 
