@@ -266,11 +266,46 @@ __device__ __forceinline__ void cluster_reduce(const GemmParams& p, uint32_t par
 // owner sums its S slots in rank order (deterministic) and runs the epilogue on row pairs.
 // Partial rows are stored with their 16-byte chunks XOR-swizzled by (global row & 15).
 template <int EPI, int S>
-__device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, const float* s_rinv, int etid,
-                                            int row0, int fbase, int m0, int contrib) {
+__device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, uint32_t recv_bar,
+                                            const float* s_rinv, int etid, int row0, int fbase, int m0,
+                                            int contrib) {
   constexpr int RS = 128 / S, HALF = RS / 2, ITEMS = HALF * 64;
+  constexpr int PRE = ITEMS / 128 < 8 ? ITEMS / 128 : 8;   // items whose operands are prefetched
   constexpr bool RESID = EPI == EPI_RESID || EPI == EPI_BIAS_STORE;
-  for (int it = etid; it < ITEMS; it += 128) {
+  // 1. operands of the epilogue, loaded while the partial tiles are still in flight
+  float2 pa[PRE], pb[PRE], pc[PRE];
+#pragma unroll
+  for (int k = 0; k < PRE; ++k) {
+    const int it = etid + k * 128;
+    const int rp = it % HALF, c = it / HALF;
+    const int m = m0 + c, fn0 = fbase + 2 * rp;
+    pa[k] = pb[k] = pc[k] = make_float2(0.0f, 0.0f);
+    if (m >= p.m_tok) continue;
+    if constexpr (EPI == EPI_RESID) {
+      pa[k] = *reinterpret_cast<const float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0);
+      pb[k] = p.vec ? *reinterpret_cast<const float2*>(p.vec + fn0) : make_float2(1.0f, 1.0f);
+      if (p.zout) pc[k] = *reinterpret_cast<const float2*>(p.zmod + fn0);
+    } else if constexpr (EPI == EPI_BIAS_STORE) {
+      pb[k] = *reinterpret_cast<const float2*>(p.vec + fn0);
+      if (p.zout) pc[k] = *reinterpret_cast<const float2*>(p.zmod + fn0);
+    } else {
+      if (s_rinv && p.cvec) pb[k] = *reinterpret_cast<const float2*>(p.cvec + fn0);
+      if constexpr (EPI == EPI_QKV) {
+        const int pr = fn0 >> 1, DH = p.head_dim >> 1;
+        if (pr < (p.n_heads + 1) * DH) {   // rotated rows (Q, K)
+          const int sq = m % p.seq;
+          pa[k] = reinterpret_cast<const float2*>(p.rope)[sq * DH + (pr % DH)];
+        }
+      }
+    }
+  }
+  // 2. the partial tiles of all S ranks
+  mbar_wait(recv_bar, 0, p.err);
+  if (etid == 0) trace_stamp(p.trace, 7);
+  // 3. sum in rank order (deterministic) and finish
+#pragma unroll
+  for (int k = 0; k < ITEMS / 128; ++k) {
+    const int it = etid + k * 128;
     const int rp = it % HALF, c = it / HALF;
     const int lr0 = 2 * rp, lr1 = lr0 + 1;
     const int i0 = lr0 * 64 + ((((c >> 2) ^ ((row0 + lr0) & 15))) << 2) + (c & 3);
@@ -283,32 +318,33 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
     }
     const int m = m0 + c;
     const int fn0 = fbase + lr0;
+    const bool pre = k < PRE;
     if constexpr (RESID) {
-      // new residual values (+ z for the next GEMM) -> per-token sum of squares
       float ss = 0.0f;
       if (m < p.m_tok) {
         const size_t off = static_cast<size_t>(m) * p.ld_resid + fn0;
-        float2* dst = reinterpret_cast<float2*>(p.resid + off);
         float2 r = make_float2(0.0f, 0.0f);
         bool wrote = true;
         if constexpr (EPI == EPI_RESID) {
-          const float g0 = p.vec ? p.vec[fn0] : 1.0f, g1 = p.vec ? p.vec[fn0 + 1] : 1.0f;
-          r = *dst;
-          r.x += g0 * v0;
-          r.y += g1 * v1;
-          *dst = r;
+          const float2 old = pre ? pa[k] : *reinterpret_cast<const float2*>(p.resid + off);
+          const float2 g = pre ? pb[k] : (p.vec ? *reinterpret_cast<const float2*>(p.vec + fn0) : make_float2(1.0f, 1.0f));
+          r = make_float2(fmaf(g.x, v0, old.x), fmaf(g.y, v1, old.y));
+          *reinterpret_cast<float2*>(p.resid + off) = r;
         } else {
           wrote = !(p.has_state && (m % p.seq) == 0);
           if (wrote) {
-            r = make_float2(v0 + p.vec[fn0], v1 + p.vec[fn0 + 1]);
-            *dst = r;
+            const float2 bias = pre ? pb[k] : *reinterpret_cast<const float2*>(p.vec + fn0);
+            r = make_float2(v0 + bias.x, v1 + bias.y);
+            *reinterpret_cast<float2*>(p.resid + off) = r;
           }
         }
         if (wrote) {
           ss = r.x * r.x + r.y * r.y;
-          if (p.zout)
+          if (p.zout) {
+            const float2 zm = pre ? pc[k] : *reinterpret_cast<const float2*>(p.zmod + fn0);
             *reinterpret_cast<__nv_bfloat162*>(p.zout + off) =
-                __floats2bfloat162_rn(r.x * (1.0f + p.zmod[fn0]), r.y * (1.0f + p.zmod[fn0 + 1]));
+                __floats2bfloat162_rn(r.x * (1.0f + zm.x), r.y * (1.0f + zm.y));
+          }
         }
       }
       if (p.rstat_out) {
@@ -323,10 +359,48 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
       if (s_rinv) {
         // folded norm: out = rinv[m] * (W z) + W shift
         const float rv = s_rinv[c];
-        v0 = fmaf(rv, v0, p.cvec ? p.cvec[fn0] : 0.0f);
-        v1 = fmaf(rv, v1, p.cvec ? p.cvec[fn0 + 1] : 0.0f);
+        const float2 cv = pre ? pb[k] : (p.cvec ? *reinterpret_cast<const float2*>(p.cvec + fn0) : make_float2(0.0f, 0.0f));
+        v0 = fmaf(rv, v0, cv.x);
+        v1 = fmaf(rv, v1, cv.y);
       }
-      epi_pair<EPI>(p, fn0, m, v0, v1);
+      if constexpr (EPI == EPI_QKV) {
+        if (m < p.m_tok) {
+          const int D = p.head_dim, DH = D >> 1, H = p.n_heads;
+          const int pr = fn0 >> 1;
+          if (pr < (H + 2) * DH) {
+            const int b = m / p.seq, sq = m - b * p.seq;
+            int kind, head = 0, i;
+            if (pr < H * DH) {
+              kind = 0;
+              head = pr / DH;
+              i = pr - head * DH;
+            } else if (pr < (H + 1) * DH) {
+              kind = 1;
+              i = pr - H * DH;
+            } else {
+              kind = 2;
+              i = pr - (H + 1) * DH;
+            }
+            float o0 = v0, o1 = v1;
+            if (kind < 2) {
+              const float2 cs = pre ? pa[k] : reinterpret_cast<const float2*>(p.rope)[sq * DH + i];
+              o0 = fmaf(v0, cs.x, -v1 * cs.y);
+              o1 = fmaf(v1, cs.x, v0 * cs.y);
+            }
+            bf16* dst = kind == 0 ? p.out + static_cast<size_t>(m) * p.ld_out + head * D
+                                  : (kind == 1 ? p.kc : p.vc) + (static_cast<size_t>(b) * p.kcap + p.dyn_off + sq) * D;
+            dst[i] = __float2bfloat16_rn(o0);
+            dst[i + DH] = __float2bfloat16_rn(o1);
+            if (kind == 2 && p.vtc) {
+              bf16* vt = p.vtc + static_cast<size_t>(b) * D * p.kcap + p.dyn_off + sq;
+              vt[static_cast<size_t>(i) * p.kcap] = __float2bfloat16_rn(o0);
+              vt[static_cast<size_t>(i + DH) * p.kcap] = __float2bfloat16_rn(o1);
+            }
+          }
+        }
+      } else {
+        epi_pair<EPI>(p, fn0, m, v0, v1);
+      }
     }
   }
 }
@@ -514,24 +588,23 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t rank = cluster_ctarank();
       if (etid == 0) {
         trace_stamp(p.trace, 6);
+        // slice q (rows owned by rank q) -> slot [my rank] of rank q's receive buffer
         const uint32_t slice = static_cast<uint32_t>(RS * 64 * 4);
         const uint32_t src = smem_u32(part), dst = smem_u32(recv) + rank * slice;
         for (int q = 0; q < S; ++q)
           bulk_copy_to_peer(mapa_shared(dst, q), src + q * slice, slice, mapa_shared(recv_bar, q));
         bulk_commit();
       }
-      mbar_wait(recv_bar, 0, p.err);
-      if (etid == 0) trace_stamp(p.trace, 7);
       const int row0 = static_cast<int>(rank) * RS;
       const int fbase = n_tile * G::BM + row0;
       const int contrib = n_tile * S + static_cast<int>(rank);
       const float* rv = p.rstat_in ? s_rinv : nullptr;
       switch (S) {
-        case 1: push_reduce<EPI, 1>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
-        case 2: push_reduce<EPI, 2>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
-        case 4: push_reduce<EPI, 4>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
-        case 8: push_reduce<EPI, 8>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
-        default: push_reduce<EPI, 16>(p, recv, rv, etid, row0, fbase, m0, contrib); break;
+        case 1: push_reduce<EPI, 1>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
+        case 2: push_reduce<EPI, 2>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
+        case 4: push_reduce<EPI, 4>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
+        case 8: push_reduce<EPI, 8>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
+        default: push_reduce<EPI, 16>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
       }
       if (etid == 0) {
         trace_stamp(p.trace, 8);
