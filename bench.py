@@ -74,7 +74,8 @@ def source_sha(files):
 KERNEL_SOURCES = {
     "gemm": ["flow_matching_vla_euler_b200/csrc/gemm_tc.cu", "flow_matching_vla_euler_b200/csrc/ptx.cuh",
              "flow_matching_vla_euler_b200/csrc/kernels.h"],
-    "attention": ["flow_matching_vla_euler_b200/csrc/attention.cu", "flow_matching_vla_euler_b200/csrc/ptx.cuh",
+    "attention": ["flow_matching_vla_euler_b200/csrc/attention.cu", "flow_matching_vla_euler_b200/csrc/attention_tc.cu",
+                  "flow_matching_vla_euler_b200/csrc/ptx.cuh",
                   "flow_matching_vla_euler_b200/csrc/kernels.h"],
 }
 

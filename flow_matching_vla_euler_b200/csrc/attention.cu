@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
       cp_async_wait<0>();
     }
     __syncthreads();
+    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 6);
     const uint32_t sK = sK0 + st * KT * D * 2, sV = sV0 + st * KT * D * 2;
     int trow, tcnt, dyn_start;
     tile_info<D>(sg, t, trow, tcnt, dyn_start);
@@ -320,6 +321,7 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
       }
     }
     __syncthreads();
+    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 7);
   }
 
   if (threadIdx.x == 0) trace_stamp(p.trace, 2);

@@ -266,9 +266,9 @@ __device__ __forceinline__ void cluster_reduce(const GemmParams& p, uint32_t par
 // owner sums its S slots in rank order (deterministic) and runs the epilogue on row pairs.
 // Partial rows are stored with their 16-byte chunks XOR-swizzled by (global row & 15).
 template <int EPI, int S>
-__device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, uint32_t recv_bar,
-                                            const float* s_rinv, int etid, int row0, int fbase, int m0,
-                                            int contrib) {
+__device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, const float* own,
+                                            uint32_t recv_bar, const float* s_rinv, int etid, int rank,
+                                            int row0, int fbase, int m0, int contrib) {
   constexpr int RS = 128 / S, HALF = RS / 2, ITEMS = HALF * 64;
   constexpr int PRE = ITEMS / 128 < 8 ? ITEMS / 128 : 8;   // items whose operands are prefetched
   constexpr bool RESID = EPI == EPI_RESID || EPI == EPI_BIAS_STORE;
@@ -307,14 +307,14 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
   for (int k = 0; k < ITEMS / 128; ++k) {
     const int it = etid + k * 128;
     const int rp = it % HALF, c = it / HALF;
-    const int lr0 = 2 * rp, lr1 = lr0 + 1;
-    const int i0 = lr0 * 64 + ((((c >> 2) ^ ((row0 + lr0) & 15))) << 2) + (c & 3);
-    const int i1 = lr1 * 64 + ((((c >> 2) ^ ((row0 + lr1) & 15))) << 2) + (c & 3);
+    const int lr0 = 2 * rp;
     float v0 = 0.0f, v1 = 0.0f;
 #pragma unroll
     for (int q = 0; q < S; ++q) {
-      v0 += recv[q * RS * 64 + i0];
-      v1 += recv[q * RS * 64 + i1];
+      const float* src = q == rank ? own : recv + q * 64 * RS;   // slot [sender][token][row]
+      const float2 t = *reinterpret_cast<const float2*>(src + c * RS + lr0);
+      v0 += t.x;
+      v1 += t.y;
     }
     const int m = m0 + c;
     const int fn0 = fbase + lr0;
@@ -453,8 +453,12 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(accf, 1);
     if (push) {
+      // S - 1 peers each send this CTA's rows for the tile's valid tokens
+      const int m_valid = min(TN, p.m_tok - m_tile * TN);
+      const uint32_t rx = static_cast<uint32_t>((p.splits - 1) * m_valid * (128 / p.splits) * 4);
       mbar_init(recv_bar, 1);
-      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(128 * TN * 4));   // S slices
+      if (rx) mbar_arrive_expect_tx(recv_bar, rx);
+      else mbar_arrive(recv_bar);
     }
     *s_last = 0;
     fence_mbar_init();
@@ -565,46 +569,47 @@ __global__ void __launch_bounds__(192, 1)
     if (etid == 0) trace_stamp(p.trace, 5);
 
     if (push) {
-      // partial tile -> own shared memory as [row][64 tokens] fp32, 16-byte chunks
-      // swizzled by (row & 15); the pipeline buffers are idle once the MMAs completed
+      // partial tile -> own shared memory as [owner rank][token][row within owner] fp32,
+      // owners RS + (RS % 32 ? RS : 0) floats apart per token row so that the lanes of a
+      // warp (consecutive rows, up to four owners) hit distinct banks; the pipeline
+      // buffers are idle once the MMAs completed
+      const int S = p.splits, RS = 128 / S;
+      const int OS = TN * RS + ((RS & 31) ? RS : 0);
       float* part = reinterpret_cast<float*>(smem);
+      float* mine = part + (r / RS) * OS + (r % RS);
       for (int c = 0; c < TN; c += 16) {
         float v[16];
         tmem_ld16(taddr + c, v);
-        if (nkb == 0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        }
-#pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-          const int chunk = ((c >> 2) + j4) ^ (r & 15);
-          *reinterpret_cast<float4*>(part + r * 64 + chunk * 4) =
-              make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-        }
+        for (int j = 0; j < 16; ++j) mine[(c + j) * RS] = nkb == 0 ? 0.0f : v[j];
       }
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
-      const int S = p.splits, RS = 128 / S;
       const uint32_t rank = cluster_ctarank();
       if (etid == 0) {
         trace_stamp(p.trace, 6);
-        // slice q (rows owned by rank q) -> slot [my rank] of rank q's receive buffer
-        const uint32_t slice = static_cast<uint32_t>(RS * 64 * 4);
-        const uint32_t src = smem_u32(part), dst = smem_u32(recv) + rank * slice;
+        // slice q (rows owned by rank q, valid tokens only) -> slot [my rank] of rank q's
+        // receive buffer; the own slice is read in place
+        const int m_valid = min(TN, p.m_tok - m0);
+        const uint32_t bytes = static_cast<uint32_t>(m_valid * RS * 4);
+        const uint32_t dst = smem_u32(recv) + rank * static_cast<uint32_t>(TN * RS * 4);
         for (int q = 0; q < S; ++q)
-          bulk_copy_to_peer(mapa_shared(dst, q), src + q * slice, slice, mapa_shared(recv_bar, q));
+          if (q != static_cast<int>(rank))
+            bulk_copy_to_peer(mapa_shared(dst, q), smem_u32(part + q * OS), bytes, mapa_shared(recv_bar, q));
         bulk_commit();
       }
       const int row0 = static_cast<int>(rank) * RS;
       const int fbase = n_tile * G::BM + row0;
       const int contrib = n_tile * S + static_cast<int>(rank);
       const float* rv = p.rstat_in ? s_rinv : nullptr;
+      const float* own = part + rank * OS;
+      const int rk = static_cast<int>(rank);
       switch (S) {
-        case 1: push_reduce<EPI, 1>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
-        case 2: push_reduce<EPI, 2>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
-        case 4: push_reduce<EPI, 4>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
-        case 8: push_reduce<EPI, 8>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
-        default: push_reduce<EPI, 16>(p, recv, recv_bar, rv, etid, row0, fbase, m0, contrib); break;
+        case 1: push_reduce<EPI, 1>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
+        case 2: push_reduce<EPI, 2>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
+        case 4: push_reduce<EPI, 4>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
+        case 8: push_reduce<EPI, 8>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
+        default: push_reduce<EPI, 16>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
       }
       if (etid == 0) {
         trace_stamp(p.trace, 8);
