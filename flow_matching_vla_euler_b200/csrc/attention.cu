@@ -12,8 +12,9 @@
 // segment (static [0, n_static), ring [ring_off, ring_off + n_ring), dynamic
 // [dyn_off, dyn_off + S)), staged through shared memory by a 2-deep cp.async pipeline,
 // and contracted with bf16 mma.sync (fp32 accumulate) with an online softmax in fp32.
-// Splits write unnormalised partials; the last CTA of a query tile to arrive merges them
-// in split order (deterministic).
+// The key splits of a query tile form one thread-block cluster: each CTA owns 64/splits
+// query rows and merges the splits' unnormalised partials for them, pushed through
+// distributed shared memory, in split order (deterministic).
 //
 // Mask (prefix-LM): every suffix row sees every cached key; action rows see the whole
 // suffix; with a state token, suffix row 0 sees the cached keys and itself only.
@@ -399,6 +400,9 @@ static cudaError_t configure_d() {
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(AttnCfg<D>::SMEM));
   if (e == cudaSuccess) e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   return e;
 }
 

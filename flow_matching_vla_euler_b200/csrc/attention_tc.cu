@@ -317,6 +317,9 @@ cudaError_t configure_attention_tc_kernel() {
   static cudaError_t done = cudaErrorNotReady;
   if (done == cudaSuccess) return done;
   done = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
+  if (done == cudaSuccess)
+    done = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared);
   return done;
 }
 

@@ -33,12 +33,20 @@ struct GemmCfg {
   static constexpr int B_BYTES = TN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // token tile 64 with cluster splits: partial tiles are pushed to their owners' receive
-  // buffers (32 KB); three stages keep two CTAs per SM
+  // buffers. These kernels size their pipeline (2..4 stages) and receive buffer (S - 1
+  // slots) per launch, so that a CTA stays small enough to share its SM with a CTA of the
+  // kernel before or after it (weights stream in while that one runs).
   static constexpr bool PUSH = CL && TN == 64;
-  static constexpr int STAGES = PUSH ? 3 : 4;
-  static constexpr int RECV_BYTES = PUSH ? 128 * TN * 4 : 0;
+  static constexpr int STAGES = 4;                // maximum
+  static constexpr int RECV_BYTES = PUSH ? 128 * TN * 4 : 0;   // maximum
   static constexpr int TMEM_COLS = TN;            // fp32 accumulator columns (power of 2)
-  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + RECV_BYTES + 1024;   // + barriers, rinv
+  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + RECV_BYTES + 2048;   // + barriers, rinv
+  // the fp32 partial tile lives in the idle stages after the main loop
+  static constexpr int push_need(int) { return 128 * TN * 4; }
+  static constexpr size_t push_smem(int stages, int splits) {
+    return 1024 + static_cast<size_t>(stages) * STAGE_BYTES + static_cast<size_t>(splits - 1) * (128 / splits) * TN * 4 +
+           2048;
+  }
 };
 
 template <int EPI>
@@ -262,63 +270,72 @@ __device__ __forceinline__ void cluster_reduce(const GemmParams& p, uint32_t par
 }
 
 // Push-mode reduction, token tile 64: every CTA of the cluster has sent rows
-// [q*128/S, (q+1)*128/S) of its partial tile to CTA q (receive slot = sender rank); the
-// owner sums its S slots in rank order (deterministic) and runs the epilogue on row pairs.
-// Partial rows are stored with their 16-byte chunks XOR-swizzled by (global row & 15).
+// [q*128/S, (q+1)*128/S) of its partial tile to CTA q (receive slots = the other ranks in
+// rank order); the owner sums its S partials in rank order (deterministic) and runs the
+// epilogue on row pairs, 256 threads. A thread keeps one row pair (feature pair) for all
+// its items, so the per-feature operands (gate, bias, z modulation, W.shift, the rotary
+// slot) are loaded once; the per-token operands of the first items (residual, rotary
+// cos/sin) are fetched before the wait.
 template <int EPI, int S>
 __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* recv, const float* own,
                                             uint32_t recv_bar, const float* s_rinv, int etid, int rank,
-                                            int row0, int fbase, int m0, int contrib) {
-  constexpr int RS = 128 / S, HALF = RS / 2, ITEMS = HALF * 64;
-  constexpr int PRE = ITEMS / 128 < 8 ? ITEMS / 128 : 8;   // items whose operands are prefetched
+                                            int fbase, int m0, int contrib) {
+  constexpr int RS = 128 / S, HALF = RS / 2, ITEMS = HALF * 64, NIT = ITEMS / 256, CSTEP = 256 / HALF;
+  constexpr int PRE = NIT < 8 ? NIT : 8;
   constexpr bool RESID = EPI == EPI_RESID || EPI == EPI_BIAS_STORE;
-  // 1. operands of the epilogue, loaded while the partial tiles are still in flight
-  float2 pa[PRE], pb[PRE], pc[PRE];
-#pragma unroll
-  for (int k = 0; k < PRE; ++k) {
-    const int it = etid + k * 128;
-    const int rp = it % HALF, c = it / HALF;
-    const int m = m0 + c, fn0 = fbase + 2 * rp;
-    pa[k] = pb[k] = pc[k] = make_float2(0.0f, 0.0f);
-    if (m >= p.m_tok) continue;
-    if constexpr (EPI == EPI_RESID) {
-      pa[k] = *reinterpret_cast<const float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0);
-      pb[k] = p.vec ? *reinterpret_cast<const float2*>(p.vec + fn0) : make_float2(1.0f, 1.0f);
-      if (p.zout) pc[k] = *reinterpret_cast<const float2*>(p.zmod + fn0);
-    } else if constexpr (EPI == EPI_BIAS_STORE) {
-      pb[k] = *reinterpret_cast<const float2*>(p.vec + fn0);
-      if (p.zout) pc[k] = *reinterpret_cast<const float2*>(p.zmod + fn0);
-    } else {
-      if (s_rinv && p.cvec) pb[k] = *reinterpret_cast<const float2*>(p.cvec + fn0);
-      if constexpr (EPI == EPI_QKV) {
-        const int pr = fn0 >> 1, DH = p.head_dim >> 1;
-        if (pr < (p.n_heads + 1) * DH) {   // rotated rows (Q, K)
-          const int sq = m % p.seq;
-          pa[k] = reinterpret_cast<const float2*>(p.rope)[sq * DH + (pr % DH)];
-        }
-      }
+  static_assert(ITEMS % 256 == 0, "whole items per thread");
+  const int rp = etid % HALF, c0 = etid / HALF;
+  const int lr0 = 2 * rp, fn0 = fbase + lr0;
+  const bool folded = s_rinv != nullptr;
+  // per-feature operands
+  float2 vec2 = make_float2(1.0f, 1.0f), zm2 = make_float2(0.0f, 0.0f), cv2 = make_float2(0.0f, 0.0f);
+  if constexpr (RESID) {
+    if (p.vec) vec2 = *reinterpret_cast<const float2*>(p.vec + fn0);
+    if (p.zout) zm2 = *reinterpret_cast<const float2*>(p.zmod + fn0);
+  } else if (folded && p.cvec) {
+    cv2 = *reinterpret_cast<const float2*>(p.cvec + fn0);
+  }
+  // EPI_QKV: destination of this feature pair (Q head / K / V, element i and i + D/2)
+  int kind = 3, i_q = 0;
+  bf16* qbase = nullptr;
+  if constexpr (EPI == EPI_QKV) {
+    const int D = p.head_dim, DH = D >> 1, H = p.n_heads, pr = fn0 >> 1;
+    if (pr < (H + 2) * DH) {
+      kind = pr < H * DH ? 0 : (pr < (H + 1) * DH ? 1 : 2);
+      const int head = kind == 0 ? pr / DH : 0;
+      i_q = pr - (kind == 0 ? head : H + kind - 1) * DH;
+      qbase = kind == 0 ? p.out + head * D : (kind == 1 ? p.kc : p.vc);
     }
   }
-  // 2. the partial tiles of all S ranks
+  // per-token operands of the first items
+  float2 pre[PRE];
+#pragma unroll
+  for (int k = 0; k < PRE; ++k) {
+    const int m = m0 + c0 + k * CSTEP;
+    pre[k] = make_float2(0.0f, 0.0f);
+    if (m < p.m_tok) {
+      if constexpr (EPI == EPI_RESID)
+        pre[k] = *reinterpret_cast<const float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0);
+      if constexpr (EPI == EPI_QKV)
+        if (kind < 2) pre[k] = reinterpret_cast<const float2*>(p.rope)[(m % p.seq) * (p.head_dim >> 1) + i_q];
+    }
+  }
+  // the partial tiles of all S ranks
   mbar_wait(recv_bar, 0, p.err);
   if (etid == 0) trace_stamp(p.trace, 7);
-  // 3. sum in rank order (deterministic) and finish
-#pragma unroll
-  for (int k = 0; k < ITEMS / 128; ++k) {
-    const int it = etid + k * 128;
-    const int rp = it % HALF, c = it / HALF;
-    const int lr0 = 2 * rp;
+#pragma unroll 4
+  for (int k = 0; k < NIT; ++k) {
+    const int c = c0 + k * CSTEP;
     float v0 = 0.0f, v1 = 0.0f;
 #pragma unroll
     for (int q = 0; q < S; ++q) {
-      const float* src = q == rank ? own : recv + q * 64 * RS;   // slot [sender][token][row]
-      const float2 t = *reinterpret_cast<const float2*>(src + c * RS + lr0);
-      v0 += t.x;
-      v1 += t.y;
+      // slot [sender, own rank skipped][token / 4][row][token % 4]
+      const float* src = (q == rank ? own : recv + (q < rank ? q : q - 1) * 64 * RS) + (c >> 2) * RS * 4 + lr0 * 4 + (c & 3);
+      v0 += src[0];
+      v1 += src[4];
     }
+    if (k == 0 && etid == 0) trace_stamp(p.trace, 12);
     const int m = m0 + c;
-    const int fn0 = fbase + lr0;
-    const bool pre = k < PRE;
     if constexpr (RESID) {
       float ss = 0.0f;
       if (m < p.m_tok) {
@@ -326,25 +343,21 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
         float2 r = make_float2(0.0f, 0.0f);
         bool wrote = true;
         if constexpr (EPI == EPI_RESID) {
-          const float2 old = pre ? pa[k] : *reinterpret_cast<const float2*>(p.resid + off);
-          const float2 g = pre ? pb[k] : (p.vec ? *reinterpret_cast<const float2*>(p.vec + fn0) : make_float2(1.0f, 1.0f));
-          r = make_float2(fmaf(g.x, v0, old.x), fmaf(g.y, v1, old.y));
+          const float2 old = k < PRE ? pre[k < PRE ? k : 0] : *reinterpret_cast<const float2*>(p.resid + off);
+          r = make_float2(fmaf(vec2.x, v0, old.x), fmaf(vec2.y, v1, old.y));
           *reinterpret_cast<float2*>(p.resid + off) = r;
         } else {
           wrote = !(p.has_state && (m % p.seq) == 0);
           if (wrote) {
-            const float2 bias = pre ? pb[k] : *reinterpret_cast<const float2*>(p.vec + fn0);
-            r = make_float2(v0 + bias.x, v1 + bias.y);
+            r = make_float2(v0 + vec2.x, v1 + vec2.y);
             *reinterpret_cast<float2*>(p.resid + off) = r;
           }
         }
         if (wrote) {
           ss = r.x * r.x + r.y * r.y;
-          if (p.zout) {
-            const float2 zm = pre ? pc[k] : *reinterpret_cast<const float2*>(p.zmod + fn0);
+          if (p.zout)
             *reinterpret_cast<__nv_bfloat162*>(p.zout + off) =
-                __floats2bfloat162_rn(r.x * (1.0f + zm.x), r.y * (1.0f + zm.y));
-          }
+                __floats2bfloat162_rn(r.x * (1.0f + zm2.x), r.y * (1.0f + zm2.y));
         }
       }
       if (p.rstat_out) {
@@ -356,46 +369,30 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
           p.rstat_out[static_cast<size_t>(p.rstat_slot0 + contrib * SUB + (rp >> 5)) * p.ld_rstat + m] = ss;
       }
     } else {
-      if (s_rinv) {
+      if (folded) {
         // folded norm: out = rinv[m] * (W z) + W shift
         const float rv = s_rinv[c];
-        const float2 cv = pre ? pb[k] : (p.cvec ? *reinterpret_cast<const float2*>(p.cvec + fn0) : make_float2(0.0f, 0.0f));
-        v0 = fmaf(rv, v0, cv.x);
-        v1 = fmaf(rv, v1, cv.y);
+        v0 = fmaf(rv, v0, cv2.x);
+        v1 = fmaf(rv, v1, cv2.y);
       }
       if constexpr (EPI == EPI_QKV) {
-        if (m < p.m_tok) {
-          const int D = p.head_dim, DH = D >> 1, H = p.n_heads;
-          const int pr = fn0 >> 1;
-          if (pr < (H + 2) * DH) {
-            const int b = m / p.seq, sq = m - b * p.seq;
-            int kind, head = 0, i;
-            if (pr < H * DH) {
-              kind = 0;
-              head = pr / DH;
-              i = pr - head * DH;
-            } else if (pr < (H + 1) * DH) {
-              kind = 1;
-              i = pr - H * DH;
-            } else {
-              kind = 2;
-              i = pr - (H + 1) * DH;
-            }
-            float o0 = v0, o1 = v1;
-            if (kind < 2) {
-              const float2 cs = pre ? pa[k] : reinterpret_cast<const float2*>(p.rope)[sq * DH + i];
-              o0 = fmaf(v0, cs.x, -v1 * cs.y);
-              o1 = fmaf(v1, cs.x, v0 * cs.y);
-            }
-            bf16* dst = kind == 0 ? p.out + static_cast<size_t>(m) * p.ld_out + head * D
-                                  : (kind == 1 ? p.kc : p.vc) + (static_cast<size_t>(b) * p.kcap + p.dyn_off + sq) * D;
-            dst[i] = __float2bfloat16_rn(o0);
-            dst[i + DH] = __float2bfloat16_rn(o1);
-            if (kind == 2 && p.vtc) {
-              bf16* vt = p.vtc + static_cast<size_t>(b) * D * p.kcap + p.dyn_off + sq;
-              vt[static_cast<size_t>(i) * p.kcap] = __float2bfloat16_rn(o0);
-              vt[static_cast<size_t>(i + DH) * p.kcap] = __float2bfloat16_rn(o1);
-            }
+        if (m < p.m_tok && kind < 3) {
+          const int D = p.head_dim, DH = D >> 1;
+          const int b = m / p.seq, sq = m - b * p.seq;
+          float o0 = v0, o1 = v1;
+          if (kind < 2) {
+            const float2 cs = k < PRE ? pre[k < PRE ? k : 0] : reinterpret_cast<const float2*>(p.rope)[sq * DH + i_q];
+            o0 = fmaf(v0, cs.x, -v1 * cs.y);
+            o1 = fmaf(v1, cs.x, v0 * cs.y);
+          }
+          bf16* dst = kind == 0 ? qbase + static_cast<size_t>(m) * p.ld_out
+                                : qbase + (static_cast<size_t>(b) * p.kcap + p.dyn_off + sq) * D;
+          dst[i_q] = __float2bfloat16_rn(o0);
+          dst[i_q + DH] = __float2bfloat16_rn(o1);
+          if (kind == 2 && p.vtc) {
+            bf16* vt = p.vtc + static_cast<size_t>(b) * D * p.kcap + p.dyn_off + sq;
+            vt[static_cast<size_t>(i_q) * p.kcap] = __float2bfloat16_rn(o0);
+            vt[static_cast<size_t>(i_q + DH) * p.kcap] = __float2bfloat16_rn(o1);
           }
         }
       } else {
@@ -411,17 +408,22 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
 // partial tile in its own shared memory and CTA rank r sums rows [r*128/S, (r+1)*128/S)
 // over all ranks through distributed shared memory, in rank order (deterministic).
 template <int TN, int EPI, bool CL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                    const GemmParams p) {
   using G = GemmCfg<TN, CL>;
+  static_assert(!G::PUSH || G::push_need(1) <= 2 * G::STAGE_BYTES,
+                "the partial tile fits in two idle pipeline stages");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + G::STAGES * G::A_BYTES;
-  float* recv = reinterpret_cast<float*>(smem + G::STAGES * G::STAGE_BYTES);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES + G::RECV_BYTES);
+  // push kernels: p.stages stages and S - 1 receive slots, set by the launcher
+  const int stages = G::PUSH ? p.stages : G::STAGES;
+  const int recv_bytes = G::PUSH ? (p.splits - 1) * (128 / p.splits) * TN * 4 : 0;
+  uint8_t* sB = smem + stages * G::A_BYTES;
+  float* recv = reinterpret_cast<float*>(smem + stages * G::STAGE_BYTES);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + stages * G::STAGE_BYTES + recv_bytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2 * G::STAGES + 2);
   volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -443,7 +445,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t empty0 = smem_u32(&bar[G::STAGES]);
   const uint32_t accf = smem_u32(&bar[2 * G::STAGES]);
   const uint32_t recv_bar = smem_u32(&bar[2 * G::STAGES + 1]);
-  const int npre = min(nkb, G::STAGES);
+  const int npre = min(nkb, stages);
 
   if (threadIdx.x == 0) {
     trace_stamp(p.trace, 0);
@@ -454,8 +456,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(accf, 1);
     if (push) {
       // S - 1 peers each send this CTA's rows for the tile's valid tokens
-      const int m_valid = min(TN, p.m_tok - m_tile * TN);
-      const uint32_t rx = static_cast<uint32_t>((p.splits - 1) * m_valid * (128 / p.splits) * 4);
+      const int m_groups = (min(TN, p.m_tok - m_tile * TN) + 3) / 4;
+      const uint32_t rx = static_cast<uint32_t>((p.splits - 1) * m_groups * (128 / p.splits) * 16);
       mbar_init(recv_bar, 1);
       if (rx) mbar_arrive_expect_tx(recv_bar, rx);
       else mbar_arrive(recv_bar);
@@ -474,13 +476,17 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), G::TMEM_COLS);
+    if (lane == 0) trace_stamp(p.trace, 13);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (push) cluster_sync_all();              // every receive barrier of the cluster is armed
+  if (threadIdx.x == 0) trace_stamp(p.trace, 11);
+  // push: this CTA's receive barrier is armed; the matching wait comes right before the
+  // first access to another CTA's shared memory, long after every CTA has arrived
+  if (push) cluster_arrive();
   if (threadIdx.x == 0) {
     pdl_trigger();
     trace_stamp(p.trace, 1);
@@ -498,8 +504,8 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(smem_u32(sB + i * G::B_BYTES), &tm_x, full0 + 8 * i, (kb0 + i) * G::BK, y_x, pol_x);
       int issued = npre;
       for (int i = npre; i < nkb; ++i) {
-        const int s = i % G::STAGES;
-        if (!mbar_wait(empty0 + 8 * s, ((i / G::STAGES) - 1) & 1, p.err)) break;
+        const int s = i % stages;
+        if (!mbar_wait(empty0 + 8 * s, ((i / stages) - 1) & 1, p.err)) break;
         mbar_arrive_expect_tx(full0 + 8 * s, G::STAGE_BYTES);
         tma_load_2d(smem_u32(sA + s * G::A_BYTES), &tm_w, full0 + 8 * s, (kb0 + i) * G::BK, y_w,
                     pol_w);
@@ -508,18 +514,19 @@ __global__ void __launch_bounds__(192, 1)
         issued = i + 1;
       }
       // Do not leave with copies in flight: the last load of each stage has landed.
-      for (int s = 0; s < G::STAGES && s < issued; ++s) {
-        const int last_i = s + ((issued - 1 - s) / G::STAGES) * G::STAGES;
-        mbar_wait(full0 + 8 * s, (last_i / G::STAGES) & 1, p.err);
+      for (int s = 0; s < stages && s < issued; ++s) {
+        const int last_i = s + ((issued - 1 - s) / stages) * stages;
+        mbar_wait(full0 + 8 * s, (last_i / stages) & 1, p.err);
       }
     }
     __syncwarp();
+    if (push) cluster_wait();
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, TN);
       for (int i = 0; i < nkb; ++i) {
-        const int s = i % G::STAGES;
-        if (!mbar_wait(full0 + 8 * s, (i / G::STAGES) & 1, p.err)) break;
+        const int s = i % stages;
+        if (!mbar_wait(full0 + 8 * s, (i / stages) & 1, p.err)) break;
         if (i == 0) trace_stamp(p.trace, 3);
         tc_fence_after();
         const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * G::A_BYTES));
@@ -533,88 +540,106 @@ __global__ void __launch_bounds__(192, 1)
       trace_stamp(p.trace, 4);
     }
     __syncwarp();
+    if (push) cluster_wait();
   } else {
     pdl_wait();
+    // warps 2..9: the push path uses all eight (two per TMEM lane quarter, each half of
+    // the token columns); the other paths use warps 2..5 with whole rows
+    const int ew = warp - 2;
     const int q = warp & 3;                  // TMEM lanes [32q, 32q + 32) for this warp
     const int r = q * 32 + lane;             // tile row = output feature
-    const int etid = (warp - 2) * 32 + lane;
+    const int etid = ew * 32 + lane;         // 0..255
+    const bool main4 = ew < 4;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int tile = m_tile * gridDim.x + n_tile;
     const int fn = n_tile * G::BM + r;
     const int m0 = m_tile * TN;
-    float* s_rinv = reinterpret_cast<float*>(tmem_slot + 4);
+    float* s_rinv = reinterpret_cast<float*>(tmem_slot + 4);   // [4][64]
     if (p.rstat_in) {
       // rinv per token from the residual producers' sum-of-squares partials, computed while
-      // the main loop runs (two threads per token, loads unrolled)
+      // the main loop runs (four threads per token, loads unrolled)
       const int tok = etid & 63, par = etid >> 6;
       const int m = m0 + tok;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       if (m < p.m_tok) {
         int c = par;
-        for (; c + 14 < p.rstat_n; c += 16) {
+        for (; c + 28 < p.rstat_n; c += 32) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u) acc[u] += p.rstat_in[static_cast<size_t>(c + 2 * u) * p.ld_rstat + m];
+          for (int u = 0; u < 8; ++u) acc[u] += p.rstat_in[static_cast<size_t>(c + 4 * u) * p.ld_rstat + m];
         }
-        for (; c < p.rstat_n; c += 2) acc[0] += p.rstat_in[static_cast<size_t>(c) * p.ld_rstat + m];
+        for (; c < p.rstat_n; c += 4) acc[0] += p.rstat_in[static_cast<size_t>(c) * p.ld_rstat + m];
       }
-      float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      if (par == 1) s_rinv[64 + tok] = ss;
-      named_bar_sync(1, 128);
-      if (par == 0)
-        s_rinv[tok] = m < p.m_tok ? 1.0f / sqrtf((ss + s_rinv[64 + tok]) / static_cast<float>(p.k_dim) + p.eps) : 0.0f;
-      named_bar_sync(1, 128);
+      const float ss = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      if (par > 0) s_rinv[64 * par + tok] = ss;
+      named_bar_sync(1, 256);
+      if (par == 0) {
+        const float tot = (ss + s_rinv[64 + tok]) + (s_rinv[128 + tok] + s_rinv[192 + tok]);
+        s_rinv[tok] = m < p.m_tok ? 1.0f / sqrtf(tot / static_cast<float>(p.k_dim) + p.eps) : 0.0f;
+      }
+      named_bar_sync(1, 256);
     }
     mbar_wait(accf, 0, p.err);
     tc_fence_after();
     if (etid == 0) trace_stamp(p.trace, 5);
 
     if (push) {
-      // partial tile -> own shared memory as [owner rank][token][row within owner] fp32,
-      // owners RS + (RS % 32 ? RS : 0) floats apart per token row so that the lanes of a
-      // warp (consecutive rows, up to four owners) hit distinct banks; the pipeline
-      // buffers are idle once the MMAs completed
+      // partial tile -> own shared memory as [owner rank][token / 4][row within owner]
+      // [token % 4] fp32: 16-byte stores, eight consecutive rows per 128 bytes; the
+      // pipeline buffers are idle once the MMAs completed
       const int S = p.splits, RS = 128 / S;
-      const int OS = TN * RS + ((RS & 31) ? RS : 0);
+      const int OS = TN * RS;
       float* part = reinterpret_cast<float*>(smem);
-      float* mine = part + (r / RS) * OS + (r % RS);
-      for (int c = 0; c < TN; c += 16) {
+      float* mine = part + (r / RS) * OS + (r % RS) * 4;
+      const int cbeg = (ew >> 2) * (TN / 2);
+#pragma unroll
+      for (int c = cbeg; c < cbeg + TN / 2; c += 16) {
         float v[16];
         tmem_ld16(taddr + c, v);
+        if (nkb == 0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) mine[(c + j) * RS] = nkb == 0 ? 0.0f : v[j];
+          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        }
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4)
+          *reinterpret_cast<float4*>(mine + ((c >> 2) + j4) * RS * 4) =
+              make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      cluster_wait();                        // every receive barrier of the cluster is armed
+      named_bar_sync(1, 256);
       const uint32_t rank = cluster_ctarank();
       if (etid == 0) {
         trace_stamp(p.trace, 6);
-        // slice q (rows owned by rank q, valid tokens only) -> slot [my rank] of rank q's
-        // receive buffer; the own slice is read in place
-        const int m_valid = min(TN, p.m_tok - m0);
-        const uint32_t bytes = static_cast<uint32_t>(m_valid * RS * 4);
-        const uint32_t dst = smem_u32(recv) + rank * static_cast<uint32_t>(TN * RS * 4);
-        for (int q = 0; q < S; ++q)
-          if (q != static_cast<int>(rank))
-            bulk_copy_to_peer(mapa_shared(dst, q), smem_u32(part + q * OS), bytes, mapa_shared(recv_bar, q));
+        // slice q (rows owned by rank q, valid tokens only) -> rank q's receive slot for
+        // this rank (the S - 1 other ranks in rank order); the own slice is read in place
+        const int m_groups = (min(TN, p.m_tok - m0) + 3) / 4;
+        const uint32_t bytes = static_cast<uint32_t>(m_groups * RS * 16);
+        for (int qq = 0; qq < S; ++qq) {
+          if (qq == static_cast<int>(rank)) continue;
+          const int slot = static_cast<int>(rank) < qq ? static_cast<int>(rank) : static_cast<int>(rank) - 1;
+          const uint32_t dst = smem_u32(recv) + static_cast<uint32_t>(slot * TN * RS * 4);
+          bulk_copy_to_peer(mapa_shared(dst, qq), smem_u32(part + qq * OS), bytes, mapa_shared(recv_bar, qq));
+        }
         bulk_commit();
       }
-      const int row0 = static_cast<int>(rank) * RS;
-      const int fbase = n_tile * G::BM + row0;
+      const int fbase = n_tile * G::BM + static_cast<int>(rank) * RS;
       const int contrib = n_tile * S + static_cast<int>(rank);
       const float* rv = p.rstat_in ? s_rinv : nullptr;
       const float* own = part + rank * OS;
       const int rk = static_cast<int>(rank);
       switch (S) {
-        case 1: push_reduce<EPI, 1>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
-        case 2: push_reduce<EPI, 2>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
-        case 4: push_reduce<EPI, 4>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
-        case 8: push_reduce<EPI, 8>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
-        default: push_reduce<EPI, 16>(p, recv, own, recv_bar, rv, etid, rk, row0, fbase, m0, contrib); break;
+        case 1: push_reduce<EPI, 1>(p, recv, own, recv_bar, rv, etid, rk, fbase, m0, contrib); break;
+        case 2: push_reduce<EPI, 2>(p, recv, own, recv_bar, rv, etid, rk, fbase, m0, contrib); break;
+        case 4: push_reduce<EPI, 4>(p, recv, own, recv_bar, rv, etid, rk, fbase, m0, contrib); break;
+        case 8: push_reduce<EPI, 8>(p, recv, own, recv_bar, rv, etid, rk, fbase, m0, contrib); break;
+        default: push_reduce<EPI, 16>(p, recv, own, recv_bar, rv, etid, rk, fbase, m0, contrib); break;
       }
       if (etid == 0) {
         trace_stamp(p.trace, 8);
         bulk_wait_all();                     // own outgoing copies finished before exit
       }
+    } else if (!main4) {
+      // not needed outside the push path
     } else if (cluster_red) {
       // partial tile -> own shared memory, [token][row] fp32 (the pipeline buffers are idle)
       float* part = reinterpret_cast<float*>(smem);
@@ -677,7 +702,7 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 64) trace_stamp(p.trace, 6);
     cluster_sync_all();                      // every partial tile is in its CTA's smem
     if (threadIdx.x == 64) trace_stamp(p.trace, 7);
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 6) {
       const int etid = (warp - 2) * 32 + lane;
       const int row0 = static_cast<int>(cluster_ctarank()) * (128 / p.splits);
       const uint32_t part = smem_u32(smem);
@@ -898,7 +923,9 @@ static cudaError_t configure_persist_tn() {
                   gemm_persist_kernel<TN, EPI_GEGLU>, gemm_persist_kernel<TN, EPI_SWISH_VEC>,
                   gemm_persist_kernel<TN, EPI_BIAS_STORE>, gemm_persist_kernel<TN, EPI_STORE>})
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(PersistCfg<TN>::SMEM))) != cudaSuccess)
+                                  static_cast<int>(PersistCfg<TN>::SMEM))) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;
   return cudaSuccess;
 }
@@ -909,6 +936,11 @@ static cudaError_t configure_one() {
                                        static_cast<int>(GemmCfg<TN, CL>::SMEM));
   if (e == cudaSuccess && CL)
     e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  // every kernel of the denoise chain asks for the largest shared-memory carve-out, so an
+  // SM configured by one of them has room for a CTA of the next (PDL overlap)
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   return e;
 }
 
@@ -946,7 +978,7 @@ cudaError_t configure_gemm_kernels() {
 int gemm_max_cluster(int tn) {
   if (configure_gemm_kernels() != cudaSuccess) return 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   cfg.attrs = attr;
@@ -988,8 +1020,22 @@ static cudaError_t launch_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, 
   using G = GemmCfg<TN, CL>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_tiles, m_tiles, p.splits);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
   cfg.dynamicSmemBytes = G::SMEM;
+  GemmParams q = p;
+  if constexpr (G::PUSH) {
+    // as many stages as a split has K blocks, at most the caller's cap (p.stages, default
+    // 3) and at least enough to hold the partial tile after the main loop
+    const int nkb_split = (p.k_dim / G::BK + p.splits - 1) / p.splits;
+    const int cap = p.stages > 0 ? p.stages : 3;   // caller's shared-memory budget
+    int st = nkb_split < cap ? nkb_split : cap;
+    if (st < 2) st = 2;
+    if (st > G::STAGES) st = G::STAGES;
+    while (st * G::STAGE_BYTES < G::push_need(p.splits)) ++st;
+    if (st > G::STAGES) return cudaErrorInvalidValue;
+    q.stages = st;
+    cfg.dynamicSmemBytes = G::push_smem(st, p.splits);
+  }
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -1009,7 +1055,7 @@ static cudaError_t launch_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI, CL>, tm_w, tm_x, p);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI, CL>, tm_w, tm_x, q);
 }
 
 template <int TN, bool CL>

@@ -39,6 +39,8 @@ struct GemmParams {
   int w_row0;         // first row of this weight in the stacked weight tensor map
   int splits;         // K splits (grid.z)
   int kb_per_split;   // 64-wide K blocks per split
+  int stages;         // cluster push kernels: cap on pipeline stages (0: 3); the launcher
+                      // passes the count it chose
   int w_stream;       // 1: each weight tile is read once (L2 evict-first), 0: reused
   float* resid;       // fp32 residual [m][ld_resid]
   int ld_resid;
@@ -111,6 +113,7 @@ cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q
                              cudaStream_t s, bool pdl);
 int attn_q_tile();                       // query rows per CTA
 cudaError_t configure_attention_kernels();
+cudaError_t configure_small_kernels();
 int attn_key_tile(int head_dim);         // keys per pipeline stage
 int attn_max_cluster(int head_dim);      // largest co-schedulable split cluster
 

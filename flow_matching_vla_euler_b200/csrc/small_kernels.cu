@@ -381,4 +381,21 @@ cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int 
   return cudaGetLastError();
 }
 
+// The per-step kernels of the denoise chain prefer the largest shared-memory carve-out
+// too, so that an SM they configured still takes a CTA of the projection that follows.
+cudaError_t configure_small_kernels() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaSuccess) return done;
+  cudaError_t e = cudaSuccess;
+  const void* fns[] = {reinterpret_cast<const void*>(norm_kernel<2>), reinterpret_cast<const void*>(norm_kernel<4>),
+                       reinterpret_cast<const void*>(norm_kernel<8>), reinterpret_cast<const void*>(norm_kernel<16>),
+                       reinterpret_cast<const void*>(embed_kernel), reinterpret_cast<const void*>(final_kernel)};
+  for (const void* fn : fns)
+    if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+  done = cudaSuccess;
+  return done;
+}
+
 }  // namespace vla
