@@ -125,16 +125,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// bf16 [rows][inner] row-major, boxes of 64 (inner) x box_rows, 128-byte swizzle.
-int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+// bf16 [rows][inner] row-major, boxes of box_cols (inner) x box_rows; 128-byte swizzle for
+// 64-column boxes, 64-byte swizzle for 32-column boxes.
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows,
+              uint32_t box_cols = 64) {
   auto enc = get_encode();
   if (!enc) return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (box_cols != 64 && box_cols != 32) return fail(VLA_ERR_ARG, "TMA box width %u", box_cols);
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llu x %llu, box rows %u",
@@ -192,6 +196,7 @@ struct vla_expert {
 
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
   CUtensorMap tm_q, tm_kc, tm_vt;   // tensor-core attention operands (head_dim 256)
+  CUtensorMap tm_qa, tm_ka, tm_va;  // split-KV attention operands (any head_dim)
 
   // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
   unsigned long long* trace = nullptr;
@@ -552,9 +557,8 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           int rc = enqueue_gemm(h, rec, VLA_K_GEMM_QKV, EPI_QKV, h->tm_wqkv, am.hb, p, h->qkv_rows, W, M, pdl);
           if (rc) return rc;
           AttnParams a{};
-          a.q = h->qb;
-          a.kc = p.kc;
-          a.vc = p.vc;
+          a.layer = l;
+          a.max_batch = h->cfg.max_batch;
           a.out = h->ob;
           a.cache = h->desc;
           a.seq = h->S;
@@ -585,7 +589,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
             t.trace = tr(1);
             CU(launch_attention_tc(h->tm_q, h->tm_kc, h->tm_vt, t, B, rec.s, pdl));
           } else {
-            CU(launch_attention(h->D, a, B, ap.q_tiles, rec.s, pdl));
+            CU(launch_attention(h->D, h->tm_qa, h->tm_ka, h->tm_va, a, B, ap.q_tiles, rec.s, pdl));
           }
           rec.end(VLA_K_ATTN);
           GemmParams o{};
@@ -919,6 +923,14 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  {
+    const uint64_t rows = static_cast<uint64_t>(L) * cfg->max_batch * h->kcap;
+    const uint32_t bc = static_cast<uint32_t>(attn_box_cols(D)), kt = static_cast<uint32_t>(attn_key_tile(D));
+    if ((rc = make_tmap(&h->tm_qa, h->qb, D, static_cast<uint64_t>(h->max_M) * H, attn_q_tile(), bc)))
+      return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_ka, h->kc, D, rows, kt, bc))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_va, h->vc, D, rows, kt, bc))) return cleanup(rc);
+  }
   if (h->vtc) {
     const uint64_t rows = static_cast<uint64_t>(L) * cfg->max_batch;
     if ((rc = make_tmap(&h->tm_q, h->qb, D, static_cast<uint64_t>(h->max_M) * H, 128))) return cleanup(rc);

@@ -10,8 +10,11 @@
 // form one [S*H, D] matrix against one key sequence. A CTA takes 64 query rows (4 warps
 // x 16) and one contiguous range of key tiles ("split"); keys are walked segment by
 // segment (static [0, n_static), ring [ring_off, ring_off + n_ring), dynamic
-// [dyn_off, dyn_off + S)), staged through shared memory by a 2-deep cp.async pipeline,
-// and contracted with bf16 mma.sync (fp32 accumulate) with an online softmax in fp32.
+// [dyn_off, dyn_off + S)), staged through shared memory by TMA (Q once, then a 2-deep
+// K/V pipeline on mbarriers, one thread issuing), and contracted with bf16 mma.sync (fp32
+// accumulate) with an online softmax in fp32. Key rows past a segment's end that a tile
+// still covers hold finite data (zero-initialised padding or other cache rows); their
+// scores are masked to -inf, so they get weight exactly 0.
 // The key splits of a query tile form one thread-block cluster: each CTA owns 64/splits
 // query rows and merges the splits' unnormalised partials for them, pushed through
 // distributed shared memory, in split order (deterministic).
@@ -26,16 +29,6 @@
 namespace vla {
 
 constexpr int kQT = 64;   // query rows per CTA
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -64,8 +57,16 @@ template <int D>
 struct AttnCfg {
   static constexpr int KT = D >= 256 ? 32 : 64;            // keys per stage
   static constexpr int CPR = D / 8;                        // 16-byte chunks per row
-  static constexpr int SWZ = (CPR >= 8 ? 8 : CPR) - 1;     // XOR mask for chunk swizzle
-  static constexpr size_t MAIN = (size_t)(kQT + 4 * KT) * D * 2;   // Q + 2 K/V stages
+  // TMA boxes: BW columns wide (128-byte rows with the 128-byte swizzle; 64-byte rows with
+  // the 64-byte swizzle for D = 32), NBOX boxes across a row
+  static constexpr int BW = D >= 64 ? 64 : D;
+  static constexpr int ROWB = BW * 2;
+  static constexpr int CPB = ROWB / 16;                    // 16-byte chunks per box row
+  static constexpr int NBOX = D / BW;
+  static constexpr int Q_BYTES = kQT * D * 2;
+  static constexpr int KV_BYTES = KT * D * 2;              // one K (or V) stage
+  // 1 KB alignment slack, Q, 2 x (K, V) stages, 3 mbarriers
+  static constexpr size_t MAIN = 1024 + (size_t)Q_BYTES + 4 * (size_t)KV_BYTES + 64;
   // split merge: each CTA receives, from every split of its cluster, the unnormalised O
   // rows it owns ([splits][64/splits][D], 64 rows in total) and their (m, l)
   static constexpr size_t RECV_O = (size_t)kQT * D * 4;
@@ -73,11 +74,15 @@ struct AttnCfg {
   static constexpr size_t SMEM = MAIN + RECV_O + RECV_ML + 16;
 };
 
-// byte offset of (row, chunk) in a swizzled [rows][D] bf16 tile
-template <int D>
+// Byte offset of 16-byte chunk `chunk` of row `row` in a [ROWS][D] bf16 tile as TMA
+// writes it: NBOX boxes of [ROWS][ROWB bytes], chunks XOR-swizzled within a row by
+// (row & 7) (128-byte rows) or ((row >> 1) & 3) (64-byte rows).
+template <int D, int ROWS>
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   using C = AttnCfg<D>;
-  return static_cast<uint32_t>((row * C::CPR + (chunk ^ (row & C::SWZ))) * 16);
+  const int box = chunk / C::CPB, w = chunk % C::CPB;
+  const int x = C::ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
+  return static_cast<uint32_t>(box * ROWS * C::ROWB + row * C::ROWB + ((w ^ x) << 4));
 }
 
 // Key tile t of the concatenated segment list -> (segment row offset, first key, count).
@@ -99,16 +104,19 @@ __device__ __forceinline__ void tile_info(const Segs& sg, int t, int& row, int& 
   dyn_start = seg == 2 ? start : -1;
 }
 
+// TMA loads of key tile t (K and V) into stage buffers sk / sv, completing on bar.
 template <int D>
-__device__ __forceinline__ void load_kv_tile(const bf16* kbase, const bf16* vbase, int row, int cnt,
-                                             uint32_t sk, uint32_t sv) {
+__device__ __forceinline__ void issue_kv_tile(const CUtensorMap* tm_k, const CUtensorMap* tm_v, const Segs& sg,
+                                              int t, int row_base, uint32_t sk, uint32_t sv, uint32_t bar,
+                                              uint64_t pol) {
   using C = AttnCfg<D>;
-  for (int idx = threadIdx.x; idx < C::KT * C::CPR; idx += blockDim.x) {
-    const int r = idx / C::CPR, c = idx % C::CPR;
-    const bool ok = r < cnt;
-    const size_t g = static_cast<size_t>(ok ? row + r : row) * D + c * 8;
-    cp_async16(sk + swz<D>(r, c), kbase + g, ok ? 16 : 0);
-    cp_async16(sv + swz<D>(r, c), vbase + g, ok ? 16 : 0);
+  int row, cnt, ds;
+  tile_info<D>(sg, t, row, cnt, ds);
+  mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
+#pragma unroll
+  for (int bx = 0; bx < C::NBOX; ++bx) {
+    tma_load_2d(sk + bx * C::KT * C::ROWB, tm_k, bar, bx * C::BW, row_base + row, pol);
+    tma_load_2d(sv + bx * C::KT * C::ROWB, tm_v, bar, bx * C::BW, row_base + row, pol);
   }
 }
 
@@ -151,37 +159,45 @@ __device__ __forceinline__ void merge_received(const AttnParams& p, const float*
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(128)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D>;
   constexpr int KT = C::KT;
   constexpr int NB = KT / 8;     // 8-key column blocks of S
   constexpr int OB = D / 8;      // 8-dim column blocks of O
-  extern __shared__ __align__(128) uint8_t sm[];
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sQ = smem_u32(sm);
-  const uint32_t sK0 = sQ + kQT * D * 2;
-  const uint32_t sV0 = sK0 + 2 * KT * D * 2;
+  const uint32_t sK0 = sQ + C::Q_BYTES;
+  const uint32_t sV0 = sK0 + 2 * C::KV_BYTES;
+  const uint32_t qbar = sV0 + 2 * C::KV_BYTES;   // then full[0], full[1]
 
   const int qt = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.n_heads, R = p.seq * H;
   const int row0 = qt * kQT;
 
-  float* recv_o = reinterpret_cast<float*>(sm + C::MAIN);
-  float* recv_ml = reinterpret_cast<float*>(sm + C::MAIN + C::RECV_O);
-  const uint32_t recv_bar = smem_u32(sm + C::MAIN + C::RECV_O + C::RECV_ML);
+  float* recv_o = reinterpret_cast<float*>(sm_raw + C::MAIN);
+  float* recv_ml = reinterpret_cast<float*>(sm_raw + C::MAIN + C::RECV_O);
+  const uint32_t recv_bar = smem_u32(sm_raw + C::MAIN + C::RECV_O + C::RECV_ML);
   if (threadIdx.x == 0) {
     trace_stamp(p.trace, 0);
+    mbar_init(qbar, 1);
+    mbar_init(qbar + 8, 1);
+    mbar_init(qbar + 16, 1);
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
     if (p.n_splits > 1) {
       mbar_init(recv_bar, 1);
       mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(C::RECV_O + C::RECV_ML));
-      fence_mbar_init();
     }
+    fence_mbar_init();
     pdl_trigger();
   }
-  if (p.n_splits > 1) {
-    __syncthreads();
-    cluster_sync_all();                      // every receive barrier of the cluster is armed
-  }
+  __syncthreads();
+  if (p.n_splits > 1) cluster_sync_all();    // every receive barrier of the cluster is armed
   pdl_wait();
   if (threadIdx.x == 0) trace_stamp(p.trace, 1);
   const CacheDesc cd = *p.cache;
@@ -201,23 +217,19 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
   const int t_begin = static_cast<int>((static_cast<long long>(split) * T) / p.n_splits);
   const int t_end = static_cast<int>((static_cast<long long>(split + 1) * T) / p.n_splits);
 
-  const bf16* qbase = p.q + static_cast<size_t>(b) * R * D;
-  const bf16* kbase = p.kc + static_cast<size_t>(b) * p.kcap * D;
-  const bf16* vbase = p.vc + static_cast<size_t>(b) * p.kcap * D;
-
-  // Q tile, zero rows past the end
-  for (int idx = threadIdx.x; idx < kQT * C::CPR; idx += blockDim.x) {
-    const int r = idx / C::CPR, c = idx % C::CPR;
-    const bool ok = row0 + r < R;
-    cp_async16(sQ + swz<D>(r, c), qbase + static_cast<size_t>(ok ? row0 + r : 0) * D + c * 8,
-               ok ? 16 : 0);
+  // K/V rows of observation b of this layer in the stacked [L][max_batch][kcap] caches
+  const int kv_base = (p.layer * p.max_batch + b) * p.kcap;
+  if (threadIdx.x == 0) {
+    // Q tile (rows past this observation's R are other rows or zero fill: computed, never
+    // stored), then the first key tile
+    const uint64_t pol = policy_evict_last();
+    mbar_arrive_expect_tx(qbar, C::Q_BYTES);
+#pragma unroll
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_2d(sQ + bx * kQT * C::ROWB, &tm_q, qbar, bx * C::BW, b * R + row0, pol);
+    if (t_begin < t_end) issue_kv_tile<D>(&tm_k, &tm_v, sg, t_begin, kv_base, sK0, sV0, qbar + 8, pol);
   }
-  if (t_begin < t_end) {
-    int row, cnt, ds;
-    tile_info<D>(sg, t_begin, row, cnt, ds);
-    load_kv_tile<D>(kbase, vbase, row, cnt, sK0, sV0);
-  }
-  cp_async_commit();
+  mbar_wait(qbar, 0, p.err);
 
   float o[OB][4];
 #pragma unroll
@@ -231,18 +243,13 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
 
   for (int t = t_begin; t < t_end; ++t) {
     const int st = (t - t_begin) & 1;
-    if (t + 1 < t_end) {
-      int row, cnt, ds;
-      tile_info<D>(sg, t + 1, row, cnt, ds);
-      load_kv_tile<D>(kbase, vbase, row, cnt, sK0 + (st ^ 1) * KT * D * 2, sV0 + (st ^ 1) * KT * D * 2);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
+    // the other stage was released by the __syncthreads that ended the previous tile
+    if (threadIdx.x == 0 && t + 1 < t_end)
+      issue_kv_tile<D>(&tm_k, &tm_v, sg, t + 1, kv_base, sK0 + (st ^ 1) * C::KV_BYTES,
+                       sV0 + (st ^ 1) * C::KV_BYTES, qbar + 8 * (1 + (st ^ 1)), policy_evict_last());
+    mbar_wait(qbar + 8 * (1 + st), ((t - t_begin) >> 1) & 1, p.err);
     if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 6);
-    const uint32_t sK = sK0 + st * KT * D * 2, sV = sV0 + st * KT * D * 2;
+    const uint32_t sK = sK0 + st * C::KV_BYTES, sV = sV0 + st * C::KV_BYTES;
     int trow, tcnt, dyn_start;
     tile_info<D>(sg, t, trow, tcnt, dyn_start);
 
@@ -253,11 +260,11 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t a[4];
-      ldsm_x4(a, sQ + swz<D>(wrow + (lane & 15), kk * 2 + (lane >> 4)));
+      ldsm_x4(a, sQ + swz<D, kQT>(wrow + (lane & 15), kk * 2 + (lane >> 4)));
 #pragma unroll
       for (int nb2 = 0; nb2 < KT / 16; ++nb2) {
         uint32_t bf[4];
-        ldsm_x4(bf, sK + swz<D>(nb2 * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
+        ldsm_x4(bf, sK + swz<D, KT>(nb2 * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
         mma_bf16_16816(sacc[2 * nb2], a, bf[0], bf[1]);
         mma_bf16_16816(sacc[2 * nb2 + 1], a, bf[2], bf[3]);
       }
@@ -316,7 +323,7 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
 #pragma unroll
       for (int db = 0; db < D / 16; ++db) {
         uint32_t vf[4];
-        ldsm_x4_t(vf, sV + swz<D>(kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), db * 2 + (lane >> 4)));
+        ldsm_x4_t(vf, sV + swz<D, KT>(kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), db * 2 + (lane >> 4)));
         mma_bf16_16816(o[2 * db], pa, vf[0], vf[1]);
         mma_bf16_16816(o[2 * db + 1], pa, vf[2], vf[3]);
       }
@@ -419,7 +426,8 @@ cudaError_t configure_attention_kernels() {
 }
 
 template <int D>
-static cudaError_t launch_d(const AttnParams& p, int batch, int q_tiles, cudaStream_t s, bool pdl) {
+static cudaError_t launch_d(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                           const AttnParams& p, int batch, int q_tiles, cudaStream_t s, bool pdl) {
   using C = AttnCfg<D>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(q_tiles, p.n_splits, batch);
@@ -442,17 +450,18 @@ static cudaError_t launch_d(const AttnParams& p, int batch, int q_tiles, cudaStr
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, attn_kernel<D>, p);
+  return cudaLaunchKernelEx(&cfg, attn_kernel<D>, tm_q, tm_k, tm_v, p);
 }
 
-cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
+cudaError_t launch_attention(int head_dim, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const AttnParams& p, int batch, int q_tiles,
                              cudaStream_t s, bool pdl) {
   if (p.n_splits < 1 || p.n_splits > 16 || (p.n_splits & (p.n_splits - 1))) return cudaErrorInvalidValue;
   switch (head_dim) {
-    case 32: return launch_d<32>(p, batch, q_tiles, s, pdl);
-    case 64: return launch_d<64>(p, batch, q_tiles, s, pdl);
-    case 128: return launch_d<128>(p, batch, q_tiles, s, pdl);
-    case 256: return launch_d<256>(p, batch, q_tiles, s, pdl);
+    case 32: return launch_d<32>(tm_q, tm_k, tm_v, p, batch, q_tiles, s, pdl);
+    case 64: return launch_d<64>(tm_q, tm_k, tm_v, p, batch, q_tiles, s, pdl);
+    case 128: return launch_d<128>(tm_q, tm_k, tm_v, p, batch, q_tiles, s, pdl);
+    case 256: return launch_d<256>(tm_q, tm_k, tm_v, p, batch, q_tiles, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -489,6 +498,9 @@ int attn_max_cluster(int head_dim) {
     default: return max_cluster_d<256>();
   }
 }
+
+// TMA box of the attention operands: columns (elements) and swizzle span in bytes
+int attn_box_cols(int head_dim) { return head_dim >= 64 ? 64 : head_dim; }
 
 int attn_key_tile(int head_dim) {
   switch (head_dim) {

@@ -92,12 +92,13 @@ int gemm_stages(int tn);
 
 // ------------------------------------------------------------------ attention
 
+// Operands come through TMA: tm_q over Q [B*S*H rows][D], tm_k / tm_v over the stacked
+// caches [L*max_batch*kcap rows][D], boxes attn_box_cols(D) wide and 64 (Q) or
+// attn_key_tile(D) (K, V) rows high.
 struct AttnParams {
-  const bf16* q;        // [B][S][H][D] (rows (s, h) contiguous per observation)
-  const bf16* kc;       // this layer's K cache [max_batch][kcap][D]
-  const bf16* vc;
   bf16* out;            // [B][S][H][D]
   const CacheDesc* cache;
+  int layer, max_batch;
   int seq, n_heads, kcap;
   int ring_off;         // first ring slot row (= n_static_max)
   int dyn_off;          // first dynamic row (= n_static_max + n_sliding)
@@ -109,8 +110,10 @@ struct AttnParams {
   unsigned long long* trace;   // optional: [ctas][16] %globaltimer stamps, or null
 };
 
-cudaError_t launch_attention(int head_dim, const AttnParams& p, int batch, int q_tiles,
+cudaError_t launch_attention(int head_dim, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, const AttnParams& p, int batch, int q_tiles,
                              cudaStream_t s, bool pdl);
+int attn_box_cols(int head_dim);         // TMA box width of the attention operands
 int attn_q_tile();                       // query rows per CTA
 cudaError_t configure_attention_kernels();
 cudaError_t configure_small_kernels();
