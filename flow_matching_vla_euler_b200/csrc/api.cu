@@ -540,7 +540,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.ld_out = h->HD;
           p.kc = h->kc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
           p.vc = h->vc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
-          p.vtc = h->vtc ? h->vtc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D : nullptr;
+          p.vtc = nullptr;   // the transposed V of the chunk is written by launch_vt_dyn below
           p.kcap = h->kcap;
           p.dyn_off = h->dyn_off;
           p.seq = h->S;
@@ -571,6 +571,12 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h->D));
           a.err = h->err;
           a.trace = tr(1);
+          if (use_tc_attn) {   // transposed V of the chunk (counted with attention)
+            const size_t lofs = static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
+            rec.begin(VLA_K_ATTN);
+            CU(launch_vt_dyn(p.vc, h->vtc + lofs, B, h->D, h->kcap, h->dyn_off, h->S, rec.s, pdl));
+            rec.end(VLA_K_ATTN);
+          }
           rec.begin(VLA_K_ATTN);
           if (use_tc_attn) {
             AttnTcParams t{};
