@@ -20,6 +20,7 @@ VLA_OK, VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_STATE = 0, 1, 2, 3
 VLA_ERR_OOM, VLA_ERR_CUDA, VLA_ERR_TIMEOUT, VLA_ERR_UNSUPPORTED = 4, 5, 6, 7
 VLA_TIME_PI0_MLP, VLA_TIME_ADA_SINCOS, VLA_TIME_ADA_MLP = 0, 1, 2
 VLA_FLAG_NO_PDL = 1
+VLA_FLAG_NORM_KERNELS = 2
 KERNEL_KINDS = ["gemm_qkv", "attention", "gemm_o", "gemm_gateup", "gemm_down", "norm", "embed",
                 "final_euler", "time_mlp"]
 

@@ -282,6 +282,7 @@ int validate(const vla_config* c, const vla_weights* w) {
   if (c->max_steps < 1 || c->max_steps > kMaxSteps)
     return fail(VLA_ERR_SHAPE, "max_steps must be in [1, %d]", kMaxSteps);
   if (!(c->eps > 0.0f)) return fail(VLA_ERR_ARG, "eps must be > 0");
+  if (c->flags & ~(VLA_FLAG_NO_PDL | VLA_FLAG_NORM_KERNELS)) return fail(VLA_ERR_ARG, "unknown flag bits 0x%x", c->flags);
   const bool need_common = w->action_in_w && w->action_in_b && w->action_out_w && w->action_out_b &&
                            w->wq && w->wk && w->wv && w->wo && w->w_gate && w->w_up && w->w_down;
   if (!need_common) return fail(VLA_ERR_ARG, "missing a projection weight");
@@ -390,12 +391,16 @@ struct Recorder {
   }
 };
 
-// Sum-of-squares contributor rows a push-mode residual epilogue writes for this plan.
-int contributors(const GemmPlan& g) { return g.n_tiles * g.m_tiles * g.splits * (g.splits == 1 ? 2 : 1); }
-
 GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
   const int tn = plan_gemm(n_feat, k_dim, M, h->sm_count).tn;
   return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, cluster_cap(h, tn));
+}
+
+// Sum-of-squares contributor rows a push-mode residual epilogue (one token tile) writes
+// per token: one per (weight tile, split owner, 32-row group).
+int contributors(const vla_expert* h, int n_feat, int k_dim, int M) {
+  const GemmPlan g = denoise_plan(h, n_feat, k_dim, M);
+  return g.n_tiles * g.m_tiles * g.splits * (g.splits == 1 ? 2 : 1);
 }
 
 int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensorMap& tw,
@@ -445,9 +450,11 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
   // tensor-core attention once every 128-row query tile has a CTA of its own
   const bool use_tc_attn = h->vtc && B * cdiv(h->S * h->H, attn_tc_q_tile()) >= h->sm_count;
   const float dt = -1.0f / static_cast<float>(steps);
-  // All suffix tokens in one 64-token tile: the norms are fused into the QKV and gate/up
-  // GEMMs, fed by per-token sum-of-squares partials from the residual writers.
-  const bool fused = M <= 64;
+  // All suffix tokens in one 64-token tile: the norms are folded into the QKV and gate/up
+  // GEMMs, fed by per-token sum-of-squares partials from the residual writers (unless norm
+  // kernels are asked for). With several token tiles the persistent GEMMs' epilogues are
+  // the bottleneck and separate norm kernels are faster (measured at batch 64).
+  const bool fused = M <= 64 && !(h->cfg.flags & VLA_FLAG_NORM_KERNELS);
   const long cw = h->qkv_rows + 2L * h->F;
   // modulation the next norm applies to z: AdaRMSNorm (1 + scale_j) or RMSNorm (1 + w)
   auto zmod = [&](const float* tk, int j) -> const float* {
@@ -455,9 +462,9 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
     if (h->ada) return tk + (static_cast<long>(j) * 3 + 0) * W;
     return ((j & 1) ? h->n2_w : h->n1_w) + static_cast<long>(j / 2) * W;
   };
-  const int n_mlp2 = contributors(denoise_plan(h, W, W, M));
-  const int n_o = contributors(denoise_plan(h, W, h->HD, M));
-  const int n_down = contributors(denoise_plan(h, W, h->F, M));
+  const int n_mlp2 = contributors(h, W, W, M);
+  const int n_o = contributors(h, W, h->HD, M);
+  const int n_down = contributors(h, W, h->F, M);
   for (int k = 0; k < steps; ++k) {
     const float* tk = tbl + static_cast<long>(k) * h->table_stride;
     EmbedParams e{};

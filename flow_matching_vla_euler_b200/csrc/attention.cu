@@ -93,15 +93,17 @@ struct Segs {
 template <int D>
 __device__ __forceinline__ void tile_info(const Segs& sg, int t, int& row, int& cnt, int& dyn_start) {
   using C = AttnCfg<D>;
-  int seg = 0;
-  while (seg < 2 && t >= sg.ntile[seg]) {
-    t -= sg.ntile[seg];
-    ++seg;
-  }
-  const int start = t * C::KT;
-  row = sg.off[seg] + start;
-  cnt = min(C::KT, sg.cnt[seg] - start);
-  dyn_start = seg == 2 ? start : -1;
+  // segment selection by compares and selects (no indexing of the arrays by a run-time value,
+  // which would place them in local memory)
+  const bool s0 = t < sg.ntile[0];
+  const bool s1 = !s0 && t < sg.ntile[0] + sg.ntile[1];
+  const int first = s0 ? 0 : (s1 ? sg.ntile[0] : sg.ntile[0] + sg.ntile[1]);
+  const int off = s0 ? sg.off[0] : (s1 ? sg.off[1] : sg.off[2]);
+  const int n = s0 ? sg.cnt[0] : (s1 ? sg.cnt[1] : sg.cnt[2]);
+  const int start = (t - first) * C::KT;
+  row = off + start;
+  cnt = min(C::KT, n - start);
+  dyn_start = (!s0 && !s1) ? start : -1;
 }
 
 // TMA loads of key tile t (K and V) into stage buffers sk / sv, completing on bar.

@@ -73,6 +73,10 @@ typedef enum vla_time_kind {
 
 /* Option bits for vla_config.flags. */
 #define VLA_FLAG_NO_PDL 1u      /* launch without programmatic dependent launch edges */
+#define VLA_FLAG_NORM_KERNELS 2u /* with one token tile (batch x suffix <= 64), run the
+                                    pre-attention / pre-MLP norms as kernels of their own
+                                    instead of folding them into the projections (cross-check;
+                                    larger batches always use norm kernels) */
 
 typedef struct vla_config {
   int n_layers;      /* L */

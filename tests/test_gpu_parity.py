@@ -67,6 +67,35 @@ def test_repeat_calls_are_bit_identical_and_pdl_free_equal():
     assert np.array_equal(a, c)
 
 
+def test_norm_kernels_path_matches_folded_norms():
+    """Norms folded into the projections (z = bf16(r (1 + mod)), rinv from partial sums of
+    squares, W.shift added in the epilogue) against separate norm kernels, on one token
+    tile: tiny and mid_d128 (AdaRMSNorm), and observation 0 of mid_pi0_b3 alone (RMSNorm,
+    Pi0 time MLP, state token; 51 tokens). Both within tolerance of the oracle and of each
+    other."""
+    from dataclasses import replace
+    import flow_matching_vla_euler_b200 as V
+    for name, obs in (("tiny", None), ("mid_d128", None), ("mid_pi0_b3", 1)):
+        wl = get(name)
+        inp = make_inputs(wl)
+        ref = golden_actions(name)
+        if obs is not None:
+            wl = replace(wl, batch=obs)
+            inp = dict(inp, noise=inp["noise"][:obs], prefix_k=inp["prefix_k"][:, :obs],
+                       prefix_v=inp["prefix_v"][:, :obs])
+            if inp.get("state") is not None:
+                inp["state"] = inp["state"][:obs]
+            ref = ref[:obs]
+        outs = []
+        for flags in (0, V.VLA_FLAG_NORM_KERNELS):
+            ex, _ = make_expert(wl, inp, flags=flags)
+            load_prefix(ex, inp)
+            outs.append(run(ex, inp, wl.steps))
+        check_actions(outs[0], ref, name + " folded")
+        check_actions(outs[1], ref, name + " norm kernels")
+        check_actions(outs[0], outs[1], name + " folded vs norm kernels")
+
+
 def test_batch_rows_match_single_observation_runs():
     wl = get("mid_ada_b2")
     ex, inp = make_expert(wl)
