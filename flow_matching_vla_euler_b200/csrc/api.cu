@@ -152,7 +152,7 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 struct vla_expert {
   vla_config cfg;
   int dev = 0, sm_count = 148;
-  int gemm_cluster[3] = {1, 1, 1};   // largest split cluster for token tiles 64 / 128 / 256
+  int gemm_cluster = 1;   // largest split cluster of the 64-token push GEMM
   int attn_cluster = 1;
   int L, W, H, D, F, A, C, Sd, S, hs, HD, Td, Cd, qkv_rows, kcap, ring_off, dyn_off, max_M;
   bool ada, pi0;
@@ -213,9 +213,6 @@ struct vla_expert {
 
 namespace {
 
-int cluster_cap(const vla_expert* h, int tn) {
-  return h->gemm_cluster[tn == 64 ? 0 : (tn == 128 ? 1 : 2)];
-}
 
 template <typename T>
 int dalloc(vla_expert* h, T** p, size_t count) {
@@ -393,7 +390,7 @@ struct Recorder {
 
 GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
   const int tn = plan_gemm(n_feat, k_dim, M, h->sm_count).tn;
-  return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, cluster_cap(h, tn));
+  return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, tn == 64 ? h->gemm_cluster : 1);
 }
 
 // Sum-of-squares contributor rows a push-mode residual epilogue (one token tile) writes
@@ -800,9 +797,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   h->dyn_off = h->ring_off + cdiv(cfg->n_sliding, 64) * 64;
   h->kcap = cdiv(h->dyn_off + h->S, 64) * 64;
   h->max_M = cfg->max_batch * h->S;
-  h->gemm_cluster[0] = gemm_max_cluster(64);
-  h->gemm_cluster[1] = gemm_max_cluster(128);
-  h->gemm_cluster[2] = gemm_max_cluster(256);
+  h->gemm_cluster = gemm_max_cluster();
   h->attn_cluster = attn_max_cluster(h->D);
   const int L = h->L, W = h->W, H = h->H, D = h->D, F = h->F, DH = D / 2;
 

@@ -229,46 +229,6 @@ __device__ __forceinline__ void epi_pair(const GemmParams& p, int fn0, int m, fl
   }
 }
 
-// Sum of rows [row0, row0 + 128/S) of the S partial tiles of this cluster (rank order,
-// so the result does not depend on timing), then the epilogue on row pairs. Loads of
-// G items x S ranks are issued before any add so the distributed-shared-memory latency
-// is paid once per group, not once per rank.
-template <int EPI, int TN, int S>
-__device__ __forceinline__ void cluster_reduce(const GemmParams& p, uint32_t part, int etid, int row0,
-                                               int fbase, int m0) {
-  constexpr int HALF = 64 / S;                 // row pairs per rank
-  constexpr int ITEMS = HALF * TN;             // (row pair, token) items per rank
-  constexpr int G = S >= 16 ? 1 : 16 / S;      // items per group
-  uint32_t peer[S];
-#pragma unroll
-  for (int q = 0; q < S; ++q) peer[q] = mapa_shared(part, q);
-  for (int base = etid; base < ITEMS; base += 128 * G) {
-    float2 t[G][S];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int it = base + g * 128;
-      const int rp = it % HALF, c = it / HALF;
-      const uint32_t off = static_cast<uint32_t>((c * 128 + row0 + 2 * rp) * 4);
-#pragma unroll
-      for (int q = 0; q < S; ++q)
-        t[g][q] = it < ITEMS ? ld_dsmem_f2(peer[q] + off) : make_float2(0.0f, 0.0f);
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int it = base + g * 128;
-      if (it >= ITEMS) break;
-      float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll
-      for (int q = 0; q < S; ++q) {
-        v0 += t[g][q].x;
-        v1 += t[g][q].y;
-      }
-      const int rp = it % HALF, c = it / HALF;
-      epi_pair<EPI>(p, fbase + 2 * rp, m0 + c, v0, v1);
-    }
-  }
-}
-
 // Push-mode reduction, token tile 64: every CTA of the cluster has sent rows
 // [q*128/S, (q+1)*128/S) of its partial tile to CTA q (receive slots = the other ranks in
 // rank order); the owner sums its S partials in rank order (deterministic) and runs the
@@ -412,6 +372,7 @@ __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                    const GemmParams p) {
   using G = GemmCfg<TN, CL>;
+  static_assert(!CL || TN == 64, "cluster (split-K push) kernels take one 64-token tile");
   static_assert(!G::PUSH || G::push_need(1) <= 2 * G::STAGE_BYTES,
                 "the partial tile fits in two idle pipeline stages");
   extern __shared__ uint8_t smem_raw[];
@@ -438,7 +399,6 @@ __global__ void __launch_bounds__(320, 1)
     kb0 = split * p.kb_per_split;
     nkb = min(p.kb_per_split, nkb_total - kb0);
   }
-  const bool cluster_red = CL && p.splits > 1;
   const bool push = G::PUSH;                 // token tile 64: always through the receive buffer
 
   const uint32_t full0 = smem_u32(&bar[0]);
@@ -640,19 +600,6 @@ __global__ void __launch_bounds__(320, 1)
       }
     } else if (!main4) {
       // not needed outside the push path
-    } else if (cluster_red) {
-      // partial tile -> own shared memory, [token][row] fp32 (the pipeline buffers are idle)
-      float* part = reinterpret_cast<float*>(smem);
-      for (int c = 0; c < TN; c += 16) {
-        float v[16];
-        tmem_ld16(taddr + c, v);
-        if (nkb == 0) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) part[(c + j) * 128 + r] = v[j];
-      }
     } else {
       bool last = true;
       if (p.splits > 1) {
@@ -696,27 +643,6 @@ __global__ void __launch_bounds__(320, 1)
         if (p.splits > 1 && etid == 0) p.counters[tile] = 0;
       }
     }
-  }
-
-  if (cluster_red && !push) {
-    if (threadIdx.x == 64) trace_stamp(p.trace, 6);
-    cluster_sync_all();                      // every partial tile is in its CTA's smem
-    if (threadIdx.x == 64) trace_stamp(p.trace, 7);
-    if (warp >= 2 && warp < 6) {
-      const int etid = (warp - 2) * 32 + lane;
-      const int row0 = static_cast<int>(cluster_ctarank()) * (128 / p.splits);
-      const uint32_t part = smem_u32(smem);
-      const int m0 = m_tile * TN, fbase = n_tile * G::BM + row0;
-      switch (p.splits) {
-        case 2: cluster_reduce<EPI, TN, 2>(p, part, etid, row0, fbase, m0); break;
-        case 4: cluster_reduce<EPI, TN, 4>(p, part, etid, row0, fbase, m0); break;
-        case 8: cluster_reduce<EPI, TN, 8>(p, part, etid, row0, fbase, m0); break;
-        default: cluster_reduce<EPI, TN, 16>(p, part, etid, row0, fbase, m0); break;
-      }
-    }
-    if (threadIdx.x == 64) trace_stamp(p.trace, 8);
-    cluster_sync_all();                      // peers finished reading this CTA's smem
-    if (threadIdx.x == 64) trace_stamp(p.trace, 9);
   }
 
   tc_fence_before();
@@ -965,8 +891,6 @@ cudaError_t configure_gemm_kernels() {
   if ((e = configure_tn<128, false>()) != cudaSuccess) return e;
   if ((e = configure_tn<256, false>()) != cudaSuccess) return e;
   if ((e = configure_tn<64, true>()) != cudaSuccess) return e;
-  if ((e = configure_tn<128, true>()) != cudaSuccess) return e;
-  if ((e = configure_tn<256, true>()) != cudaSuccess) return e;
   if ((e = configure_persist_tn<128>()) != cudaSuccess) return e;
   if ((e = configure_persist_tn<256>()) != cudaSuccess) return e;
   done = cudaSuccess;
@@ -975,43 +899,26 @@ cudaError_t configure_gemm_kernels() {
 
 // Largest cluster (power of two <= 16) that the device can co-schedule for the
 // TN-token kernel.
-int gemm_max_cluster(int tn) {
+int gemm_max_cluster() {
   if (configure_gemm_kernels() != cudaSuccess) return 1;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = GemmCfg<64, true>::SMEM;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  int best = 1;
   for (int c = 16; c >= 2; c >>= 1) {
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = c;
     cfg.gridDim = dim3(1, 1, c);
     int n = 0;
-    cudaError_t e;
-    switch (tn) {
-      case 64:
-        cfg.dynamicSmemBytes = GemmCfg<64, true>::SMEM;
-        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<64, EPI_RESID, true>, &cfg);
-        break;
-      case 128:
-        cfg.dynamicSmemBytes = GemmCfg<128, true>::SMEM;
-        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<128, EPI_RESID, true>, &cfg);
-        break;
-      default:
-        cfg.dynamicSmemBytes = GemmCfg<256, true>::SMEM;
-        e = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<256, EPI_RESID, true>, &cfg);
-        break;
-    }
-    if (e == cudaSuccess && n > 0) {
-      best = c;
-      break;
-    }
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<64, EPI_RESID, true>, &cfg) == cudaSuccess && n > 0)
+      return c;
     cudaGetLastError();
   }
-  return best;
+  return 1;
 }
 
 template <int TN, int EPI, bool CL>
@@ -1076,30 +983,17 @@ static cudaError_t launch_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap
 cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                         const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl,
                         bool cluster) {
-  if (cluster && (p.splits & (p.splits - 1))) return cudaErrorInvalidValue;   // power of two
+  if (cluster) {
+    // split-K push kernels: one 64-token tile, a power-of-two split count
+    if (tn != 64 || (p.splits & (p.splits - 1))) return cudaErrorInvalidValue;
+    return launch_tn<64, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+  }
   switch (tn) {
-    case 64:
-      return cluster ? launch_tn<64, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
-                     : launch_tn<64, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case 128:
-      return cluster ? launch_tn<128, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
-                     : launch_tn<128, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
-    case 256:
-      return cluster ? launch_tn<256, true>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl)
-                     : launch_tn<256, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 64: return launch_tn<64, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 128: return launch_tn<128, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+    case 256: return launch_tn<256, false>(epi, tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
-
-size_t gemm_smem_bytes(int tn) {
-  switch (tn) {
-    case 64: return GemmCfg<64, false>::SMEM;
-    case 128: return GemmCfg<128, false>::SMEM;
-    case 256: return GemmCfg<256, false>::SMEM;
-    default: return 0;
-  }
-}
-
-int gemm_stages(int) { return 4; }
 
 }  // namespace vla

@@ -75,20 +75,19 @@ struct GemmParams {
 };
 
 // tn: token tile (64, 128 or 256). cluster = false: split partials through p.ws /
-// p.counters (any split count); cluster = true: the splits (a power of two, at most
-// gemm_max_cluster(tn)) of a tile form a cluster and reduce in distributed shared memory.
+// p.counters (any split count); cluster = true (tn 64 only): the splits (a power of two,
+// at most gemm_max_cluster()) of a tile form a cluster, each pushes its partial rows to
+// their owners' shared memory, and the owners reduce them in rank order.
 cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                         const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s, bool pdl,
                         bool cluster = false);
 
-int gemm_max_cluster(int tn);
+int gemm_max_cluster();   // largest co-schedulable cluster of the 64-token push kernel
 // Persistent launch over n_tiles x m_tiles output tiles (splits must be 1), grid CTAs;
 // tn 128 or 256, two TMEM accumulators so epilogues overlap the next tile's main loop.
 cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                    const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl);
-size_t gemm_smem_bytes(int tn);
 cudaError_t configure_gemm_kernels();
-int gemm_stages(int tn);
 
 // ------------------------------------------------------------------ attention
 
