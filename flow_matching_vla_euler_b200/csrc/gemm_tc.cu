@@ -10,14 +10,18 @@
 // Orientation: the 128-row MMA operand A is a tile of WEIGHT rows (output features), the
 // N side is a tile of TN tokens, so the accumulator D[feature][token] lives in TMEM with
 // one output feature per TMEM lane. At batch 1 (50 tokens) this keeps the 128-wide M side
-// full; K is split across CTAs so that >= 148 SMs stream weights, and the last CTA to
-// finish a tile sums the partial tiles in split order (deterministic) and runs the
-// epilogue.
+// full, and K is split across the CTAs of a thread-block cluster so that >= 148 SMs stream
+// weights: each CTA stages its fp32 partial tile in shared memory and pushes the rows of
+// each owner (rank q owns rows [q*128/S, (q+1)*128/S)) into q's receive buffer with bulk
+// copies to distributed shared memory; the owner sums the S partials in rank order
+// (deterministic) and runs the epilogue. Without a cluster (the standalone GEMM) split
+// partials go through a global workspace and the last CTA of a tile sums them. Several
+// token tiles use the persistent variant at the end of this file.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
-// tcgen05.mma, warps 2..5 drain TMEM (tcgen05.ld) and run the epilogue (the persistent
-// variant below uses eight epilogue warps). Every wait is
-// bounded: on timeout the kernel sets the status word and winds down.
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
+// tcgen05.mma, warps 2..9 drain TMEM (tcgen05.ld) and run the epilogue (push path: all
+// eight; workspace path: warps 2..5). Every wait is bounded: on timeout the kernel sets
+// the status word and winds down.
 #include <cstdio>
 
 #include "kernels.h"
