@@ -146,7 +146,7 @@ __device__ __forceinline__ void merge_received(const AttnParams& p, const float*
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
     for (int q = 0; q < NS; ++q) {
-      const float w = (ml[q].x == -INFINITY) ? 0.0f : exp2f(ml[q].x - M);
+      const float w = (ml[q].x == -INFINITY) ? 0.0f : exp2_approx(ml[q].x - M);
       wsum += w * ml[q].y;
       acc.x += w * v[q].x;
       acc.y += w * v[q].y;
@@ -271,6 +271,7 @@ __global__ void __launch_bounds__(128)
         mma_bf16_16816(sacc[2 * nb2 + 1], a, bf[2], bf[3]);
       }
     }
+    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 8);
     // scale into the log2 domain and mask
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(128)
       mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
       mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
       const float m_new = fmaxf(m_run[h2], mx[h2]);
-      corr[h2] = (m_run[h2] == -INFINITY) ? 0.0f : exp2f(m_run[h2] - m_new);
+      corr[h2] = (m_run[h2] == -INFINITY) ? 0.0f : exp2_approx(m_run[h2] - m_new);
       m_run[h2] = m_new;
     }
     float lsum[2] = {0.0f, 0.0f};
@@ -300,20 +301,23 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float mref = m_run[e >> 1];
-        const float pv = (mref == -INFINITY) ? 0.0f : exp2f(sacc[nb][e] - mref);
+        const float pv = (mref == -INFINITY) ? 0.0f : exp2_approx(sacc[nb][e] - mref);
         sacc[nb][e] = pv;
         lsum[e >> 1] += pv;
       }
     }
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) l_run[h2] = l_run[h2] * corr[h2] + lsum[h2];
+    if (!__all_sync(0xffffffffu, corr[0] == 1.0f && corr[1] == 1.0f)) {   // the running max moved
 #pragma unroll
-    for (int i = 0; i < OB; ++i) {
-      o[i][0] *= corr[0];
-      o[i][1] *= corr[0];
-      o[i][2] *= corr[1];
-      o[i][3] *= corr[1];
+      for (int i = 0; i < OB; ++i) {
+        o[i][0] *= corr[0];
+        o[i][1] *= corr[0];
+        o[i][2] *= corr[1];
+        o[i][3] *= corr[1];
+      }
     }
+    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 9);
     // O += P V
 #pragma unroll
     for (int kb = 0; kb < KT / 16; ++kb) {
@@ -330,6 +334,7 @@ __global__ void __launch_bounds__(128)
         mma_bf16_16816(o[2 * db + 1], pa, vf[2], vf[3]);
       }
     }
+    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 10);
     __syncthreads();
     if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 7);
   }
