@@ -255,10 +255,13 @@ __global__ void __launch_bounds__(128)
     int trow, tcnt, dyn_start;
     tile_info<D>(sg, t, trow, tcnt, dyn_start);
 
-    // S = Q K^T for this warp's 16 rows x KT keys
-    float sacc[NB][4];
+    // S = Q K^T for this warp's 16 rows x KT keys; even and odd 16-wide K steps accumulate
+    // separately (two dependent MMA chains of D/32 instead of one of D/16), summed after
+    float sacc[NB][4], sodd[NB][4];
 #pragma unroll
-    for (int i = 0; i < NB; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.0f;
+    for (int i = 0; i < NB; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[i][e] = sodd[i][e] = 0.0f;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       uint32_t a[4];
@@ -267,10 +270,16 @@ __global__ void __launch_bounds__(128)
       for (int nb2 = 0; nb2 < KT / 16; ++nb2) {
         uint32_t bf[4];
         ldsm_x4(bf, sK + swz<D, KT>(nb2 * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
-        mma_bf16_16816(sacc[2 * nb2], a, bf[0], bf[1]);
-        mma_bf16_16816(sacc[2 * nb2 + 1], a, bf[2], bf[3]);
+        float (&acc0)[4] = (kk & 1) ? sodd[2 * nb2] : sacc[2 * nb2];
+        float (&acc1)[4] = (kk & 1) ? sodd[2 * nb2 + 1] : sacc[2 * nb2 + 1];
+        mma_bf16_16816(acc0, a, bf[0], bf[1]);
+        mma_bf16_16816(acc1, a, bf[2], bf[3]);
       }
     }
+#pragma unroll
+    for (int i = 0; i < NB; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[i][e] += sodd[i][e];
     if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 8);
     // scale into the log2 domain and mask
     float mx[2] = {-INFINITY, -INFINITY};
