@@ -200,8 +200,9 @@ __global__ void __launch_bounds__(128)
   }
   __syncthreads();
   if (p.n_splits > 1) cluster_sync_all();    // every receive barrier of the cluster is armed
-  pdl_wait();
-  if (threadIdx.x == 0) trace_stamp(p.trace, 1);
+  // The cache descriptor and the static / ring regions were written before this denoise
+  // started (set_prefix / append calls), so they can be read before the dependency wait;
+  // Q and the dynamic region come from the QKV launch just before this one.
   const CacheDesc cd = *p.cache;
   Segs sg;
   sg.off[0] = 0;
@@ -218,18 +219,22 @@ __global__ void __launch_bounds__(128)
   }
   const int t_begin = static_cast<int>((static_cast<long long>(split) * T) / p.n_splits);
   const int t_end = static_cast<int>((static_cast<long long>(split + 1) * T) / p.n_splits);
-
   // K/V rows of observation b of this layer in the stacked [L][max_batch][kcap] caches
   const int kv_base = (p.layer * p.max_batch + b) * p.kcap;
+  const bool first_dynamic = t_begin < t_end && t_begin >= sg.ntile[0] + sg.ntile[1];
+  if (threadIdx.x == 0 && t_begin < t_end && !first_dynamic)   // a cached tile: load it now
+    issue_kv_tile<D>(&tm_k, &tm_v, sg, t_begin, kv_base, sK0, sV0, qbar + 8, policy_evict_last());
+  pdl_wait();
   if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 1);
     // Q tile (rows past this observation's R are other rows or zero fill: computed, never
-    // stored), then the first key tile
+    // stored), then the first key tile if it is the chunk's own
     const uint64_t pol = policy_evict_last();
     mbar_arrive_expect_tx(qbar, C::Q_BYTES);
 #pragma unroll
     for (int bx = 0; bx < C::NBOX; ++bx)
       tma_load_2d(sQ + bx * kQT * C::ROWB, &tm_q, qbar, bx * C::BW, b * R + row0, pol);
-    if (t_begin < t_end) issue_kv_tile<D>(&tm_k, &tm_v, sg, t_begin, kv_base, sK0, sV0, qbar + 8, pol);
+    if (first_dynamic) issue_kv_tile<D>(&tm_k, &tm_v, sg, t_begin, kv_base, sK0, sV0, qbar + 8, pol);
   }
   mbar_wait(qbar, 0, p.err);
 
