@@ -189,6 +189,14 @@ def max_over_ranks(x: float, ws: int, device=None) -> float:
     return float(t.item())
 
 
+def job_timing(total_ms: float, steps: int, ws: int, device=None):
+    """Whole-job timing from each rank's device time for `steps` timed denoises: the
+    slowest rank's time, its ms per step, and the whole-job ms per denoise (all ranks'
+    denoises over that time)."""
+    t_max = max_over_ranks(total_ms, ws, device)
+    return t_max, t_max / steps, t_max / (steps * ws)
+
+
 # --------------------------------------------------------------- workload set-up
 
 def build_expert(wl, inp):
@@ -375,9 +383,7 @@ def run_ours(args):
         total_ms, per, _ = time_device(ex, noise, state, steps, args.steps, args.warmup, ws)
     clocks = clk.summary()
     ex.device_status()
-    t_max = max_over_ranks(total_ms, ws)
-    ms_per_step = t_max / args.steps
-    value = t_max / (args.steps * ws)
+    t_max, ms_per_step, value = job_timing(total_ms, args.steps, ws)
     e2e = None
     if not args.no_e2e:
         k_e = max(10, args.steps // 4)

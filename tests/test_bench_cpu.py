@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py, on CPU: the multi-process (replica) timing reduction over a
+world-size-2 gloo group, and the reference arm's JSON line (the fp64 oracle on the host
+cores) for the small workload."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, ws, port, out_dir):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(ws)
+        # rank r spent 100 + 50 r ms on 4 denoises: the slowest rank decides
+        t_max, per_step, value = bench.job_timing(100.0 + 50.0 * rank, 4, ws, device="cpu")
+        # the reference arm runs on rank 0 only; the other ranks return at once
+        rc = bench.run_reference(bench.parse_args(["--impl", "reference", "--workload", "tiny"])) if rank else 0
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"t_max": t_max, "per_step": per_step, "value": value, "rc": rc}, f)
+        bench.barrier(ws)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replica_timing_takes_the_max_over_ranks(tmp_path):
+    import torch.multiprocessing as mp
+    ws = 2
+    mp.start_processes(_rank_main, args=(ws, _free_port(), str(tmp_path)), nprocs=ws, join=True,
+                       start_method="spawn")
+    for r in range(ws):
+        d = json.load(open(tmp_path / f"r{r}.json"))
+        assert d["t_max"] == 150.0 and d["per_step"] == 37.5
+        assert d["value"] == 150.0 / (4 * ws)      # whole-job ms per denoise
+        assert d["rc"] == 0
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["higher_is_better"] is False and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "tiny"
