@@ -63,11 +63,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_text(src: str) -> str:
+    """C++/CUDA source with comments and blank lines removed (a comment edit does not
+    change the kernel, so it must not invalidate its ncu counters)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(l.rstrip() for l in src.splitlines() if l.strip())
+
+
 def source_sha(files):
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(code_text(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -427,9 +427,9 @@ int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensor
   p.w_stream = g.m_tiles == 1 ? 1 : 0;   // weights reused by every token tile stay in L2
   p.err = h->err;
   p.ld_rstat = h->max_M;
-  // Shared-memory budget (pipeline stages, at most 3 = 98..104 KB per CTA) so that a CTA
-  // fits on an SM beside one of the kernel before it and starts streaming its weights
-  // early; gate/up (two CTAs per SM) and O at 2..3 stages
+  // Shared-memory budget: at most 3 pipeline stages (about 80-104 KB per CTA with the
+  // receive slots), so that a CTA can share its SM with one of another projection and
+  // start streaming its weights while that one runs
   p.stages = 3;
   rec.begin(kind);
   CU(launch_gemm(g.tn, epi, tw, tx, p, g.n_tiles, g.m_tiles, rec.s, pdl, true));

@@ -368,9 +368,9 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
 
 // CL = false: one CTA per (tile, split); split partials, if any, go through the global
 // workspace p.ws and the last CTA of a tile to arrive sums them (any split count).
-// CL = true: the p.splits CTAs of a tile are one thread-block cluster; each leaves its
-// partial tile in its own shared memory and CTA rank r sums rows [r*128/S, (r+1)*128/S)
-// over all ranks through distributed shared memory, in rank order (deterministic).
+// CL = true (TN = 64): the p.splits CTAs of a tile are one thread-block cluster; each
+// stages its partial tile in its own shared memory and pushes rows [r*128/S, (r+1)*128/S)
+// to CTA rank r, which sums the S partials in rank order (deterministic).
 template <int TN, int EPI, bool CL>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
