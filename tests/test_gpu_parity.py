@@ -125,6 +125,38 @@ def test_step_counts_and_host_entry_point():
     assert np.array_equal(host, run(ex, inp, 4))
 
 
+def test_prefix_lengths_below_capacity_and_empty():
+    """The static region holds fewer keys than its capacity: a prefix of P keys, a longer
+    one (P + 20) and P again on the same handle and captured graph, and an empty prefix
+    (the chunk attends to itself only). Each run matches the oracle on exactly its keys;
+    rows left over from the longer prefix are masked out exactly (bit-identical rerun);
+    more keys than the capacity are refused."""
+    import flow_matching_vla_euler_b200 as V
+    wl = get("tiny")
+    inp = make_inputs(wl)
+    ex = V.Expert(wl.expert, inp["params"], n_static_max=wl.n_static + 37, max_batch=wl.batch,
+                  max_steps=wl.steps)
+    pk, pv = inp["prefix_k"], inp["prefix_v"]
+    load_prefix(ex, inp)
+    a = run(ex, inp, wl.steps)
+    check_actions(a, golden_actions("tiny"), "tiny, capacity + 37")
+    longer = dict(inp, prefix_k=np.concatenate([pk, pk[:, :, :20]], axis=2),
+                  prefix_v=np.concatenate([pv, pv[:, :, :20]], axis=2))
+    load_prefix(ex, longer)
+    check_actions(run(ex, longer, wl.steps), oracle_actions(wl, longer), "tiny, P + 20 keys")
+    load_prefix(ex, inp)
+    assert np.array_equal(run(ex, inp, wl.steps), a)
+    empty = dict(inp, prefix_k=pk[:, :, :0], prefix_v=pv[:, :, :0])
+    load_prefix(ex, empty)
+    check_actions(run(ex, empty, wl.steps), oracle_actions(wl, empty), "tiny, empty prefix")
+    too_many = np.concatenate([pk, pk], axis=2)
+    with pytest.raises(V.VlaError) as e:
+        load_prefix(ex, dict(inp, prefix_k=too_many, prefix_v=too_many))
+    assert e.value.code == V.VLA_ERR_SHAPE
+    ex.device_status()
+    ex.close()
+
+
 def test_error_paths_on_device():
     import torch
     import flow_matching_vla_euler_b200 as V
