@@ -290,16 +290,20 @@ def roofline(ex, noise, state, steps, peaks, peak_src, workload, bound, reps=3):
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
     else:
+        # the kernel is timed inside a whole denoise (a long step), so its denominator is
+        # the sustained bf16 figure; the burst one is reported beside it
         achieved = d["flops"] / max(1, d["launches"]) / (per_launch_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit = "TFLOP/s"
     tr = ncu_traffic(dom, workload)
+    extra = {} if bound == "hbm" else {"frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                                        "burst_peak": peaks["bf16_tflops"]}
     return {"kernel": dom, "bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": tr,
+            "frac": round(achieved / peak, 4), "traffic": tr, **extra,
             "algorithmic_per_launch": d["bytes"] / max(1, d["launches"]) if bound == "hbm"
             else d["flops"] / max(1, d["launches"]),
             "mean_launch_us": round(per_launch_ms * 1e3, 2), "launches_per_denoise": d["launches"],
-            "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+            "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
             "time_shares": shares}, acc
 
 
@@ -425,6 +429,8 @@ def run_ours(args):
             fl = sum(v["flops"] for v in acc2.values())
             r2["denoise_tflops_achieved"] = round(fl / (ms2 * 1e-3) / 1e12, 1)
             r2["denoise_frac_of_burst_peak"] = round(fl / (ms2 * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)
+            r2["denoise_frac_of_sustained_peak"] = round(
+                fl / (ms2 * 1e-3) / 1e12 / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4)
         secondary = {"workload": wl2.name, "metric": "chunks/s @batch 64", "unit": "chunks/s",
                      "value": round(wl2.batch * k2 * ws / (t2 * 1e-3), 1),
                      "ms_per_denoise": round(ms2, 3), "steps": k2, "roofline": r2}

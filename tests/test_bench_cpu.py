@@ -65,3 +65,28 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "tiny"
+
+
+def test_roofline_denominators_and_dominant_kernel():
+    """The dominant kernel is the one with the largest event-timed share; an HBM-bound
+    line divides algorithmic bytes by the measured copy bandwidth, a tensor-bound one
+    (kernels timed inside a whole denoise) FLOPs by the sustained bf16 figure, with the
+    burst fraction beside it."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Stub:
+        def profile_kernels(self, noise, state, steps):
+            return None, {"gemm_gateup": {"ms": 3.0, "launches": 180, "bytes": 180 * 17e6, "flops": 180 * 2e9},
+                          "attention": {"ms": 1.0, "launches": 180, "bytes": 180 * 1e6, "flops": 180 * 1e9}}
+
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    r, acc = bench.roofline(Stub(), None, None, 10, peaks, "measured", "no_such_workload", "hbm", reps=2)
+    assert r["kernel"] == "gemm_gateup" and r["unit"] == "GB/s" and r["peak"] == 6000.0
+    per_launch_s = 3.0e-3 / 180
+    assert abs(r["achieved"] - round(17e6 / per_launch_s / 1e9, 1)) < 1e-6
+    assert abs(r["frac"] - round(r["achieved"] / 6000.0, 4)) < 1e-4
+    assert r["traffic"] is None and abs(sum(r["time_shares"].values()) - 1.0) < 1e-3
+    r, _ = bench.roofline(Stub(), None, None, 10, peaks, "measured", "no_such_workload", "tensor", reps=1)
+    assert r["peak"] == 1400.0 and r["burst_peak"] == 1600.0
+    assert abs(r["frac"] - r["achieved"] / 1400.0) < 1e-3 and abs(r["frac_of_burst_peak"] - r["achieved"] / 1600.0) < 1e-3
