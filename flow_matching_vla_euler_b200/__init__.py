@@ -77,6 +77,8 @@ _SIGNATURES = {
     "vla_profile_kernels": (_I, [_P, _P, _P, _I, _P, _I, ctypes.POINTER(vla_kernel_times), _P]),
     "vla_gemm_bf16": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "vla_gemm_bf16_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "vla_selftest_wait_timeout": (_I, [_P, _I, _P]),
+    "vla_gemm_status": (_I, [_P]),
     "vla_last_error": (ctypes.c_char_p, []),
     "vla_version": (ctypes.c_char_p, []),
 }
@@ -147,6 +149,14 @@ def vla_cache_export(h, K_ptr, V_ptr, batch, stream):
 
 def vla_device_status(h, stream):
     _check(load_library().vla_device_status(h, stream))
+
+
+def vla_selftest_wait_timeout(h, limit_us, stream):
+    _check(load_library().vla_selftest_wait_timeout(h, limit_us, stream))
+
+
+def vla_gemm_status(stream):
+    _check(load_library().vla_gemm_status(stream))
 
 
 def vla_profile_kernels(h, noise_ptr, state_ptr, steps, out_ptr, batch, stream) -> vla_kernel_times:

@@ -1119,6 +1119,15 @@ int vla_device_status(vla_expert* h, void* cuda_stream) {
   return VLA_OK;
 }
 
+int vla_selftest_wait_timeout(vla_expert* h, int limit_us, void* cuda_stream) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (limit_us < 1 || limit_us > 1000000) return fail(VLA_ERR_ARG, "limit_us %d outside [1, 1000000]", limit_us);
+  CU(launch_wait_selftest(h->err, static_cast<unsigned long long>(limit_us) * 1000ull,
+                          static_cast<cudaStream_t>(cuda_stream)));
+  return VLA_OK;
+}
+
 int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, int steps, float* out_actions,
                         int batch, vla_kernel_times* times, void* cuda_stream) {
   g_err.clear();
@@ -1182,9 +1191,95 @@ int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, i
   return rc;
 }
 
-int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim, int m_tok,
-                  int split_k, void* cuda_stream) {
-  g_err.clear();
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Standalone projection entry points (vla_gemm_bf16, vla_gemm_bf16_noalloc) and their
+// device status words. Neither call keeps a caller pointer or a handle, so a bounded
+// wait that gives up inside their kernel is recorded in a library-owned device word,
+// which vla_gemm_status reads (and clears) after synchronising the caller's stream.
+namespace {
+
+constexpr size_t kNoAllocPartialBytes = size_t(8) << 20;
+constexpr int kNoAllocCounters = 4096;   // 4095 tile counters + 1 status word
+constexpr int kMaxDevices = 64;
+
+// Scratch of the allocation-free variant: split-K partial tiles (8 MiB) followed by 4096
+// ints (tile arrival counters, then its status word).
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartialBytes / 4 + kNoAllocCounters];
+// Status word of the allocating variant (its own scratch is freed right after the launch).
+static __device__ int g_gemm_status;
+
+struct SymbolAddrs {
+  unsigned long long ctx_id = 0;   // CUDA context the addresses belong to (0: none yet)
+  float* scratch = nullptr;
+  int* gemm_status = nullptr;
+};
+
+std::mutex g_sym_mu;
+SymbolAddrs g_sym[kMaxDevices];
+
+// Unique id of the calling thread's current CUDA context (never reused in a process, so a
+// context created after cudaDeviceReset gets a new one).
+int current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  if (!get_cur || !get_id) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return fail(VLA_ERR_CUDA, "cuCtxGetCurrent is not available from the driver");
+    get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return fail(VLA_ERR_CUDA, "cuCtxGetId is not available from the driver");
+    get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  }
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) {
+    // no context yet in this thread: a runtime call that needs the module (it allocates
+    // nothing) initialises the device's primary context and makes it current
+    void* p = nullptr;
+    cudaGetSymbolAddress(&p, g_gemm_status);
+    if (get_cur(&ctx) != CUDA_SUCCESS || !ctx) return fail(VLA_ERR_CUDA, "no current CUDA context");
+  }
+  if (get_id(ctx, id) != CUDA_SUCCESS) return fail(VLA_ERR_CUDA, "cuCtxGetId failed");
+  return VLA_OK;
+}
+
+// Device addresses of the file-scope arrays on device `dev` (which is current, with the
+// runtime's context made current by an earlier runtime call). In host code an array's
+// name is only a host-side handle, so the addresses are looked up with
+// cudaGetSymbolAddress once per device and context and cached; a new context on the
+// device (after cudaDeviceReset) triggers a new look-up.
+int symbol_addrs(int dev, SymbolAddrs* out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(VLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  unsigned long long id = 0;
+  int rc = current_context_id(&id);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_sym_mu);
+  SymbolAddrs& a = g_sym[dev];
+  if (a.ctx_id != id) {
+    void* p = nullptr;
+    void* q = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(VLA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
+    e = cudaGetSymbolAddress(&q, g_gemm_status);
+    if (e != cudaSuccess || !q)
+      return fail(VLA_ERR_CUDA, "cudaGetSymbolAddress(status) on device %d: %s", dev, cudaGetErrorString(e));
+    a.scratch = static_cast<float*>(p);
+    a.gemm_status = static_cast<int*>(q);
+    a.ctx_id = id;
+  }
+  *out = a;
+  return VLA_OK;
+}
+
+// Checks shared by both standalone entry points; fills the device, SM count and plan.
+int gemm_prologue(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim, int m_tok, int split_k,
+                  int* dev, GemmPlan* g) {
   if (!W || !X || !Y) return fail(VLA_ERR_ARG, "null W, X or Y");
   if (n_feat < 128 || n_feat % 128 || k_dim < 64 || k_dim % 64 || m_tok < 1)
     return fail(VLA_ERR_SHAPE, "need n_feat %% 128 == 0, k_dim %% 64 == 0, m_tok >= 1 (got %d, %d, %d)", n_feat,
@@ -1192,29 +1287,21 @@ int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, in
   if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(X)) & 15)
     return fail(VLA_ERR_ARG, "W and X must be 16-byte aligned");
   if (split_k < 0) return fail(VLA_ERR_ARG, "split_k must be >= 0");
-  int dev = 0, major = 0, sms = 148;
-  CU(cudaGetDevice(&dev));
-  CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+  int major = 0, sms = 148;
+  CU(cudaGetDevice(dev));
+  CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev));
   if (major != 10) return fail(VLA_ERR_UNSUPPORTED, "device is sm_%d0; this library is built for sm_100a", major);
-  CU(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  CU(configure_gemm_kernels());
-  GemmPlan g = plan_gemm(n_feat, k_dim, m_tok, sms);
+  CU(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev));
+  *g = plan_gemm(n_feat, k_dim, m_tok, sms);
   if (split_k > 0) {
     const int nkb = k_dim / 64;
-    g.kb_per_split = cdiv(nkb, std::min(split_k, nkb));
-    g.splits = cdiv(nkb, g.kb_per_split);
+    g->kb_per_split = cdiv(nkb, std::min(split_k, nkb));
+    g->splits = cdiv(nkb, g->kb_per_split);
   }
-  CUtensorMap tw, tx;
-  int rc;
-  if ((rc = make_tmap(&tw, W, k_dim, n_feat, 128))) return rc;
-  if ((rc = make_tmap(&tx, X, k_dim, m_tok, g.tn))) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  const size_t n_ctr = static_cast<size_t>(g.n_tiles) * g.m_tiles + 1;
-  const size_t ws_bytes = g.splits > 1 ? static_cast<size_t>(g.n_tiles) * g.m_tiles * g.splits * g.tn * 128 * 4 : 0;
-  void* scratch = nullptr;
-  CU(cudaMallocAsync(&scratch, ws_bytes + n_ctr * sizeof(int), s));
-  int* ctr = reinterpret_cast<int*>(static_cast<char*>(scratch) + ws_bytes);
-  cudaError_t e = cudaMemsetAsync(ctr, 0, n_ctr * sizeof(int), s);
+  return VLA_OK;
+}
+
+GemmParams store_params(float* Y, int n_feat, int k_dim, int m_tok, const GemmPlan& g) {
   GemmParams p{};
   p.n_feat = n_feat;
   p.k_dim = k_dim;
@@ -1224,9 +1311,37 @@ int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, in
   p.w_stream = g.m_tiles == 1 ? 1 : 0;
   p.resid = Y;
   p.ld_resid = n_feat;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim, int m_tok,
+                  int split_k, void* cuda_stream) {
+  g_err.clear();
+  int dev = 0;
+  GemmPlan g;
+  int rc = gemm_prologue(W, X, Y, n_feat, k_dim, m_tok, split_k, &dev, &g);
+  if (rc) return rc;
+  SymbolAddrs sa;
+  if ((rc = symbol_addrs(dev, &sa))) return rc;
+  CU(configure_gemm_kernels());
+  CUtensorMap tw, tx;
+  if ((rc = make_tmap(&tw, W, k_dim, n_feat, 128))) return rc;
+  if ((rc = make_tmap(&tx, X, k_dim, m_tok, g.tn))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t n_ctr = static_cast<size_t>(g.n_tiles) * g.m_tiles;
+  const size_t ws_bytes = g.splits > 1 ? static_cast<size_t>(g.n_tiles) * g.m_tiles * g.splits * g.tn * 128 * 4 : 0;
+  void* scratch = nullptr;
+  CU(cudaMallocAsync(&scratch, ws_bytes + n_ctr * sizeof(int), s));
+  int* ctr = reinterpret_cast<int*>(static_cast<char*>(scratch) + ws_bytes);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, n_ctr * sizeof(int), s);
+  GemmParams p = store_params(Y, n_feat, k_dim, m_tok, g);
   p.ws = static_cast<float*>(scratch);
   p.counters = ctr;
-  p.err = ctr + n_ctr - 1;
+  p.err = sa.gemm_status;   // library-owned: outlives the scratch (read by vla_gemm_status)
   if (e == cudaSuccess) e = launch_gemm(g.tn, EPI_STORE, tw, tx, p, g.n_tiles, g.m_tiles, s, false);
   cudaError_t e2 = cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) return fail(VLA_ERR_CUDA, "vla_gemm_bf16 launch: %s", cudaGetErrorString(e));
@@ -1234,63 +1349,15 @@ int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, in
   return VLA_OK;
 }
 
-}  // extern "C"
-
-// ---------------------------------------------------------------------------------
 // Allocation-free variant of vla_gemm_bf16 for callers that may not allocate device
-// memory while they run. Its scratch is this one static array: split-K partial tiles
-// (8 MiB) followed by 4096 ints (tile arrival counters, then the status word).
-namespace {
-
-constexpr size_t kNoAllocPartialBytes = size_t(8) << 20;
-constexpr int kNoAllocCounters = 4096;   // 4095 tile counters + 1 status word
-constexpr int kMaxDevices = 64;
-
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocPartialBytes / 4 + kNoAllocCounters];
-
-std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on device `dev` (which is current). In host code
-// the array's name is only a host-side handle, so the address is looked up once per
-// device and cached.
-int noalloc_scratch(int dev, float** out) {
-  if (dev < 0 || dev >= kMaxDevices) return fail(VLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(VLA_ERR_CUDA, "cudaGetSymbolAddress(scratch) on device %d: %s", dev, cudaGetErrorString(e));
-    g_noalloc_addr[dev] = p;
-  }
-  *out = static_cast<float*>(g_noalloc_addr[dev]);
-  return VLA_OK;
-}
-
-}  // namespace
-
-extern "C" int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim,
-                                     int m_tok, int split_k, void* cuda_stream) {
+// memory while they run; its scratch is the static array above.
+int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim, int m_tok,
+                          int split_k, void* cuda_stream) {
   g_err.clear();
-  if (!W || !X || !Y) return fail(VLA_ERR_ARG, "null W, X or Y");
-  if (n_feat < 128 || n_feat % 128 || k_dim < 64 || k_dim % 64 || m_tok < 1)
-    return fail(VLA_ERR_SHAPE, "need n_feat %% 128 == 0, k_dim %% 64 == 0, m_tok >= 1 (got %d, %d, %d)", n_feat,
-                k_dim, m_tok);
-  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(X)) & 15)
-    return fail(VLA_ERR_ARG, "W and X must be 16-byte aligned");
-  if (split_k < 0) return fail(VLA_ERR_ARG, "split_k must be >= 0");
-  int dev = 0, major = 0, sms = 148;
-  CU(cudaGetDevice(&dev));
-  CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
-  if (major != 10) return fail(VLA_ERR_UNSUPPORTED, "device is sm_%d0; this library is built for sm_100a", major);
-  CU(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  GemmPlan g = plan_gemm(n_feat, k_dim, m_tok, sms);
-  if (split_k > 0) {
-    const int nkb = k_dim / 64;
-    g.kb_per_split = cdiv(nkb, std::min(split_k, nkb));
-    g.splits = cdiv(nkb, g.kb_per_split);
-  }
+  int dev = 0;
+  GemmPlan g;
+  int rc = gemm_prologue(W, X, Y, n_feat, k_dim, m_tok, split_k, &dev, &g);
+  if (rc) return rc;
   const size_t tiles = static_cast<size_t>(g.n_tiles) * g.m_tiles;
   const size_t need = g.splits > 1 ? tiles * g.splits * g.tn * 128 * sizeof(float) : 0;
   if (need > kNoAllocPartialBytes || tiles > static_cast<size_t>(kNoAllocCounters - 1))
@@ -1298,30 +1365,46 @@ extern "C" int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float
                 "vla_gemm_bf16_noalloc: this shape needs %zu bytes of split-K scratch and %zu tile counters; "
                 "the static scratch holds %zu bytes and %d counters (use vla_gemm_bf16, or a smaller split_k)",
                 need, tiles, kNoAllocPartialBytes, kNoAllocCounters - 1);
-  float* scratch = nullptr;
-  int rc = noalloc_scratch(dev, &scratch);
-  if (rc) return rc;
+  SymbolAddrs sa;
+  if ((rc = symbol_addrs(dev, &sa))) return rc;
   CU(configure_gemm_kernels());
   CUtensorMap tw, tx;
   if ((rc = make_tmap(&tw, W, k_dim, n_feat, 128))) return rc;
   if ((rc = make_tmap(&tx, X, k_dim, m_tok, g.tn))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  int* ctr = reinterpret_cast<int*>(scratch + kNoAllocPartialBytes / 4);
-  // counters and the status word must start at zero; the partial tiles are overwritten
-  CU(cudaMemsetAsync(ctr, 0, kNoAllocCounters * sizeof(int), s));
-  GemmParams p{};
-  p.n_feat = n_feat;
-  p.k_dim = k_dim;
-  p.m_tok = m_tok;
-  p.splits = g.splits;
-  p.kb_per_split = g.kb_per_split;
-  p.w_stream = g.m_tiles == 1 ? 1 : 0;
-  p.resid = Y;
-  p.ld_resid = n_feat;
-  p.ws = scratch;
+  int* ctr = reinterpret_cast<int*>(sa.scratch + kNoAllocPartialBytes / 4);
+  // the tile counters must start at zero (a call that timed out may have left some set);
+  // the status word after them is left alone until vla_gemm_status reads it, and the
+  // partial tiles are overwritten before they are read
+  CU(cudaMemsetAsync(ctr, 0, (kNoAllocCounters - 1) * sizeof(int), s));
+  GemmParams p = store_params(Y, n_feat, k_dim, m_tok, g);
+  p.ws = sa.scratch;
   p.counters = ctr;
   p.err = ctr + kNoAllocCounters - 1;
   CU(launch_gemm(g.tn, EPI_STORE, tw, tx, p, g.n_tiles, g.m_tiles, s, false));
   return VLA_OK;
 }
 
+int vla_gemm_status(void* cuda_stream) {
+  g_err.clear();
+  int dev = 0;
+  CU(cudaGetDevice(&dev));
+  SymbolAddrs sa;
+  int rc = symbol_addrs(dev, &sa);
+  if (rc) return rc;
+  CU(cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)));
+  int* words[2] = {sa.gemm_status, reinterpret_cast<int*>(sa.scratch + kNoAllocPartialBytes / 4) + kNoAllocCounters - 1};
+  int v[2] = {0, 0};
+  for (int i = 0; i < 2; ++i) CU(cudaMemcpy(&v[i], words[i], sizeof(int), cudaMemcpyDeviceToHost));
+  if (v[0] || v[1]) {
+    const int zero = 0;
+    for (int i = 0; i < 2; ++i)
+      if (v[i]) CU(cudaMemcpy(words[i], &zero, sizeof(int), cudaMemcpyHostToDevice));
+    return fail(VLA_ERR_TIMEOUT, "a bounded wait gave up inside %s%s%s (device status %d); the word was cleared",
+                v[0] ? "vla_gemm_bf16" : "", v[0] && v[1] ? " and " : "", v[1] ? "vla_gemm_bf16_noalloc" : "",
+                v[0] ? v[0] : v[1]);
+  }
+  return VLA_OK;
+}
+
+}  // extern "C"

@@ -201,4 +201,8 @@ cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, 
 cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch,
                                int kcap, int rows, int D, int n_static_max, int ring_off, cudaStream_t s);
 
+// Arms an mbarrier nothing arrives on and waits on it for limit_ns, so the wait gives up
+// and records a timeout in *err (failure-path self-test).
+cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t s);
+
 }  // namespace vla

@@ -71,18 +71,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; gives up after kWaitLimitNs,
-// sets the status word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+// Waits for the phase with the given parity to complete; gives up after limit_ns, sets
+// the status word and returns false.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, int* err,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       report(err, kDevTimeout);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  return mbar_wait_limit(bar, parity, err, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA

@@ -413,6 +413,26 @@ cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int 
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ self-test
+// Exercises the failure-reporting path of the bounded waits: one thread arms an mbarrier
+// that nothing ever arrives on and waits on it with a short limit, so the wait gives up,
+// records a timeout in the status word and the kernel returns. No copy is in flight and
+// no tensor memory is held when it gives up.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    mbar_wait_limit(b, 0, err, limit_ns);
+  }
+}
+
+cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
 // The per-step kernels of the denoise chain prefer the largest shared-memory carve-out
 // too, so that an SM they configured still takes a CTA of the projection that follows.
 cudaError_t configure_small_kernels() {

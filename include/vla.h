@@ -172,6 +172,11 @@ VLA_API int vla_cache_append_sliding(vla_expert* h, const uint16_t* K_tok, const
  * vla_denoise -- the hot path: `steps` explicit Euler steps x <- x + dt * v(x, t),
  * t_k = 1 - k/steps, dt = -1/steps, from x = noise to out_actions, every step running
  * the action expert over the suffix tokens against the cached prefix.
+ * Passages: FlowEdge README, "Installation" (flow sampling with "euler 10");
+ * realtime-vla write-up, "The latency table, and what it assumes" (10 flow steps, chunk
+ * 50) and "Copying an inference file into your own project" (forward(images, state (32,),
+ * noise (traj_len, 32)): noise and state in, the action chunk out); Reflex abstract
+ * (the cached perception K/V is reused by every step; AdaRMSNorm gated on flow phase).
  * noise: DEVICE fp32 [batch][C][A] (not modified); state: DEVICE fp32
  * [batch][state_dim], required iff state_dim > 0, else ignored; out_actions: DEVICE
  * fp32 [batch][C][A], must not overlap noise. The first call for a (batch, steps) pair
@@ -205,6 +210,17 @@ VLA_API int vla_cache_export(vla_expert* h, uint16_t* K_out, uint16_t* V_out, in
  * VLA_ERR_TIMEOUT (status word set; it is then cleared) or VLA_ERR_CUDA.
  */
 VLA_API int vla_device_status(vla_expert* h, void* cuda_stream);
+
+/*
+ * vla_selftest_wait_timeout -- exercises the failure-reporting path of the bounded waits
+ * (no counterpart on the pages): enqueues on cuda_stream one tiny kernel that arms a
+ * shared-memory barrier nothing ever arrives on and waits on it for limit_us
+ * microseconds (1..1000000), so the wait gives up, records VLA_ERR_TIMEOUT in the
+ * handle's device status word and the kernel returns. It starts no copy and holds no
+ * tensor memory, so the context and the handle stay usable; the next vla_device_status
+ * reports the timeout once and clears it. Errors: VLA_ERR_ARG, VLA_ERR_CUDA.
+ */
+VLA_API int vla_selftest_wait_timeout(vla_expert* h, int limit_us, void* cuda_stream);
 
 /* Kinds of kernels, for vla_profile_kernels. */
 typedef enum vla_kernel_kind {
@@ -241,7 +257,9 @@ VLA_API int vla_profile_kernels(vla_expert* h, const float* noise, const float* 
  * X 16-byte aligned. split_k = 0 picks the split-K factor the denoise loop would use;
  * split_k > 0 forces (at most) that many K splits. The split-K partial tiles live in a
  * workspace this call allocates and frees stream-ordered (cudaMallocAsync / cudaFreeAsync).
- * Stream-ordered. Errors: VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_UNSUPPORTED, VLA_ERR_CUDA.
+ * A bounded wait that gives up inside the kernel is recorded in a library-owned device
+ * word: call vla_gemm_status after the work to learn of it. Stream-ordered.
+ * Errors: VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_UNSUPPORTED, VLA_ERR_CUDA.
  */
 VLA_API int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_feat, int k_dim,
                           int m_tok, int split_k, void* cuda_stream);
@@ -259,19 +277,30 @@ VLA_API int vla_gemm_bf16(const uint16_t* W, const uint16_t* X, float* Y, int n_
  * loads this library holds until the process exits. A call whose plan needs more than
  * 8 MiB of partial tiles, or more than 4095 output tiles, is rejected with VLA_ERR_SHAPE
  * (the message gives the size it needed); nothing is launched then.
- * Set-up: the first call on each device looks up the device address of that array (with
- * that device current); with lazy module loading that is also when the driver backs the
- * array with device memory, so the device's free memory drops once, at that first call.
- * Make that first call before any stream capture.
- * Sharing: every call on a device uses the same array. Each call clears the counters and
- * the status word (stream-ordered) before its kernel, so the contents left by the last
- * call do not matter; but calls that can overlap on the GPU (other streams, other host
- * threads) race on the array and must be serialized by the caller.
+ * Set-up: the first call on each device (and again the first call after the device's
+ * context was replaced, e.g. by cudaDeviceReset) looks up the device address of that
+ * array with that device current; with lazy module loading that is also when the driver
+ * backs the array with device memory, so the device's free memory drops once, at that
+ * first call. Make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array. Each call clears the counters
+ * (stream-ordered) before its kernel, so the counts left by the last call do not matter;
+ * calls that can overlap on the GPU (other streams, other host threads) race on the array
+ * and must be serialized by the caller.
+ * Status: a bounded wait that gives up inside the kernel sets the status word at the end
+ * of the array; it stays set (later calls do not clear it) until vla_gemm_status reads it.
  * The call allocates nothing: no cudaMalloc, cudaMallocAsync, cudaFree or allocating
  * library routine. Stream-ordered. Errors: as vla_gemm_bf16, plus VLA_ERR_SHAPE above.
  */
 VLA_API int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y, int n_feat,
                                   int k_dim, int m_tok, int split_k, void* cuda_stream);
+
+/*
+ * vla_gemm_status -- synchronize cuda_stream, then read and clear the device status words
+ * of vla_gemm_bf16 and vla_gemm_bf16_noalloc on the current device. Returns VLA_OK, or
+ * VLA_ERR_TIMEOUT if a bounded wait gave up inside one of their kernels since the last
+ * query (that call's Y is then not valid), or VLA_ERR_CUDA. Allocates nothing.
+ */
+VLA_API int vla_gemm_status(void* cuda_stream);
 
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VLA_API const char* vla_last_error(void);

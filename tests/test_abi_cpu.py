@@ -104,6 +104,7 @@ def test_host_argument_checks(lib):
     assert lib.vla_cache_set_prefix(None, None, None, 1, 1, None) == V.VLA_ERR_ARG
     assert lib.vla_cache_append_sliding(None, None, None, 1, None) == V.VLA_ERR_ARG
     assert lib.vla_device_status(None, None) == V.VLA_ERR_ARG
+    assert lib.vla_selftest_wait_timeout(None, 100, None) == V.VLA_ERR_ARG
     assert lib.vla_gemm_bf16(None, None, None, 128, 64, 1, 0, None) == V.VLA_ERR_ARG
     one = ctypes.c_void_p(256)
     assert lib.vla_gemm_bf16(one, one, one, 100, 64, 1, 0, None) == V.VLA_ERR_SHAPE

@@ -64,7 +64,10 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["higher_is_better"] is False and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"] == "tiny"
+    assert d["config"]["workload"] == "tiny" and d["config"]["layers"] == 2
+    # each timed step is one whole denoise, and the line counts the steps it timed
+    assert 1 <= d["steps"] <= 2 and "whole" in d["cpu_baseline"]["sample"]
+    assert d["cpu_baseline"]["single_thread_ms"] > 0
 
 
 def test_roofline_denominators_and_dominant_kernel():
@@ -87,6 +90,28 @@ def test_roofline_denominators_and_dominant_kernel():
     assert abs(r["achieved"] - round(17e6 / per_launch_s / 1e9, 1)) < 1e-6
     assert abs(r["frac"] - round(r["achieved"] / 6000.0, 4)) < 1e-4
     assert r["traffic"] is None and abs(sum(r["time_shares"].values()) - 1.0) < 1e-3
-    r, _ = bench.roofline(Stub(), None, None, 10, peaks, "measured", "no_such_workload", "tensor", reps=1)
-    assert r["peak"] == 1400.0 and r["burst_peak"] == 1600.0
-    assert abs(r["frac"] - r["achieved"] / 1400.0) < 1e-3 and abs(r["frac_of_burst_peak"] - r["achieved"] / 1600.0) < 1e-3
+    # at full clocks (or unknown clocks) the burst figure is the denominator ...
+    for mhz in (None, 1965.0):
+        r, _ = bench.roofline(Stub(), None, None, 10, peaks, "measured", "no_such_workload", "tensor", reps=1,
+                              sm_mhz=mhz)
+        assert r["peak"] == 1600.0 and r["burst_peak"] == 1600.0 and r["sustained_peak"] == 1400.0
+        assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-3
+        assert abs(r["frac_of_sustained_peak"] - r["achieved"] / 1400.0) < 1e-3
+    # ... and the sustained one only for a run held near the clock it was measured at
+    r, _ = bench.roofline(Stub(), None, None, 10, peaks, "measured", "no_such_workload", "tensor", reps=1,
+                          sm_mhz=1275.0)
+    assert r["peak"] == 1400.0 and "sustained" in r["peak_source"]
+
+
+def test_denoise_bytes_follow_the_scope_table():
+    """Weights once per Euler step + bf16 action maps + cached K/V once per layer per step:
+    6.375 GB for the 3-view Pi05 denoise, 6.319 GB for 1-view Pi0, 15.5 GB at batch 64."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from vla_inputs import get
+    per_step = 2 * 18 * (1024 * 2560 + 1024 * 2048 + 2 * 4096 * 1024 + 1024 * 4096) + 2 * 2 * 1024 * 32
+    kv = 2 * 2 * 18 * 788 * 256
+    assert bench.denoise_bytes(get("pi05_3view")) == 10 * (per_step + kv)
+    assert abs(bench.denoise_bytes(get("pi05_3view")) / 1e9 - 6.375) < 1e-3
+    assert abs(bench.denoise_bytes(get("pi0_1view")) / 1e9 - 6.3196) < 1e-3
+    assert abs(bench.denoise_bytes(get("pi05_3view_b64")) / 1e9 - 15.525) < 1e-3

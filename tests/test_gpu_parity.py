@@ -29,16 +29,56 @@ def test_full_size_batch1_matches_oracle(name):
     ex.device_status()
 
 
-def test_batch64_sampled_observations_match_oracle():
-    """64 independent observations in one call; the oracle checks a sample of them."""
+def _batch64_run():
     wl = get("pi05_3view_b64")
     ex, inp = make_expert(wl)
     load_prefix(ex, inp)
     got = run(ex, inp, wl.steps)
-    idx = [0, 37, 63]
-    check_actions(got[idx], oracle_actions(wl, inp, batch_idx=idx), "b64 sample")
-    assert np.all(np.isfinite(got))
     ex.device_status()
+    return wl, ex, inp, got
+
+
+def test_batch64_every_observation_matches_batch1_runs():
+    """64 independent observations in one call (persistent GEMMs, tensor-core attention,
+    norm kernels) against 64 separate batch-1 calls of the same observations on the same
+    handle (the one-token-tile path: folded norms, split-K cluster GEMMs, split-KV
+    attention), every row at the acceptance tolerance; the oracle checks a sample."""
+    wl, ex, inp, got = _batch64_run()
+    assert got.shape[0] == 64 and np.all(np.isfinite(got))
+    idx = [0, 37, 63]
+    check_actions(got[idx], oracle_actions(wl, inp, batch_idx=idx), "b64 oracle sample")
+    for b in range(wl.batch):
+        one = dict(inp, noise=inp["noise"][b:b + 1], prefix_k=inp["prefix_k"][:, b:b + 1],
+                   prefix_v=inp["prefix_v"][:, b:b + 1])
+        load_prefix(ex, one)
+        check_actions(got[b:b + 1], run(ex, one, wl.steps), f"b64 row {b} vs batch-1 run")
+    ex.device_status()
+    ex.close()
+
+
+@pytest.mark.slow
+def test_batch64_every_observation_matches_oracle():
+    """Every one of the 64 rows against the fp64 oracle (one observation per host thread,
+    BLAS single-threaded in each)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
+    wl, ex, inp, got = _batch64_run()
+    ex.close()
+    with threadpool_limits(1), ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as pool:
+        # decode the parameters once, then one observation per task
+        import oracle as O
+        P = O.decode_params(inp["params"])
+        pk, pv = O.bf16_to_f64(inp["prefix_k"]), O.bf16_to_f64(inp["prefix_v"])
+        noise = inp["noise"].astype(np.float64)
+
+        def one(b):
+            return O.denoise(wl.expert, P, noise[b:b + 1], None, pk[:, b:b + 1], pv[:, b:b + 1], wl.steps)[0]
+
+        ref = np.stack(list(pool.map(one, range(wl.batch))))
+    for b in range(wl.batch):
+        check_actions(got[b:b + 1], ref[b:b + 1], f"b64 row {b} vs oracle")
+    check_actions(got, ref, "b64 all rows vs oracle")
 
 
 def test_zero_velocity_is_bit_exact():
@@ -154,6 +194,30 @@ def test_prefix_lengths_below_capacity_and_empty():
         load_prefix(ex, dict(inp, prefix_k=too_many, prefix_v=too_many))
     assert e.value.code == V.VLA_ERR_SHAPE
     ex.device_status()
+    ex.close()
+
+
+def test_bounded_wait_gives_up_and_the_handle_stays_usable():
+    """A wait that nothing satisfies (a shared-memory barrier no thread arrives on) gives
+    up after its limit, the kernel returns, vla_device_status reports VLA_ERR_TIMEOUT once
+    and clears it, and the same handle then denoises correctly again."""
+    import flow_matching_vla_euler_b200 as V
+    wl = get("tiny")
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    ref = golden_actions("tiny")
+    check_actions(run(ex, inp, wl.steps), ref, "before the timeout")
+    ex.device_status()
+    V.vla_selftest_wait_timeout(ex.handle, 100, V._stream())
+    with pytest.raises(V.VlaError) as e:
+        ex.device_status()
+    assert e.value.code == V.VLA_ERR_TIMEOUT
+    ex.device_status()                       # cleared: reported once
+    check_actions(run(ex, inp, wl.steps), ref, "after the timeout")
+    ex.device_status()
+    with pytest.raises(V.VlaError) as e:
+        V.vla_selftest_wait_timeout(ex.handle, 0, V._stream())
+    assert e.value.code == V.VLA_ERR_ARG
     ex.close()
 
 

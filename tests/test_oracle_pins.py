@@ -16,6 +16,49 @@ import oracle as O
 EPS = 1e-6
 
 
+# ------------------------------------------------------------------ bf16 widening
+
+@pytest.mark.parametrize("bits, value", [
+    (0x3F80, 1.0),                                # sign 0, exponent 127, mantissa 0
+    (0xC040, -3.0),                               # -1.5 * 2
+    (0x0000, 0.0),
+    (0x4049, 3.140625),                           # 1.5703125 * 2
+    (0x3E80, 0.25),
+    (0x0001, 2.0 ** -133),                        # smallest subnormal: 2^-126 * 2^-7
+    (0x007F, 127 * 2.0 ** -133),                  # largest subnormal
+    (0x0080, 2.0 ** -126),                        # smallest normal
+    (0x7F7F, (2 - 2.0 ** -7) * 2.0 ** 127),       # largest finite
+    (0xFF7F, -(2 - 2.0 ** -7) * 2.0 ** 127),
+])
+def test_bf16_widening_hand_values(bits, value):
+    """bf16 = sign | 8-bit exponent (bias 127) | 7-bit mantissa; each value here follows
+    from that definition by hand, independently of any float32 reinterpretation."""
+    got = O.bf16_to_f64(np.array([bits], dtype=np.uint16))[0]
+    assert got == value and got.dtype == np.float64
+
+
+def test_bf16_widening_signed_zero_and_specials():
+    got = O.bf16_to_f64(np.array([0x8000, 0x7F80, 0xFF80, 0x7FC0], dtype=np.uint16))
+    assert got[0] == 0.0 and math.copysign(1.0, got[0]) == -1.0
+    assert got[1] == math.inf and got[2] == -math.inf and math.isnan(got[3])
+
+
+def test_bf16_widening_matches_the_definition_exhaustively():
+    """All 2^16 patterns against sign * 2^(e-127) * (1 + m/128) (normal) or
+    sign * 2^-126 * m/128 (subnormal), evaluated in exact integer/fraction arithmetic."""
+    from fractions import Fraction
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):           # NaN patterns widen to NaN
+        got = O.bf16_to_f64(allbits)
+    for b in range(1 << 16):
+        sign = -1 if b >> 15 else 1
+        e, m = (b >> 7) & 0xFF, b & 0x7F
+        if e == 0xFF:
+            continue
+        v = Fraction(m, 128) * Fraction(2) ** -126 if e == 0 else (1 + Fraction(m, 128)) * Fraction(2) ** (e - 127)
+        assert got[b] == float(sign * v), hex(b)
+
+
 # ------------------------------------------------------------------------- RMSNorm
 
 def test_rmsnorm_closed_form_3_4():

@@ -27,6 +27,12 @@ def _call(fn, W, X, Y, split_k=0):
     return rc
 
 
+def lib_status():
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    return V.load_library().vla_gemm_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
 def test_noalloc_matches_allocating_entry_point_twice():
     import torch
     import flow_matching_vla_euler_b200 as V
@@ -52,6 +58,7 @@ def test_noalloc_matches_allocating_entry_point_twice():
         assert _call("vla_gemm_bf16_noalloc", W, X, Y) == V.VLA_OK, V.vla_last_error()
     torch.cuda.synchronize()
     assert torch.cuda.mem_get_info()[0] == free_before
+    assert lib_status() == V.VLA_OK, V.vla_last_error()   # no bounded wait gave up
     for (W, X, ref), Y in zip(inputs, outs):
         k = W.shape[1]
         torch.testing.assert_close(Y, ref, rtol=1e-4, atol=2e-4 * math.sqrt(k))
