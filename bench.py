@@ -49,6 +49,10 @@ def parse_args(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-profile", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--euler-steps", type=int, default=0,
+                   help="profiling aid: Euler steps per denoise instead of the workload's (0: keep)")
+    p.add_argument("--fp8-workload", default="pi05_3view_fp8")
+    p.add_argument("--no-fp8", action="store_true")
     return p.parse_args(argv)
 
 
@@ -431,7 +435,12 @@ def denoise_bytes(wl) -> float:
         small += 2 * W * W
     if e.has_state:
         small += W * e.state_dim
-    weights = 2.0 * (L * per_layer + small)
+    if getattr(wl, "weight_format", "bf16") == "e4m3":
+        # one byte per projection weight plus an fp32 scale per output row
+        rows = (H * D + 2 * kv) + W + 2 * F + W
+        weights = 1.0 * L * per_layer + 4.0 * L * rows + 2.0 * small
+    else:
+        weights = 2.0 * (L * per_layer + small)
     kv_bytes = 2.0 * 2 * L * wl.batch * wl.n_cached * kv
     return wl.steps * (weights + kv_bytes)
 
@@ -463,6 +472,9 @@ def run_ours(args):
     ws, rank, local = dist_setup(args)
     peaks, peak_src = load_peaks()
     wl = get(args.workload)
+    if args.euler_steps:
+        from dataclasses import replace
+        wl = replace(wl, steps=args.euler_steps)
     inp = make_inputs(wl, seed=wl.seed + rank)
     ex, noise, state = build_expert(wl, inp)
     steps = wl.steps
@@ -524,6 +536,29 @@ def run_ours(args):
         del inp2
         torch.cuda.empty_cache()
 
+    fp8 = None
+    if not args.no_fp8:
+        # the same denoise with FP8 (E4M3, per-output-row scale) projection weights
+        wl3 = get(args.fp8_workload)
+        inp3 = make_inputs(wl3, seed=wl3.seed + rank)
+        ex3, n3, s3 = build_expert(wl3, inp3)
+        k3 = max(10, args.steps // 2)
+        t3, per3, _ = time_device(ex3, n3, s3, wl3.steps, k3, min(args.warmup, 5), ws)
+        ex3.device_status()
+        t3 = max_over_ranks(t3, ws)
+        ms3 = t3 / k3
+        b3 = denoise_bytes(wl3)
+        fp8 = {"workload": wl3.name, "metric": "ms per 10-step chunk-50 denoise (batch 1), FP8 weights",
+               "unit": "ms", "value": round(ms3, 4), "steps": k3,
+               "latency_ms": {"median": round(statistics.median(per3), 4)},
+               "denoise_roofline": {"algorithmic_bytes": b3,
+                                    "roofline_ms": round(b3 / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
+                                    "frac": round(b3 / (peaks["hbm_gbs"] * 1e9) * 1e3 / ms3, 4),
+                                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "peak_source": peak_src}}
+        ex3.close()
+        del ex3
+        torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         ms_cpu = OracleRunner(wl, inp, 1).ms()
@@ -553,6 +588,7 @@ def run_ours(args):
                 "library_count_adds": "activation rows (GEMM operands, Q/O rows, fp32 residual reads and "
                                       "writes), the chunk's own K/V and padded QKV rows"},
             "secondary": secondary,
+            "fp8": fp8,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": None if launches_per_denoise is None else launches_per_denoise * args.steps,

@@ -21,8 +21,10 @@ VLA_ERR_OOM, VLA_ERR_CUDA, VLA_ERR_TIMEOUT, VLA_ERR_UNSUPPORTED = 4, 5, 6, 7
 VLA_TIME_PI0_MLP, VLA_TIME_ADA_SINCOS, VLA_TIME_ADA_MLP = 0, 1, 2
 VLA_FLAG_NO_PDL = 1
 VLA_FLAG_NORM_KERNELS = 2
+VLA_FLAG_NO_PERSIST = 4
+VLA_FLAG_FP8_WEIGHTS = 8
 KERNEL_KINDS = ["gemm_qkv", "attention", "gemm_o", "gemm_gateup", "gemm_down", "norm", "embed",
-                "final_euler", "time_mlp"]
+                "final_euler", "time_mlp", "denoise_persist"]
 
 _CFG_INT_FIELDS = ["n_layers", "width", "n_heads", "n_kv_heads", "head_dim", "mlp_dim", "action_dim",
                    "chunk", "state_dim", "time_kind", "time_dim", "n_static_max", "n_sliding",
@@ -37,6 +39,7 @@ WEIGHT_FIELDS = [
     "norm1_mod_w", "norm1_mod_b", "norm2_mod_w", "norm2_mod_b",
     "final_norm_mod_w", "final_norm_mod_b",
     "wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down",
+    "wq_scale", "wk_scale", "wv_scale", "wo_scale", "w_gate_scale", "w_up_scale", "w_down_scale",
 ]
 
 
@@ -50,8 +53,8 @@ class vla_weights(ctypes.Structure):
 
 
 class vla_kernel_times(ctypes.Structure):
-    _fields_ = [("total_ms", ctypes.c_float * 9), ("launches", ctypes.c_int * 9),
-                ("bytes", ctypes.c_double * 9), ("flops", ctypes.c_double * 9)]
+    _fields_ = [("total_ms", ctypes.c_float * 10), ("launches", ctypes.c_int * 10),
+                ("bytes", ctypes.c_double * 10), ("flops", ctypes.c_double * 10)]
 
 
 class VlaError(RuntimeError):
@@ -226,13 +229,21 @@ class Expert:
         c.eps, c.rope_base, c.flags = float(cfg.eps), float(cfg.rope_base), int(flags)
         w = vla_weights()
         keep = []
+        fp8 = False
         for name, arr in params.items():
             field = name.replace(".", "_")
             if field not in WEIGHT_FIELDS:
                 raise KeyError(f"unknown parameter {name}")
-            a = np.ascontiguousarray(arr, dtype=np.uint16)
+            a = np.asarray(arr)
+            if a.dtype == np.uint8:             # E4M3 bytes (FP8 projection weights)
+                fp8 = True
+            elif a.dtype != np.float32:         # bf16 bit patterns
+                a = a.astype(np.uint16, copy=False)
+            a = np.ascontiguousarray(a)
             keep.append(a)
             setattr(w, field, a.ctypes.data)
+        if fp8:
+            c.flags |= VLA_FLAG_FP8_WEIGHTS
         self.cfg = cfg
         self.n_static_max, self.n_sliding, self.max_batch = n_static_max, n_sliding, max_batch
         self.handle = vla_expert_create(c, w)

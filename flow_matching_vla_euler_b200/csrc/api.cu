@@ -113,6 +113,25 @@ AttnPlan plan_attn(int rows, int batch, int max_key_tiles, int sm_count, int max
   return a;
 }
 
+// Persistent kernel: K splits per 128-feature tile so that tiles x splits fills the G
+// CTAs (at most one item per CTA and phase), each split covering >= 1 K block.
+// At most 20 splits, so that an owner's partials (splits x owned rows x 64 fp32) fit half
+// of the persistent kernel's 96 KB work area.
+PersistGemm persist_plan(int n_feat, int k_dim, int G) {
+  PersistGemm g;
+  g.n_tiles = n_feat / 128;
+  g.nkb = k_dim / 64;
+  int S = g.n_tiles >= G ? 1 : G / g.n_tiles;
+  S = std::min(S, g.nkb);
+  S = std::min(S, 20);
+  g.splits = std::max(S, 1);
+  return g;
+}
+
+// Embed maps in the layout the persistent kernel stages: bf16 [W][in] -> fp32 [W][in4],
+// in4 = in rounded up to a multiple of 4 (zero padded), rows contiguous.
+int upload_f32_rowpad(vla_expert* h, float** dst, const uint16_t* src, size_t rows, size_t cols);
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -147,6 +166,24 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return VLA_OK;
 }
 
+// uint8 [rows][inner] row-major (E4M3 weight bytes), boxes of 64 bytes x box_rows, no
+// swizzle: the persistent kernel widens each row in shared memory itself.
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled (uint8) failed (%d) for %llu x %llu", static_cast<int>(r),
+                static_cast<unsigned long long>(rows), static_cast<unsigned long long>(inner));
+  return VLA_OK;
+}
+
 }  // namespace
 
 struct vla_expert {
@@ -159,8 +196,11 @@ struct vla_expert {
 
   std::vector<void*> allocs;
 
-  // weights
+  // weights (bf16, or with VLA_FLAG_FP8_WEIGHTS the E4M3 bytes and per-row scales)
+  bool fp8 = false;
   bf16 *wqkv = nullptr, *wo = nullptr, *wgu = nullptr, *wdown = nullptr;
+  uint8_t *wqkv8 = nullptr, *wo8 = nullptr, *wgu8 = nullptr, *wdown8 = nullptr;
+  float *sc_qkv = nullptr, *sc_o = nullptr, *sc_gu = nullptr, *sc_down = nullptr;
   bf16 *w1a = nullptr, *w2 = nullptr, *tin_full = nullptr, *tin_b = nullptr;
   bf16 *cond1_w = nullptr, *cond1_b = nullptr, *cond2_w = nullptr, *cond2_b = nullptr;
   bf16 *mod_w = nullptr, *mod_b = nullptr;
@@ -201,6 +241,18 @@ struct vla_expert {
   // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
   unsigned long long* trace = nullptr;
   std::string trace_file;
+
+  // persistent whole-denoise kernel (one token tile): plans and scratch
+  bool persist_ok = false;       // built for this head_dim and one CTA fits per SM
+  int persist_bmax = 0;          // largest batch with batch x suffix <= 64
+  int np = 0;                    // phases per Euler step
+  PersistGemm pg[PH_COUNT] = {};
+  int p_max_tiles = 0;
+  int *p_done = nullptr, *p_tctr = nullptr;
+  float *p_ws = nullptr, *p_ws_att = nullptr, *p_ws_ml = nullptr;
+  float *p_rstat_a = nullptr, *p_rstat_b = nullptr;   // [contributor][64]
+  float *p_ain_rm = nullptr, *p_st_rm = nullptr;      // embed maps [W][in padded to 4]
+  unsigned long long* p_trace = nullptr;   // [np][G][8] stamps of the first step (diagnostics)
 
   struct GraphEntry {
     cudaGraph_t g = nullptr;
@@ -243,6 +295,17 @@ int upload_f32(vla_expert* h, float** dst, const uint16_t* src, size_t n) {
   return VLA_OK;
 }
 
+int upload_f32_rowpad(vla_expert* h, float** dst, const uint16_t* src, size_t rows, size_t cols) {
+  const size_t cp = (cols + 3) & ~static_cast<size_t>(3);
+  std::vector<float> tmp(rows * cp, 0.0f);
+  for (size_t r = 0; r < rows; ++r)
+    for (size_t c = 0; c < cols; ++c) tmp[r * cp + c] = bf16_to_f32(src[r * cols + c]);
+  int rc = dalloc(h, dst, rows * cp);
+  if (rc) return rc;
+  CU(cudaMemcpy(*dst, tmp.data(), rows * cp * 4, cudaMemcpyHostToDevice));
+  return VLA_OK;
+}
+
 // bf16 [rows][cols] -> fp32 [cols][rows] on the device.
 int upload_f32_t(vla_expert* h, float** dst, const uint16_t* src, size_t rows, size_t cols) {
   std::vector<float> tmp(rows * cols);
@@ -279,7 +342,14 @@ int validate(const vla_config* c, const vla_weights* w) {
   if (c->max_steps < 1 || c->max_steps > kMaxSteps)
     return fail(VLA_ERR_SHAPE, "max_steps must be in [1, %d]", kMaxSteps);
   if (!(c->eps > 0.0f)) return fail(VLA_ERR_ARG, "eps must be > 0");
-  if (c->flags & ~(VLA_FLAG_NO_PDL | VLA_FLAG_NORM_KERNELS)) return fail(VLA_ERR_ARG, "unknown flag bits 0x%x", c->flags);
+  if (c->flags & ~(VLA_FLAG_NO_PDL | VLA_FLAG_NORM_KERNELS | VLA_FLAG_NO_PERSIST | VLA_FLAG_FP8_WEIGHTS))
+    return fail(VLA_ERR_ARG, "unknown flag bits 0x%x", c->flags);
+  if ((c->flags & VLA_FLAG_FP8_WEIGHTS) && (c->flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS)))
+    return fail(VLA_ERR_UNSUPPORTED, "FP8 weights run on the persistent one-tile path only");
+  if ((c->flags & VLA_FLAG_FP8_WEIGHTS) &&
+      !(w->wq_scale && w->wk_scale && w->wv_scale && w->wo_scale && w->w_gate_scale && w->w_up_scale &&
+        w->w_down_scale))
+    return fail(VLA_ERR_ARG, "FP8 weights need every *_scale pointer");
   const bool need_common = w->action_in_w && w->action_in_b && w->action_out_w && w->action_out_b &&
                            w->wq && w->wk && w->wv && w->wo && w->w_gate && w->w_up && w->w_down;
   if (!need_common) return fail(VLA_ERR_ARG, "missing a projection weight");
@@ -318,10 +388,21 @@ int compute_tables(vla_expert* h, int slot, int steps, cudaStream_t s) {
     const long cw = h->qkv_rows + 2L * h->F;
     float* ct = h->ctables[slot];
     for (int l = 0; l < h->L; ++l) {
-      CU(launch_rowgemv(tbl + (static_cast<long>(2 * l) * 3 + 1) * h->W, steps, h->W, h->table_stride,
+      const float* sh1 = tbl + (static_cast<long>(2 * l) * 3 + 1) * h->W;
+      const float* sh2 = tbl + (static_cast<long>(2 * l + 1) * 3 + 1) * h->W;
+      if (h->fp8) {
+        CU(launch_rowgemv_fp8(sh1, steps, h->W, h->table_stride, h->wqkv8 + static_cast<size_t>(l) * h->qkv_rows * h->W,
+                              h->W, h->sc_qkv + static_cast<size_t>(l) * h->qkv_rows, h->qkv_rows, ct + l * cw,
+                              h->L * cw, s));
+        CU(launch_rowgemv_fp8(sh2, steps, h->W, h->table_stride, h->wgu8 + static_cast<size_t>(l) * 2 * h->F * h->W,
+                              h->W, h->sc_gu + static_cast<size_t>(l) * 2 * h->F, 2 * h->F, ct + l * cw + h->qkv_rows,
+                              h->L * cw, s));
+        continue;
+      }
+      CU(launch_rowgemv(sh1, steps, h->W, h->table_stride,
                         h->wqkv + static_cast<size_t>(l) * h->qkv_rows * h->W, h->W, nullptr, h->qkv_rows,
                         ct + l * cw, h->L * cw, 0, s));
-      CU(launch_rowgemv(tbl + (static_cast<long>(2 * l + 1) * 3 + 1) * h->W, steps, h->W, h->table_stride,
+      CU(launch_rowgemv(sh2, steps, h->W, h->table_stride,
                         h->wgu + static_cast<size_t>(l) * 2 * h->F * h->W, h->W, nullptr, 2 * h->F,
                         ct + l * cw + h->qkv_rows, h->L * cw, 0, s));
     }
@@ -689,6 +770,68 @@ int make_act_maps(vla_expert* h, int B, ActMaps* am) {
   return VLA_OK;
 }
 
+bool use_persist(const vla_expert* h, int B) {
+  return h->persist_ok && B <= h->persist_bmax &&
+         !(h->cfg.flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS));
+}
+
+void persist_params(const vla_expert* h, int B, int steps, int slot, PersistParams* pp) {
+  PersistParams& P = *pp;
+  P = PersistParams{};
+  P.G = h->sm_count;
+  P.fp8 = h->fp8 ? 1 : 0;
+  P.sc_qkv = h->sc_qkv; P.sc_o = h->sc_o; P.sc_gu = h->sc_gu; P.sc_down = h->sc_down;
+  P.L = h->L; P.W = h->W; P.H = h->H; P.D = h->D; P.F = h->F; P.A = h->A; P.C = h->C; P.S = h->S;
+  P.Sd = h->Sd; P.hs = h->hs; P.HD = h->HD; P.qkv_rows = h->qkv_rows; P.kcap = h->kcap;
+  P.ring_off = h->ring_off; P.dyn_off = h->dyn_off; P.max_batch = h->cfg.max_batch;
+  P.B = B; P.M = B * h->S; P.steps = steps; P.ada = h->ada ? 1 : 0; P.pi0 = h->pi0 ? 1 : 0; P.np = h->np;
+  P.eps = h->cfg.eps;
+  P.dt = -1.0f / static_cast<float>(steps);
+  P.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h->D));
+  for (int k = 0; k < PH_COUNT; ++k) P.g[k] = h->pg[k];
+  P.att_qtiles = cdiv(static_cast<long>(h->S) * h->H, attn_q_tile());
+  const int kt = attn_key_tile(h->D);
+  const int key_tiles = cdiv(h->cfg.n_static_max, kt) + cdiv(h->cfg.n_sliding, kt) + cdiv(h->S, kt);
+  // at most 24 splits: an owner's merge input (splits x owned rows x (D + 4) fp32) fits the
+  // kernel's 96 KB work area for every head_dim up to 256
+  P.att_splits = std::max(1, std::min(std::min(key_tiles, 24), h->sm_count / (B * P.att_qtiles)));
+  // feature groups per EMBED row and action groups per FINAL row: spread the rows over
+  // the SMs (at most 8 groups; every group at least one feature / action)
+  P.embed_splits = std::max(1, std::min(std::min(8, h->W / 128), h->sm_count / (B * h->S)));
+  P.final_splits = std::max(1, std::min(std::min(8, h->A), h->sm_count / (B * h->C)));
+  P.tbl = h->tables[slot];
+  P.table_stride = h->table_stride;
+  P.ctbl = h->ada ? h->ctables[slot] : nullptr;
+  P.cw = h->qkv_rows + 2L * h->F;
+  P.n1_w = h->n1_w; P.n2_w = h->n2_w; P.nf_w = h->nf_w;
+  P.ain_b = h->ain_b; P.aout_w = h->aout_w; P.aout_b = h->aout_b;
+  P.st_b = h->st_b; P.t2_b = h->t2_b;
+  P.ain_rm = h->p_ain_rm; P.st_rm = h->p_st_rm;
+  P.x = h->x; P.state = h->state; P.resid = h->resid;
+  P.hb = h->hb; P.qb = h->qb; P.ob = h->ob; P.ub = h->ub; P.eb = h->eb; P.h1b = h->h1b;
+  P.kc = h->kc; P.vc = h->vc; P.rope = h->rope; P.cache = h->desc;
+  P.rstat_a = h->p_rstat_a; P.rstat_b = h->p_rstat_b; P.ld_rstat = 64;
+  P.done = h->p_done; P.tctr = h->p_tctr; P.max_tiles = h->p_max_tiles;
+  P.ws = h->p_ws; P.ws_att = h->p_ws_att; P.ws_att_ml = h->p_ws_ml;
+  P.err = h->err;
+  P.trace = h->p_trace;
+}
+
+// The whole denoise as one persistent kernel: counters cleared, then one launch.
+int enqueue_persist(vla_expert* h, int B, int steps, int slot, const ActMaps& am, cudaStream_t s) {
+  PersistParams P;
+  persist_params(h, B, steps, slot, &P);
+  PersistMaps m;
+  m.wqkv = h->tm_wqkv; m.wo = h->tm_wo; m.wgu = h->tm_wgu; m.wdown = h->tm_wdown; m.w1a = h->tm_w1a; m.w2 = h->tm_w2;
+  m.hb = am.hb; m.ob = am.ob; m.ub = am.ub; m.eb = am.eb; m.h1b = am.h1b;
+  m.qa = h->tm_qa; m.ka = h->tm_ka; m.va = h->tm_va;
+  const size_t phases = static_cast<size_t>(steps) * h->np;
+  CU(cudaMemsetAsync(h->p_done, 0, phases * sizeof(int), s));
+  CU(cudaMemsetAsync(h->p_tctr, 0, phases * h->p_max_tiles * sizeof(int), s));
+  CU(launch_denoise_persist(h->D, m, P, s));
+  return VLA_OK;
+}
+
 int get_graph(vla_expert* h, int B, int steps, int slot, cudaGraphExec_t* out) {
   auto key = std::make_pair(B, steps);
   auto it = h->graphs.find(key);
@@ -707,7 +850,7 @@ int get_graph(vla_expert* h, int B, int steps, int slot, cudaGraphExec_t* out) {
   CU(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
   Recorder rec;
   rec.s = h->cap;
-  rc = enqueue_denoise(h, B, steps, slot, am, rec);
+  rc = use_persist(h, B) ? enqueue_persist(h, B, steps, slot, am, h->cap) : enqueue_denoise(h, B, steps, slot, am, rec);
   cudaGraph_t g = nullptr;
   cudaError_t e = cudaStreamEndCapture(h->cap, &g);
   if (rc) {
@@ -806,38 +949,89 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     return code;
   };
 
-  // ---- projection weights, repacked for the GEMM epilogues
+  // ---- projection weights, repacked for the GEMM epilogues: QKV rows in rotary pairs
+  // (row 2i / 2i + 1 = dims i and i + D/2 of one head of Q, then K, then V; padding rows
+  // zero), gate / up rows interleaved. FP8 weights keep their bytes (1 per element) and
+  // carry their per-row scales in the same order.
+  h->fp8 = (cfg->flags & VLA_FLAG_FP8_WEIGHTS) != 0;
   {
-    std::vector<uint16_t> pk(static_cast<size_t>(L) * h->qkv_rows * W, 0);
+    const size_t es = h->fp8 ? 1 : 2;   // bytes per weight element
+    const uint8_t* wq = reinterpret_cast<const uint8_t*>(w->wq);
+    const uint8_t* wk = reinterpret_cast<const uint8_t*>(w->wk);
+    const uint8_t* wv = reinterpret_cast<const uint8_t*>(w->wv);
+    std::vector<uint8_t> pk(static_cast<size_t>(L) * h->qkv_rows * W * es, 0);
+    std::vector<float> sc(h->fp8 ? static_cast<size_t>(L) * h->qkv_rows : 0, 0.0f);
     for (int l = 0; l < L; ++l)
       for (int r = 0; r < (H + 2) * D; ++r) {
         const int pr = r >> 1, second = r & 1;
-        const uint16_t* src;
+        const uint8_t* src;
+        size_t srow;   // source row index into its [L][rows] tensor
         if (pr < H * DH) {
           const int head = pr / DH, i = pr % DH;
-          src = w->wq + (static_cast<size_t>(l) * H * D + head * D + i + second * DH) * W;
+          srow = static_cast<size_t>(l) * H * D + head * D + i + second * DH;
+          src = wq;
+          if (h->fp8) sc[static_cast<size_t>(l) * h->qkv_rows + r] = w->wq_scale[srow];
         } else if (pr < (H + 1) * DH) {
           const int i = pr - H * DH;
-          src = w->wk + (static_cast<size_t>(l) * D + i + second * DH) * W;
+          srow = static_cast<size_t>(l) * D + i + second * DH;
+          src = wk;
+          if (h->fp8) sc[static_cast<size_t>(l) * h->qkv_rows + r] = w->wk_scale[srow];
         } else {
           const int i = pr - (H + 1) * DH;
-          src = w->wv + (static_cast<size_t>(l) * D + i + second * DH) * W;
+          srow = static_cast<size_t>(l) * D + i + second * DH;
+          src = wv;
+          if (h->fp8) sc[static_cast<size_t>(l) * h->qkv_rows + r] = w->wv_scale[srow];
         }
-        std::memcpy(&pk[(static_cast<size_t>(l) * h->qkv_rows + r) * W], src, W * 2);
+        std::memcpy(&pk[(static_cast<size_t>(l) * h->qkv_rows + r) * W * es], src + srow * W * es, W * es);
       }
-    if ((rc = upload_bf16(h, &h->wqkv, pk.data(), pk.size()))) return cleanup(rc);
+    if (h->fp8) {
+      if ((rc = dalloc(h, &h->wqkv8, pk.size()))) return cleanup(rc);
+      CU(cudaMemcpy(h->wqkv8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
+      if ((rc = dalloc(h, &h->sc_qkv, sc.size()))) return cleanup(rc);
+      CU(cudaMemcpy(h->sc_qkv, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
+    } else if ((rc = upload_bf16(h, &h->wqkv, reinterpret_cast<const uint16_t*>(pk.data()), pk.size() / 2))) {
+      return cleanup(rc);
+    }
   }
-  if ((rc = upload_bf16(h, &h->wo, w->wo, static_cast<size_t>(L) * W * h->HD))) return cleanup(rc);
   {
-    std::vector<uint16_t> pk(static_cast<size_t>(L) * 2 * F * W);
+    const size_t es = h->fp8 ? 1 : 2;
+    std::vector<uint8_t> pk(static_cast<size_t>(L) * 2 * F * W * es);
+    std::vector<float> sc(h->fp8 ? static_cast<size_t>(L) * 2 * F : 0);
+    const uint8_t* wg = reinterpret_cast<const uint8_t*>(w->w_gate);
+    const uint8_t* wu = reinterpret_cast<const uint8_t*>(w->w_up);
     for (int l = 0; l < L; ++l)
       for (int f = 0; f < F; ++f) {
-        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f) * W], w->w_gate + (static_cast<size_t>(l) * F + f) * W, W * 2);
-        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f + 1) * W], w->w_up + (static_cast<size_t>(l) * F + f) * W, W * 2);
+        const size_t srow = static_cast<size_t>(l) * F + f;
+        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f) * W * es], wg + srow * W * es, W * es);
+        std::memcpy(&pk[(static_cast<size_t>(l) * 2 * F + 2 * f + 1) * W * es], wu + srow * W * es, W * es);
+        if (h->fp8) {
+          sc[static_cast<size_t>(l) * 2 * F + 2 * f] = w->w_gate_scale[srow];
+          sc[static_cast<size_t>(l) * 2 * F + 2 * f + 1] = w->w_up_scale[srow];
+        }
       }
-    if ((rc = upload_bf16(h, &h->wgu, pk.data(), pk.size()))) return cleanup(rc);
+    if (h->fp8) {
+      if ((rc = dalloc(h, &h->wgu8, pk.size()))) return cleanup(rc);
+      CU(cudaMemcpy(h->wgu8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
+      if ((rc = dalloc(h, &h->sc_gu, sc.size()))) return cleanup(rc);
+      CU(cudaMemcpy(h->sc_gu, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
+    } else if ((rc = upload_bf16(h, &h->wgu, reinterpret_cast<const uint16_t*>(pk.data()), pk.size() / 2))) {
+      return cleanup(rc);
+    }
   }
-  if ((rc = upload_bf16(h, &h->wdown, w->w_down, static_cast<size_t>(L) * W * F))) return cleanup(rc);
+  if (h->fp8) {
+    const size_t no = static_cast<size_t>(L) * W * h->HD, nd = static_cast<size_t>(L) * W * F;
+    if ((rc = dalloc(h, &h->wo8, no))) return cleanup(rc);
+    CU(cudaMemcpy(h->wo8, w->wo, no, cudaMemcpyHostToDevice));
+    if ((rc = dalloc(h, &h->wdown8, nd))) return cleanup(rc);
+    CU(cudaMemcpy(h->wdown8, w->w_down, nd, cudaMemcpyHostToDevice));
+    if ((rc = dalloc(h, &h->sc_o, static_cast<size_t>(L) * W))) return cleanup(rc);
+    CU(cudaMemcpy(h->sc_o, w->wo_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
+    if ((rc = dalloc(h, &h->sc_down, static_cast<size_t>(L) * W))) return cleanup(rc);
+    CU(cudaMemcpy(h->sc_down, w->w_down_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
+  } else {
+    if ((rc = upload_bf16(h, &h->wo, w->wo, static_cast<size_t>(L) * W * h->HD))) return cleanup(rc);
+    if ((rc = upload_bf16(h, &h->wdown, w->w_down, static_cast<size_t>(L) * W * F))) return cleanup(rc);
+  }
 
   // ---- small fp32 parameters
   if ((rc = upload_f32_t(h, &h->ain_w, w->action_in_w, W, h->A))) return cleanup(rc);
@@ -907,11 +1101,58 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = dalloc(h, &h->vc, cache_elems))) return cleanup(rc);
   if (D == 256 && (rc = dalloc(h, &h->vtc, cache_elems))) return cleanup(rc);
   if ((rc = dalloc(h, &h->rope, static_cast<size_t>(h->S) * D))) return cleanup(rc);
-  h->rstat_rows = (W / 128) * 32 + 2;
+  // contributor rows: one per (tile, split owner, 32-row group) in the cluster kernels,
+  // one per (tile, split) item in the persistent kernel (at most one item per SM)
+  h->rstat_rows = std::max((W / 128) * 32 + 2, h->sm_count + 2);
   if ((rc = dalloc(h, &h->rstat_a, static_cast<size_t>(h->rstat_rows) * h->max_M))) return cleanup(rc);
   if ((rc = dalloc(h, &h->rstat_b, static_cast<size_t>(h->rstat_rows) * h->max_M))) return cleanup(rc);
   if ((rc = dalloc(h, &h->desc, 1))) return cleanup(rc);
   if ((rc = dalloc(h, &h->err, 1))) return cleanup(rc);
+
+  // ---- persistent whole-denoise kernel (batches whose suffix tokens fit one 64-token tile)
+  h->persist_bmax = std::min(cfg->max_batch, 64 / h->S);
+  if (h->persist_bmax >= 1) {
+    int per_sm = 0;
+    CU(configure_denoise_persist(D, &per_sm));
+    h->persist_ok = per_sm >= 1;
+  }
+  if (h->persist_ok) {
+    const int G = h->sm_count;
+    h->np = 2 + 2 * (h->pi0 ? 1 : 0) + 5 * L;
+    h->pg[PH_QKV] = persist_plan(h->qkv_rows, W, G);
+    h->pg[PH_O] = persist_plan(W, h->HD, G);
+    h->pg[PH_GU] = persist_plan(2 * F, W, G);
+    h->pg[PH_DOWN] = persist_plan(W, F, G);
+    if (h->pi0) {
+      h->pg[PH_TMLP1] = persist_plan(W, W, G);
+      h->pg[PH_TMLP2] = persist_plan(W, W, G);
+    }
+    const int qtiles = cdiv(static_cast<long>(h->S) * H, attn_q_tile());
+    int items = 0, tiles = h->persist_bmax * qtiles;
+    for (int k = 0; k < PH_COUNT; ++k) {
+      items = std::max(items, h->pg[k].n_tiles * h->pg[k].splits);
+      tiles = std::max(tiles, h->pg[k].n_tiles);
+    }
+    h->p_max_tiles = tiles;
+    const size_t att_slots = static_cast<size_t>(std::max(G, h->persist_bmax * qtiles));
+    const size_t phases = static_cast<size_t>(cfg->max_steps) * h->np;
+    if ((rc = dalloc(h, &h->p_done, phases))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_tctr, phases * tiles))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_ws, static_cast<size_t>(items) * 128 * 64))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_ws_att, att_slots * attn_q_tile() * D))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_ws_ml, att_slots * attn_q_tile() * 4))) return cleanup(rc);
+    // contributor rows: at most one per (tile, split) item, plus the embed feature groups
+    if ((rc = dalloc(h, &h->p_rstat_a, static_cast<size_t>(G + 16) * 64))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_rstat_b, static_cast<size_t>(G + 16) * 64))) return cleanup(rc);
+    if ((rc = upload_f32_rowpad(h, &h->p_ain_rm, w->action_in_w, W, h->A))) return cleanup(rc);
+    if (h->hs && (rc = upload_f32_rowpad(h, &h->p_st_rm, w->state_in_w, W, h->Sd))) return cleanup(rc);
+    if (getenv("VLA_TRACE_FILE") &&
+        (rc = dalloc(h, &h->p_trace, static_cast<size_t>(h->np) * G * 8)))
+      return cleanup(rc);
+  }
+  if (h->fp8 && !(h->persist_ok && h->persist_bmax >= cfg->max_batch))
+    return cleanup(fail(VLA_ERR_UNSUPPORTED, "FP8 weights need max_batch x suffix <= 64 (got %d x %d)",
+                        cfg->max_batch, h->S));
 
   // ---- time tables
   h->table_stride = h->ada ? static_cast<long>(2 * L + 1) * 3 * W : W;
@@ -927,10 +1168,17 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if ((rc = dalloc(h, &h->tscr2, static_cast<size_t>(cfg->max_steps) * W))) return cleanup(rc);
 
   // ---- TMA descriptors of the stacked weights
-  if ((rc = make_tmap(&h->tm_wqkv, h->wqkv, W, static_cast<uint64_t>(L) * h->qkv_rows, 128))) return cleanup(rc);
-  if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
-  if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
-  if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  if (h->fp8) {
+    if ((rc = make_tmap_u8(&h->tm_wqkv, h->wqkv8, W, static_cast<uint64_t>(L) * h->qkv_rows, 128))) return cleanup(rc);
+    if ((rc = make_tmap_u8(&h->tm_wo, h->wo8, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+    if ((rc = make_tmap_u8(&h->tm_wgu, h->wgu8, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
+    if ((rc = make_tmap_u8(&h->tm_wdown, h->wdown8, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  } else {
+    if ((rc = make_tmap(&h->tm_wqkv, h->wqkv, W, static_cast<uint64_t>(L) * h->qkv_rows, 128))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
+  }
   {
     const uint64_t rows = static_cast<uint64_t>(L) * cfg->max_batch * h->kcap;
     const uint32_t bc = static_cast<uint32_t>(attn_box_cols(D)), kt = static_cast<uint32_t>(attn_key_tile(D));
@@ -983,6 +1231,17 @@ void vla_expert_destroy(vla_expert* h) {
               const unsigned long long v = t[(static_cast<size_t>(r) * 512 + c) * 16 + k];
               if (v) fprintf(f, "%s,%d,%d,%llu\n", names[r], c, k, v);
             }
+        fclose(f);
+      }
+    }
+  }
+  if (h->p_trace && !h->trace_file.empty()) {
+    const size_t n = static_cast<size_t>(h->np) * h->sm_count * 8;
+    std::vector<unsigned long long> t(n);
+    if (cudaMemcpy(t.data(), h->p_trace, n * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
+      if (FILE* f = fopen(h->trace_file.c_str(), "a")) {
+        for (size_t i = 0; i < n; ++i)
+          if (t[i]) fprintf(f, "persist,%zu,%zu,%zu,%llu\n", i / (8 * h->sm_count), (i / 8) % h->sm_count, i % 8, t[i]);
         fclose(f);
       }
     }
@@ -1150,7 +1409,14 @@ int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, i
   rec.s = s;
   rec.events = &ev;
   rec.kinds = &kinds;
-  rc = enqueue_denoise(h, batch, steps, slot, am, rec);
+  const bool persist = use_persist(h, batch);
+  if (persist) {
+    rec.begin(VLA_K_PERSIST);
+    rc = enqueue_persist(h, batch, steps, slot, am, s);
+    rec.end(VLA_K_PERSIST);
+  } else {
+    rc = enqueue_denoise(h, batch, steps, slot, am, rec);
+  }
   if (rc == VLA_OK) {
     cudaError_t e = cudaMemcpyAsync(out_actions, h->x, xb, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -1169,13 +1435,15 @@ int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, i
     const double HD = h->HD, D = h->D, F = h->F;
     const double qkv = static_cast<double>((h->H + 2) * h->D);
     const double keys = static_cast<double>(h->n_static + h->n_ring + h->S);
-    times->bytes[VLA_K_GEMM_QKV] = N * L * (2.0 * qkv * W + 2.0 * M * W + 2.0 * M * qkv);
+    // weight bytes per element: bf16, or one E4M3 byte plus an fp32 scale per output row
+    const double wb = h->fp8 ? 1.0 : 2.0, sb = h->fp8 ? 4.0 : 0.0;
+    times->bytes[VLA_K_GEMM_QKV] = N * L * (wb * qkv * W + sb * qkv + 2.0 * M * W + 2.0 * M * qkv);
     times->flops[VLA_K_GEMM_QKV] = N * L * 2.0 * M * qkv * W;
-    times->bytes[VLA_K_GEMM_O] = N * L * (2.0 * W * HD + 2.0 * M * HD + 8.0 * M * W);
+    times->bytes[VLA_K_GEMM_O] = N * L * (wb * W * HD + sb * W + 2.0 * M * HD + 8.0 * M * W);
     times->flops[VLA_K_GEMM_O] = N * L * 2.0 * M * W * HD;
-    times->bytes[VLA_K_GEMM_GATEUP] = N * L * (2.0 * 2 * F * W + 2.0 * M * W + 2.0 * M * F);
+    times->bytes[VLA_K_GEMM_GATEUP] = N * L * (wb * 2 * F * W + sb * 2 * F + 2.0 * M * W + 2.0 * M * F);
     times->flops[VLA_K_GEMM_GATEUP] = N * L * 2.0 * M * 2 * F * W;
-    times->bytes[VLA_K_GEMM_DOWN] = N * L * (2.0 * W * F + 2.0 * M * F + 8.0 * M * W);
+    times->bytes[VLA_K_GEMM_DOWN] = N * L * (wb * W * F + sb * W + 2.0 * M * F + 8.0 * M * W);
     times->flops[VLA_K_GEMM_DOWN] = N * L * 2.0 * M * W * F;
     times->bytes[VLA_K_ATTN] = N * L * (B * keys * D * 2 * 2 + 2.0 * 2 * M * HD);
     times->flops[VLA_K_ATTN] = N * L * 4.0 * M * h->H * keys * D;
@@ -1185,6 +1453,20 @@ int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, i
     if (h->pi0) {
       times->bytes[VLA_K_TIME_MLP] = N * (2.0 * 2 * W * W + 2.0 * 2 * M * W + 2.0 * M * W + 4.0 * M * W);
       times->flops[VLA_K_TIME_MLP] = N * 2.0 * 2.0 * M * W * W;
+    }
+    if (persist) {
+      // one launch does every step of the denoise: it carries the whole denoise's counts
+      double bsum = 0.0, fsum = 0.0;
+      for (int k = 0; k < VLA_K_COUNT; ++k) {
+        if (k == VLA_K_PERSIST || k == VLA_K_NORM) continue;   // no separate norm pass
+        bsum += times->bytes[k];
+        fsum += times->flops[k];
+        times->bytes[k] = 0.0;
+        times->flops[k] = 0.0;
+      }
+      times->bytes[VLA_K_NORM] = 0.0;
+      times->bytes[VLA_K_PERSIST] = bsum;
+      times->flops[VLA_K_PERSIST] = fsum;
     }
   }
   for (auto e : ev) cudaEventDestroy(e);

@@ -21,106 +21,9 @@
 //
 // Mask (prefix-LM): every suffix row sees every cached key; action rows see the whole
 // suffix; with a state token, suffix row 0 sees the cached keys and itself only.
-#include <cfloat>
-
-#include "kernels.h"
-#include "ptx.cuh"
+#include "attn_core.cuh"
 
 namespace vla {
-
-constexpr int kQT = 64;   // query rows per CTA
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&t);
-}
-
-template <int D>
-struct AttnCfg {
-  static constexpr int KT = D >= 256 ? 32 : 64;            // keys per stage
-  static constexpr int CPR = D / 8;                        // 16-byte chunks per row
-  // TMA boxes: BW columns wide (128-byte rows with the 128-byte swizzle; 64-byte rows with
-  // the 64-byte swizzle for D = 32), NBOX boxes across a row
-  static constexpr int BW = D >= 64 ? 64 : D;
-  static constexpr int ROWB = BW * 2;
-  static constexpr int CPB = ROWB / 16;                    // 16-byte chunks per box row
-  static constexpr int NBOX = D / BW;
-  static constexpr int Q_BYTES = kQT * D * 2;
-  static constexpr int KV_BYTES = KT * D * 2;              // one K (or V) stage
-  // 1 KB alignment slack, Q, 2 x (K, V) stages, 3 mbarriers
-  static constexpr size_t MAIN = 1024 + (size_t)Q_BYTES + 4 * (size_t)KV_BYTES + 64;
-  // split merge: each CTA receives, from every split of its cluster, the unnormalised O
-  // rows it owns ([splits][64/splits][D], 64 rows in total) and their (m, l)
-  static constexpr size_t RECV_O = (size_t)kQT * D * 4;
-  static constexpr size_t RECV_ML = (size_t)kQT * 8;
-  static constexpr size_t SMEM = MAIN + RECV_O + RECV_ML + 16;
-};
-
-// Byte offset of 16-byte chunk `chunk` of row `row` in a [ROWS][D] bf16 tile as TMA
-// writes it: NBOX boxes of [ROWS][ROWB bytes], chunks XOR-swizzled within a row by
-// (row & 7) (128-byte rows) or ((row >> 1) & 3) (64-byte rows).
-template <int D, int ROWS>
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  using C = AttnCfg<D>;
-  const int box = chunk / C::CPB, w = chunk % C::CPB;
-  const int x = C::ROWB == 128 ? (row & 7) : ((row >> 1) & 3);
-  return static_cast<uint32_t>(box * ROWS * C::ROWB + row * C::ROWB + ((w ^ x) << 4));
-}
-
-// Key tile t of the concatenated segment list -> (segment row offset, first key, count).
-struct Segs {
-  int off[3], cnt[3], ntile[3];
-};
-
-template <int D>
-__device__ __forceinline__ void tile_info(const Segs& sg, int t, int& row, int& cnt, int& dyn_start) {
-  using C = AttnCfg<D>;
-  // segment selection by compares and selects (no indexing of the arrays by a run-time value,
-  // which would place them in local memory)
-  const bool s0 = t < sg.ntile[0];
-  const bool s1 = !s0 && t < sg.ntile[0] + sg.ntile[1];
-  const int first = s0 ? 0 : (s1 ? sg.ntile[0] : sg.ntile[0] + sg.ntile[1]);
-  const int off = s0 ? sg.off[0] : (s1 ? sg.off[1] : sg.off[2]);
-  const int n = s0 ? sg.cnt[0] : (s1 ? sg.cnt[1] : sg.cnt[2]);
-  const int start = (t - first) * C::KT;
-  row = off + start;
-  cnt = min(C::KT, n - start);
-  dyn_start = (!s0 && !s1) ? start : -1;
-}
-
-// TMA loads of key tile t (K and V) into stage buffers sk / sv, completing on bar.
-template <int D>
-__device__ __forceinline__ void issue_kv_tile(const CUtensorMap* tm_k, const CUtensorMap* tm_v, const Segs& sg,
-                                              int t, int row_base, uint32_t sk, uint32_t sv, uint32_t bar,
-                                              uint64_t pol) {
-  using C = AttnCfg<D>;
-  int row, cnt, ds;
-  tile_info<D>(sg, t, row, cnt, ds);
-  mbar_arrive_expect_tx(bar, 2 * C::KV_BYTES);
-#pragma unroll
-  for (int bx = 0; bx < C::NBOX; ++bx) {
-    tma_load_2d(sk + bx * C::KT * C::ROWB, tm_k, bar, bx * C::BW, row_base + row, pol);
-    tma_load_2d(sv + bx * C::KT * C::ROWB, tm_v, bar, bx * C::BW, row_base + row, pol);
-  }
-}
 
 // CTA rank r of the cluster owns rows [r*64/NS, (r+1)*64/NS) of the query tile; every
 // split has pushed its unnormalised O rows and (m, l) for them into r's receive buffers
@@ -165,8 +68,7 @@ __global__ void __launch_bounds__(128)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D>;
-  constexpr int KT = C::KT;
-  constexpr int NB = KT / 8;     // 8-key column blocks of S
+  constexpr int KT = C::KT;      // keys per tile
   constexpr int OB = D / 8;      // 8-dim column blocks of O
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -238,11 +140,8 @@ __global__ void __launch_bounds__(128)
   }
   mbar_wait(qbar, 0, p.err);
 
-  float o[OB][4];
-#pragma unroll
-  for (int i = 0; i < OB; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.0f, 0.0f};
+  AttnAcc<D> acc;
+  acc.init();
 
   const int wrow = warp * 16;                      // this warp's first row in the tile
   const int g = lane >> 2, qd = lane & 3;          // fragment row group / quad position
@@ -259,99 +158,14 @@ __global__ void __launch_bounds__(128)
     const uint32_t sK = sK0 + st * C::KV_BYTES, sV = sV0 + st * C::KV_BYTES;
     int trow, tcnt, dyn_start;
     tile_info<D>(sg, t, trow, tcnt, dyn_start);
-
-    // S = Q K^T for this warp's 16 rows x KT keys; even and odd 16-wide K steps accumulate
-    // separately (two dependent MMA chains of D/32 instead of one of D/16), summed after
-    float sacc[NB][4], sodd[NB][4];
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[i][e] = sodd[i][e] = 0.0f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t a[4];
-      ldsm_x4(a, sQ + swz<D, kQT>(wrow + (lane & 15), kk * 2 + (lane >> 4)));
-#pragma unroll
-      for (int nb2 = 0; nb2 < KT / 16; ++nb2) {
-        uint32_t bf[4];
-        ldsm_x4(bf, sK + swz<D, KT>(nb2 * 16 + (lane & 7) + ((lane >> 4) << 3), kk * 2 + ((lane >> 3) & 1)));
-        float (&acc0)[4] = (kk & 1) ? sodd[2 * nb2] : sacc[2 * nb2];
-        float (&acc1)[4] = (kk & 1) ? sodd[2 * nb2 + 1] : sacc[2 * nb2 + 1];
-        mma_bf16_16816(acc0, a, bf[0], bf[1]);
-        mma_bf16_16816(acc1, a, bf[2], bf[3]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < NB; ++i)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[i][e] += sodd[i][e];
-    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 8);
-    // scale into the log2 domain and mask
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = nb * 8 + qd * 2 + (e & 1);
-        bool ok = col < tcnt;
-        if (dyn_start >= 0 && p.has_state && s_row[e >> 1] == 0 && dyn_start + col != 0) ok = false;
-        const float v = ok ? sacc[nb][e] * p.scale_log2 : -INFINITY;
-        sacc[nb][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-    float corr[2];
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
-      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
-      const float m_new = fmaxf(m_run[h2], mx[h2]);
-      corr[h2] = (m_run[h2] == -INFINITY) ? 0.0f : exp2_approx(m_run[h2] - m_new);
-      m_run[h2] = m_new;
-    }
-    float lsum[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float mref = m_run[e >> 1];
-        const float pv = (mref == -INFINITY) ? 0.0f : exp2_approx(sacc[nb][e] - mref);
-        sacc[nb][e] = pv;
-        lsum[e >> 1] += pv;
-      }
-    }
-#pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) l_run[h2] = l_run[h2] * corr[h2] + lsum[h2];
-    if (!__all_sync(0xffffffffu, corr[0] == 1.0f && corr[1] == 1.0f)) {   // the running max moved
-#pragma unroll
-      for (int i = 0; i < OB; ++i) {
-        o[i][0] *= corr[0];
-        o[i][1] *= corr[0];
-        o[i][2] *= corr[1];
-        o[i][3] *= corr[1];
-      }
-    }
-    if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 9);
-    // O += P V
-#pragma unroll
-    for (int kb = 0; kb < KT / 16; ++kb) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16(sacc[2 * kb][0], sacc[2 * kb][1]);
-      pa[1] = pack_bf16(sacc[2 * kb][2], sacc[2 * kb][3]);
-      pa[2] = pack_bf16(sacc[2 * kb + 1][0], sacc[2 * kb + 1][1]);
-      pa[3] = pack_bf16(sacc[2 * kb + 1][2], sacc[2 * kb + 1][3]);
-#pragma unroll
-      for (int db = 0; db < D / 16; ++db) {
-        uint32_t vf[4];
-        ldsm_x4_t(vf, sV + swz<D, KT>(kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), db * 2 + (lane >> 4)));
-        mma_bf16_16816(o[2 * db], pa, vf[0], vf[1]);
-        mma_bf16_16816(o[2 * db + 1], pa, vf[2], vf[3]);
-      }
-    }
+    attn_tile_math<D>(acc, sQ, sK, sV, wrow, lane, tcnt, dyn_start, p.has_state, s_row, p.scale_log2);
     if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 10);
     __syncthreads();
     if (threadIdx.x == 0 && t == t_begin) trace_stamp(p.trace, 7);
   }
+  float (&o)[OB][4] = acc.o;
+  float (&m_run)[2] = acc.m_run;
+  float (&l_run)[2] = acc.l_run;
 
   if (threadIdx.x == 0) trace_stamp(p.trace, 2);
   // quad-reduce the row sums

@@ -72,6 +72,7 @@ struct GemmParams {
   int* counters;      // one arrival counter per output tile (left at 0)
   int* err;           // device status word
   unsigned long long* trace;   // optional: [ctas][16] %globaltimer stamps, or null
+  const float* wscale;   // FP8 weights: per-output-feature scale (indexed by feature), or null
 };
 
 // tn: token tile (64, 128 or 256). cluster = false: split partials through p.ws /
@@ -182,6 +183,9 @@ cudaError_t launch_temb(float* temb, int steps, int time_dim, cudaStream_t s);
 // y[r * ldy + o] = act(sum_i x[r * ldx + i] * w[o * ldw + i] + b[o]), r < rows, o < n_out.
 cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const bf16* w, long ldw,
                            const bf16* b, int n_out, float* y, long ldy, int act_swish, cudaStream_t s);
+// The same with E4M3 weight bytes and a per-output scale: w[o][i] = wscale[o] * e4m3(w8[o][i]).
+cudaError_t launch_rowgemv_fp8(const float* x, int rows, int n_in, long ldx, const uint8_t* w8, long ldw,
+                               const float* wscale, int n_out, float* y, long ldy, cudaStream_t s);
 
 // Cache maintenance.
 // vt: optional transposed V cache [L][max_batch][D][kcap] (null: none).
@@ -200,6 +204,66 @@ cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, 
                           cudaStream_t s, bool pdl);
 cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch,
                                int kcap, int rows, int D, int n_static_max, int ring_off, cudaStream_t s);
+
+// ------------------------------------------------------ persistent denoise kernel
+// One launch runs a whole denoise of one token tile (batch x suffix <= 64): all Euler
+// steps, all layers, every phase, with completion counters between the phases.
+
+enum PhaseKind : int {
+  PH_EMBED = 0, PH_TMLP1 = 1, PH_TMLP2 = 2,
+  PH_QKV = 3, PH_ATT = 4, PH_O = 5, PH_GU = 6, PH_DOWN = 7,   // per layer, in this order
+  PH_FINAL = 8, PH_COUNT = 9
+};
+
+struct PersistGemm {
+  int n_tiles;   // 128-feature weight tiles
+  int nkb;       // 64-wide K blocks
+  int splits;    // K splits per tile (items = n_tiles * splits)
+};
+
+struct PersistMaps {
+  CUtensorMap wqkv, wo, wgu, wdown, w1a, w2;   // stacked weights, 128 x 64 boxes
+  CUtensorMap hb, ob, ub, eb, h1b;             // activations [M][K], 64 x 64 boxes
+  CUtensorMap qa, ka, va;                      // attention operands (attn_core boxes)
+};
+
+struct PersistParams {
+  int G;                                        // CTAs (one per SM)
+  int fp8;                                      // weights are E4M3 bytes (maps wqkv..wdown)
+  const float *sc_qkv, *sc_o, *sc_gu, *sc_down; // FP8: per-row scales in the packed row order
+  int L, W, H, D, F, A, C, S, Sd, hs, HD, qkv_rows, kcap, ring_off, dyn_off, max_batch;
+  int B, M, steps, ada, pi0, np;               // np: phases per Euler step
+  float eps, dt, scale_log2;
+  PersistGemm g[PH_COUNT];                      // projection phases
+  int att_qtiles, att_splits;                   // per observation (splits <= 24)
+  int embed_splits, final_splits;               // feature / action groups per row
+  const float* tbl;                             // time tables [steps][...]
+  long table_stride;
+  const float* ctbl;                            // W . shift tables (AdaRMSNorm)
+  long cw;
+  const float *n1_w, *n2_w, *nf_w, *ain_b, *aout_w, *aout_b, *st_b, *t2_b;
+  const float *ain_rm, *st_rm;                  // embed maps row-major [W][in padded to 4]
+  float* x;
+  const float* state;
+  float* resid;
+  bf16 *hb, *qb, *ob, *ub, *eb, *h1b, *kc, *vc;
+  const float* rope;
+  const CacheDesc* cache;
+  float *rstat_a, *rstat_b;                     // [contributor][64] sums of squares
+  int ld_rstat;
+  int* done;             // [steps * np] items finished per phase (zeroed before launch)
+  int* tctr;             // [steps * np][max_tiles] partials arrived per tile (zeroed)
+  int max_tiles;
+  float* ws;             // projection partials [tile][owner][split][owned rows][64]
+  float* ws_att;         // attention partials [group][owner][split][owned rows][D]
+  float* ws_att_ml;      // [group][owner][split][owned rows][4] (running max, sum)
+  int* err;
+  unsigned long long* trace;
+};
+
+cudaError_t launch_denoise_persist(int head_dim, const PersistMaps& maps, const PersistParams& p, cudaStream_t s);
+// Sets the kernel attributes and reports how many CTAs of it fit on one SM.
+cudaError_t configure_denoise_persist(int head_dim, int* ctas_per_sm);
 
 // Arms an mbarrier nothing arrives on and waits on it for limit_ns, so the wait gives up
 // and records a timeout in *err (failure-path self-test).

@@ -8,6 +8,9 @@
 //  temb/rowgemv  per-step time tables: t-embedding, time MLP, AdaRMSNorm modulation
 //  prefix_set / ring_append / cache_update / copy_region: the static / sliding regions
 //              (Reflex abstract: O(1) incremental cache updates)
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <cmath>
 
 #include "kernels.h"
@@ -245,6 +248,40 @@ __global__ void __launch_bounds__(256) rowgemv_kernel(const float* x, int rows, 
         y[static_cast<size_t>(r0 + j) * ldy + o] = act_swish ? swishf(v) : v;
     }
   }
+}
+
+// One warp per output feature, FP8 weights widened exactly (E4M3 -> half -> float).
+__global__ void __launch_bounds__(256) rowgemv_fp8_kernel(const float* x, int rows, int n_in, long ldx,
+                                                          const uint8_t* w8, long ldw, const float* wscale,
+                                                          int n_out, float* y, long ldy) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * 8 + warp;
+  if (o >= n_out) return;
+  const uint8_t* wr = w8 + static_cast<size_t>(o) * ldw;
+  const float sc = wscale[o];
+  for (int r0 = 0; r0 < rows; r0 += 8) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    for (int i = lane; i < n_in; i += 32) {
+      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(wr[i]), __NV_E4M3);
+      const float wv = __half2float(__half(hr)) * sc;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (r0 + j < rows) acc[j] = fmaf(wv, x[static_cast<size_t>(r0 + j) * ldx + i], acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float v = warp_sum(acc[j]);
+      if (lane == 0 && r0 + j < rows) y[static_cast<size_t>(r0 + j) * ldy + o] = v;
+    }
+  }
+}
+
+cudaError_t launch_rowgemv_fp8(const float* x, int rows, int n_in, long ldx, const uint8_t* w8, long ldw,
+                               const float* wscale, int n_out, float* y, long ldy, cudaStream_t s) {
+  rowgemv_fp8_kernel<<<(n_out + 7) / 8, 256, 0, s>>>(x, rows, n_in, ldx, w8, ldw, wscale, n_out, y, ldy);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_rowgemv(const float* x, int rows, int n_in, long ldx, const bf16* w, long ldw,

@@ -76,7 +76,19 @@ typedef enum vla_time_kind {
 #define VLA_FLAG_NORM_KERNELS 2u /* with one token tile (batch x suffix <= 64), run the
                                     pre-attention / pre-MLP norms as kernels of their own
                                     instead of folding them into the projections (cross-check;
-                                    larger batches always use norm kernels) */
+                                    larger batches always use norm kernels; implies
+                                    VLA_FLAG_NO_PERSIST) */
+#define VLA_FLAG_NO_PERSIST 4u   /* with one token tile, run the denoise as one kernel launch
+                                    per projection / attention / embed / final step (captured
+                                    in a graph) instead of the single persistent kernel that
+                                    runs the whole loop (cross-check) */
+#define VLA_FLAG_FP8_WEIGHTS 8u  /* the projection matrices wq, wk, wv, wo, w_gate, w_up,
+                                    w_down are FP8 E4M3 bytes with fp32 per-output-row scales
+                                    (vla_weights *_scale); streamed as FP8 and widened to bf16
+                                    in shared memory, exactly (InstinctFlash README: the pi05
+                                    FP8 configuration). Needs max_batch x suffix <= 64 (the
+                                    persistent one-tile path); not combinable with
+                                    VLA_FLAG_NO_PERSIST or VLA_FLAG_NORM_KERNELS. */
 
 typedef struct vla_config {
   int n_layers;      /* L */
@@ -115,6 +127,9 @@ typedef struct vla_config {
  *                       norm2_mod_b (same), final_norm_mod_w [3W][Cd],
  *                       final_norm_mod_b [3W]; Cd = W (ADA_MLP) or time_dim (ADA_SINCOS);
  *                       the 3W outputs split as [scale | shift | gate].
+ *   VLA_FLAG_FP8_WEIGHTS: wq, wk, wv, wo, w_gate, w_up, w_down point to E4M3 bytes (uint8,
+ *                       same shapes; sign, 4-bit exponent with bias 7, 3-bit mantissa) and
+ *                       *_scale to fp32 scales [L][out]: weight = scale[row] * e4m3(byte).
  * Pointers a configuration does not use may be NULL.
  */
 typedef struct vla_weights {
@@ -126,6 +141,7 @@ typedef struct vla_weights {
   const uint16_t *norm1_mod_w, *norm1_mod_b, *norm2_mod_w, *norm2_mod_b;
   const uint16_t *final_norm_mod_w, *final_norm_mod_b;
   const uint16_t *wq, *wk, *wv, *wo, *w_gate, *w_up, *w_down;
+  const float *wq_scale, *wk_scale, *wv_scale, *wo_scale, *w_gate_scale, *w_up_scale, *w_down_scale;
 } vla_weights;
 
 typedef struct vla_expert vla_expert;   /* opaque, owned by the library */
@@ -226,7 +242,9 @@ VLA_API int vla_selftest_wait_timeout(vla_expert* h, int limit_us, void* cuda_st
 typedef enum vla_kernel_kind {
   VLA_K_GEMM_QKV = 0, VLA_K_ATTN = 1, VLA_K_GEMM_O = 2, VLA_K_GEMM_GATEUP = 3,
   VLA_K_GEMM_DOWN = 4, VLA_K_NORM = 5, VLA_K_EMBED = 6, VLA_K_FINAL = 7,
-  VLA_K_TIME_MLP = 8, VLA_K_COUNT = 9
+  VLA_K_TIME_MLP = 8,
+  VLA_K_PERSIST = 9,   /* the persistent whole-denoise kernel (one token tile): one launch */
+  VLA_K_COUNT = 10
 } vla_kernel_kind;
 
 typedef struct vla_kernel_times {
@@ -241,7 +259,9 @@ typedef struct vla_kernel_times {
  * a second graph that brackets every kernel with CUDA event records, and fill *times
  * (host struct) with per-kind device time, launch counts and the algorithmic byte and
  * FLOP counts. Synchronizes the stream. The events serialise the kernels, so use it for
- * per-kernel shares, not for the end-to-end time.
+ * per-kernel shares, not for the end-to-end time. When the denoise runs as the one
+ * persistent kernel, that launch is the only entry (VLA_K_PERSIST), with the byte and
+ * FLOP counts of the whole denoise.
  */
 VLA_API int vla_profile_kernels(vla_expert* h, const float* noise, const float* state, int steps,
                         float* out_actions, int batch, vla_kernel_times* times,

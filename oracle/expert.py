@@ -39,8 +39,35 @@ def bf16_to_f64(bits) -> np.ndarray:
     return u.view(np.float32).astype(F64)
 
 
+def e4m3_to_f64(bits) -> np.ndarray:
+    """Exact value of FP8 E4M3 bit patterns (uint8): sign bit, 4-bit exponent e with bias 7,
+    3-bit mantissa m; e = 0 is subnormal, m/8 * 2^-6; otherwise (1 + m/8) * 2^(e - 7); the
+    pattern with e = 15 and m = 7 is NaN (the format has no infinities). Used for the FP8
+    projection weights of the InstinctFlash README's pi05 FP8 configuration."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(F64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(F64)))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
 def decode_params(bits: dict) -> dict:
-    return {k: bf16_to_f64(v) for k, v in bits.items()}
+    """Parameters as float64. bf16 tensors (uint16 bit patterns) widen exactly; FP8 tensors
+    (uint8 E4M3 bit patterns, with an fp32 per-output-row scale under "<name>.scale") are
+    their exact E4M3 values times the row's scale."""
+    out = {}
+    for k, v in bits.items():
+        if k.endswith(".scale"):
+            continue
+        v = np.asarray(v)
+        if v.dtype == np.uint8:
+            scale = np.asarray(bits[k + ".scale"], dtype=np.float32).astype(F64)
+            out[k] = e4m3_to_f64(v) * scale[..., None]
+        else:
+            out[k] = bf16_to_f64(v)
+    return out
 
 
 # ------------------------------------------------------------------------- primitives

@@ -95,9 +95,15 @@ def test_host_argument_checks(lib):
                                  ctypes.byref(h)) == V.VLA_ERR_UNSUPPORTED
     assert lib.vla_expert_create(ctypes.byref(_cfg(time_kind=7)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG
-    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=8)), ctypes.byref(w),
+    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=16)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG
     assert "flag" in V.vla_last_error()
+    # FP8 weights: every scale pointer is required, and only the persistent one-tile path
+    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_FP8_WEIGHTS)), ctypes.byref(w),
+                                 ctypes.byref(h)) == V.VLA_ERR_ARG
+    assert "scale" in V.vla_last_error()
+    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_FP8_WEIGHTS | V.VLA_FLAG_NO_PERSIST)),
+                                 ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_UNSUPPORTED
     # a valid shape with missing weights is an argument error, still before any CUDA call
     assert lib.vla_expert_create(ctypes.byref(_cfg()), ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
     assert lib.vla_denoise(None, None, None, 4, None, 1, None) == V.VLA_ERR_ARG

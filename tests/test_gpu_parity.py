@@ -136,6 +136,73 @@ def test_norm_kernels_path_matches_folded_norms():
         check_actions(outs[0], outs[1], name + " folded vs norm kernels")
 
 
+def _first_obs(wl, inp, n):
+    from dataclasses import replace
+    inp = dict(inp, noise=inp["noise"][:n], prefix_k=inp["prefix_k"][:, :n], prefix_v=inp["prefix_v"][:, :n],
+               state=None if inp.get("state") is None else inp["state"][:n])
+    return replace(wl, batch=n), inp
+
+
+@pytest.mark.parametrize("name, obs", [("tiny", None), ("mid_d128", None), ("mid_pi0_b3", 1), ("mid_ada_b2", 1),
+                                       ("pi0_1view", None), ("pi05_3view", None)])
+def test_persistent_kernel_matches_oracle_and_the_launch_chain(name, obs):
+    """The whole denoise as one persistent kernel (the default for one token tile: D = 32,
+    64, 128, 256; AdaRMSNorm and Pi0 time MLP with a state token; two observations in one
+    tile) and as the chain of per-step kernel launches (VLA_FLAG_NO_PERSIST), on the same
+    inputs: both within the acceptance tolerance of the oracle and of each other; the
+    persistent kernel's result is bit-identical across calls (its split sums run in a
+    fixed order)."""
+    import flow_matching_vla_euler_b200 as V
+    wl = get(name)
+    inp = make_inputs(wl)
+    ref = golden_actions(name) if name in ("tiny", "mid_pi0_b3", "mid_ada_b2", "mid_d128") else None
+    if obs is not None:
+        wl, inp = _first_obs(wl, inp, obs)
+        ref = ref[:obs]
+    if ref is None:
+        ref = oracle_actions(wl, inp)
+    assert wl.batch * wl.expert.suffix_len <= 64
+    outs = []
+    for flags in (0, V.VLA_FLAG_NO_PERSIST):
+        ex, _ = make_expert(wl, inp, flags=flags)
+        load_prefix(ex, inp)
+        outs.append(run(ex, inp, wl.steps))
+        if flags == 0:
+            assert np.array_equal(run(ex, inp, wl.steps), outs[0])
+        ex.device_status()
+        ex.close()
+    check_actions(outs[0], ref, f"{name} persistent")
+    check_actions(outs[1], ref, f"{name} launch chain")
+    check_actions(outs[0], outs[1], f"{name} persistent vs launch chain")
+
+
+@pytest.mark.parametrize("name", ["tiny_fp8", "mid_d128_fp8", "mid_pi0_b1_fp8", "pi05_3view_fp8"])
+def test_fp8_weights_match_oracle(name):
+    """FP8 (E4M3, per-output-row fp32 scale) projection weights, streamed as bytes and
+    widened to bf16 in shared memory by the persistent kernel, against the oracle run on the
+    exact dequantised weights (E4M3 value x row scale, in fp64): the acceptance tolerance,
+    and bit-identical reruns."""
+    wl = get(name)
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    check_actions(got, oracle_actions(wl, inp), name)
+    assert np.array_equal(run(ex, inp, wl.steps), got)
+    ex.device_status()
+    ex.close()
+
+
+def test_fp8_weights_need_one_token_tile():
+    """FP8 weights run on the persistent one-tile path only: a handle whose largest batch
+    does not fit one 64-token tile is refused."""
+    import flow_matching_vla_euler_b200 as V
+    wl = get("mid_pi0_b1_fp8")
+    inp = make_inputs(wl)
+    with pytest.raises(V.VlaError) as e:
+        V.Expert(wl.expert, inp["params"], n_static_max=wl.n_static, max_batch=2, max_steps=wl.steps)
+    assert e.value.code == V.VLA_ERR_UNSUPPORTED
+
+
 def test_batch_rows_match_single_observation_runs():
     wl = get("mid_ada_b2")
     ex, inp = make_expert(wl)

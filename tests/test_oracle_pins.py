@@ -59,6 +59,68 @@ def test_bf16_widening_matches_the_definition_exhaustively():
         assert got[b] == float(sign * v), hex(b)
 
 
+# ------------------------------------------------------------------ FP8 (E4M3) decode
+
+@pytest.mark.parametrize("bits, value", [
+    (0x38, 1.0),                 # e = 7 (bias 7), m = 0
+    (0x39, 1.125),               # 1 + 1/8
+    (0x40, 2.0),
+    (0xB8, -1.0),
+    (0x00, 0.0),
+    (0x01, 2.0 ** -9),           # smallest subnormal: 1/8 * 2^-6
+    (0x07, 7 * 2.0 ** -9),       # largest subnormal
+    (0x08, 2.0 ** -6),           # smallest normal
+    (0x77, 240.0),               # e = 14, m = 7: 1.875 * 2^7
+    (0x7E, 448.0),               # largest finite: e = 15, m = 6: 1.75 * 2^8
+    (0xFE, -448.0),
+])
+def test_e4m3_hand_values(bits, value):
+    """E4M3 = sign | 4-bit exponent (bias 7) | 3-bit mantissa, no infinities; each value here
+    follows from that definition by hand."""
+    got = O.e4m3_to_f64(np.array([bits], dtype=np.uint8))[0]
+    assert got == value
+
+
+def test_e4m3_specials_and_all_patterns():
+    from fractions import Fraction
+    got = O.e4m3_to_f64(np.arange(256, dtype=np.uint16).astype(np.uint8))
+    assert math.copysign(1.0, got[0x80]) == -1.0 and got[0x80] == 0.0
+    assert math.isnan(got[0x7F]) and math.isnan(got[0xFF])
+    for b in range(256):
+        e, m = (b >> 3) & 15, b & 7
+        if e == 15 and m == 7:
+            continue
+        v = Fraction(m, 8) * Fraction(2) ** -6 if e == 0 else (1 + Fraction(m, 8)) * Fraction(2) ** (e - 7)
+        assert got[b] == float(-v if b & 0x80 else v), hex(b)
+
+
+def test_fp8_params_decode_to_value_times_row_scale():
+    """An FP8 weight decodes to its E4M3 value times the fp32 scale of its output row;
+    bf16 tensors beside it are untouched."""
+    q = np.array([[[0x38, 0x40], [0xB8, 0x01]]], dtype=np.uint8)        # [L=1][out=2][in=2]
+    scale = np.array([[0.5, 3.0]], dtype=np.float32)
+    P = O.decode_params({"wq": q, "wq.scale": scale, "wo": np.array([0x3F80], dtype=np.uint16)})
+    assert np.array_equal(P["wq"], np.array([[[0.5, 1.0], [-3.0, 3.0 * 2.0 ** -9]]]))
+    assert P["wo"][0] == 1.0 and "wq.scale" not in P
+
+
+def test_fp8_generator_rounds_to_nearest_even_on_the_e4m3_grid():
+    """The synthetic FP8 weights (input data, not the method) are the nearest E4M3 values of
+    the scaled fp32 draws, ties to the even mantissa, checked by brute force over the grid."""
+    from vla_inputs import f32_to_e4m3_bits
+    grid_bits = np.array([b for b in range(128) if b != 0x7F], dtype=np.uint8)
+    grid = O.e4m3_to_f64(grid_bits)
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 0.05,
+                        (grid[1:] + grid[:-1]) / 2]).astype(np.float32)      # includes exact ties
+    got = O.e4m3_to_f64(f32_to_e4m3_bits(x))
+    for xi, gi in zip(x.astype(np.float64), got):
+        d = np.abs(grid - abs(xi))
+        best = np.flatnonzero(d == d.min())
+        pick = best[0] if len(best) == 1 else [i for i in best if grid_bits[i] % 2 == 0][0]
+        assert gi == math.copysign(grid[pick], xi) or (grid[pick] == 0 and gi == 0)
+
+
 # ------------------------------------------------------------------------- RMSNorm
 
 def test_rmsnorm_closed_form_3_4():

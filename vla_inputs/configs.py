@@ -61,6 +61,7 @@ class Workload:
     steps: int
     seed: int = 0
     ticks: int = 0          # streaming control ticks (sliding workloads)
+    weight_format: str = "bf16"   # "e4m3": projection matrices in FP8 with per-row scales
 
     @property
     def n_cached(self) -> int:
@@ -87,6 +88,9 @@ WORKLOADS = {
     # the same at 64 independent observations
     "pi05_3view_b64": Workload("pi05_3view_b64", PI05, batch=64, n_static=788, n_sliding=0,
                                steps=10),
+    # the 3-view Pi05 denoise with FP8 (E4M3, per-output-channel scale) projection weights
+    "pi05_3view_fp8": Workload("pi05_3view_fp8", PI05, batch=1, n_static=788, n_sliding=0, steps=10,
+                               weight_format="e4m3"),
     # Reflex-style partition: 512 static + 64-slot ring + 50 dynamic, 1000 ticks
     "pi05_stream": Workload("pi05_stream", PI05, batch=1, n_static=512, n_sliding=64,
                             steps=10, ticks=1000),
@@ -111,6 +115,12 @@ TEST_WORKLOADS = {
                          steps=2, seed=3),
     "mid_stream": Workload("mid_stream", MID_ADA, batch=2, n_static=40, n_sliding=16,
                            steps=3, seed=4, ticks=40),
+    "tiny_fp8": Workload("tiny_fp8", TINY, batch=1, n_static=48, n_sliding=0, steps=4,
+                         weight_format="e4m3"),
+    "mid_d128_fp8": Workload("mid_d128_fp8", MID_D128, batch=2, n_static=33, n_sliding=0,
+                             steps=2, seed=3, weight_format="e4m3"),
+    "mid_pi0_b1_fp8": Workload("mid_pi0_b1_fp8", MID_PI0, batch=1, n_static=100, n_sliding=0,
+                               steps=3, seed=1, weight_format="e4m3"),
 }
 
 

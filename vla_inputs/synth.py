@@ -31,6 +31,30 @@ def f32_to_bf16_bits(x) -> np.ndarray:
     return u.astype(np.uint16)
 
 
+def f32_to_e4m3_bits(x) -> np.ndarray:
+    """Round fp32 values to FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+    finite range +-448, no infinities), nearest-even, as uint8 bit patterns. Magnitudes
+    above 448 saturate to 448 (the generator scales rows so that none does)."""
+    x = np.asarray(x, dtype=np.float32)
+    sign = np.signbit(x).astype(np.uint8) << np.uint8(7)
+    a = np.abs(x).astype(np.float64)                    # exact
+    _, ex = np.frexp(np.maximum(a, 2.0 ** -6))          # a = f * 2^ex, f in [0.5, 1)
+    e = np.clip(ex - 1, -6, 8)                          # exponent of the binade (>= the normal floor)
+    q = np.ldexp(1.0, e - 3)                            # spacing of E4M3 values in that binade
+    v = np.minimum(np.round(a / q) * q, 448.0)          # nearest-even on the grid (exact in f64)
+    sub = v < 2.0 ** -6
+    _, ev = np.frexp(np.where(sub, 1.0, v))
+    ev = ev - 1
+    mant = np.round((np.ldexp(np.where(sub, 1.0, v), -ev) - 1.0) * 8.0).astype(np.int64)
+    code = np.where(sub, np.round(v * 2.0 ** 9).astype(np.int64), ((ev + 7) << 3) | mant)
+    return (sign | code.astype(np.uint8)).astype(np.uint8)
+
+
+# Projection matrices stored in FP8 by the "e4m3" weight format (each with a per-output-row
+# fp32 scale); every other parameter stays bf16.
+FP8_NAMES = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down")
+
+
 def bf16_bits_to_f32(b) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
@@ -72,11 +96,21 @@ def param_shapes(cfg: ExpertConfig) -> dict:
     return s
 
 
-def make_params(cfg: ExpertConfig, seed: int = 0, std: float = 0.02) -> dict:
+def make_params(cfg: ExpertConfig, seed: int = 0, std: float = 0.02, weight_format: str = "bf16") -> dict:
+    """Every parameter N(0, std) in fp32 rounded to bf16 bits. With weight_format "e4m3" the
+    projection matrices (FP8_NAMES) are instead stored as E4M3 bits of the same draws
+    divided by a per-output-row fp32 scale (the row's largest magnitude / 448), with the
+    scales under "<name>.scale" ([L, out])."""
     out = {}
     for name, shape in param_shapes(cfg).items():
-        draw = rng_for(seed, "param:" + name).standard_normal(shape, dtype=np.float32)
-        out[name] = f32_to_bf16_bits(draw * np.float32(std))
+        draw = rng_for(seed, "param:" + name).standard_normal(shape, dtype=np.float32) * np.float32(std)
+        if weight_format == "e4m3" and name in FP8_NAMES:
+            amax = np.max(np.abs(draw), axis=-1)
+            scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+            out[name] = f32_to_e4m3_bits(draw / scale[..., None])
+            out[name + ".scale"] = scale
+        else:
+            out[name] = f32_to_bf16_bits(draw)
     return out
 
 
@@ -119,13 +153,13 @@ def make_inputs(wl: Workload, seed: int | None = None) -> dict:
     seed = wl.seed if seed is None else seed
     pk, pv = make_prefix(wl, seed)
     return {
-        "params": make_params(wl.expert, seed),
+        "params": make_params(wl.expert, seed, weight_format=wl.weight_format),
         "prefix_k": pk, "prefix_v": pv,
         "noise": make_noise(wl, seed),
         "state": make_state(wl, seed),
     }
 
 
-__all__ = ["rng_for", "f32_to_bf16_bits", "bf16_bits_to_f32", "param_shapes", "make_params",
+__all__ = ["rng_for", "f32_to_bf16_bits", "f32_to_e4m3_bits", "FP8_NAMES", "bf16_bits_to_f32", "param_shapes", "make_params",
            "make_prefix", "make_noise", "make_state", "make_ring_token", "make_inputs",
            "TIME_ADA_MLP", "TIME_PI0_MLP"]
