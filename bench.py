@@ -53,6 +53,9 @@ def parse_args(argv=None):
                    help="profiling aid: Euler steps per denoise instead of the workload's (0: keep)")
     p.add_argument("--fp8-workload", default="pi05_3view_fp8")
     p.add_argument("--no-fp8", action="store_true")
+    p.add_argument("--path", choices=["auto", "chain", "persistent"], default="auto",
+                   help="denoise path for the bf16 lines: the library's choice, the launch "
+                        "chain, or the persistent whole-denoise kernel")
     return p.parse_args(argv)
 
 
@@ -211,12 +214,13 @@ def job_timing(total_ms: float, steps: int, ws: int, device=None):
 
 # --------------------------------------------------------------- workload set-up
 
-def build_expert(wl, inp):
+def build_expert(wl, inp, path="auto"):
     import numpy as np
     import torch
     import flow_matching_vla_euler_b200 as V
+    flags = {"auto": 0, "chain": V.VLA_FLAG_NO_PERSIST, "persistent": V.VLA_FLAG_PERSIST}[path]
     ex = V.Expert(wl.expert, inp["params"], n_static_max=wl.n_static, n_sliding=wl.n_sliding,
-                  max_batch=wl.batch, max_steps=wl.steps)
+                  max_batch=wl.batch, max_steps=wl.steps, flags=flags)
     bits = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
     ex.set_prefix(bits(inp["prefix_k"]), bits(inp["prefix_v"]))
     noise = torch.from_numpy(inp["noise"]).cuda()
@@ -468,6 +472,7 @@ def cpu_model():
 def run_ours(args):
     import numpy as np
     import torch
+    import flow_matching_vla_euler_b200 as V
     from vla_inputs import get, make_inputs
     ws, rank, local = dist_setup(args)
     peaks, peak_src = load_peaks()
@@ -476,7 +481,7 @@ def run_ours(args):
         from dataclasses import replace
         wl = replace(wl, steps=args.euler_steps)
     inp = make_inputs(wl, seed=wl.seed + rank)
-    ex, noise, state = build_expert(wl, inp)
+    ex, noise, state = build_expert(wl, inp, args.path)
     steps = wl.steps
     with ClockSampler(local, enabled=not args.no_clocks and rank == 0) as clk:
         total_ms, per, _ = time_device(ex, noise, state, steps, args.steps, args.warmup, ws)
@@ -490,6 +495,7 @@ def run_ours(args):
         e_ms = max_over_ranks(e_ms, ws)
         e2e = {"value": round(e_ms / (k_e * ws), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": k_e}
+    persist = V.vla_persist_info(ex.handle)
     roof, acc = (None, None)
     if not args.no_profile:
         roof, acc = roofline(ex, noise, state, steps, peaks, peak_src, wl.name, "hbm")
@@ -572,7 +578,7 @@ def run_ours(args):
             "metric": METRIC, "value": round(value, 4), "unit": "ms", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config_dict(wl, ws),
+            "config": dict(config_dict(wl, ws), persistent_kernel=persist),
             "latency_ms": {"median": round(statistics.median(per), 4),
                            "p10": round(float(np.percentile(per, 10)), 4),
                            "p90": round(float(np.percentile(per, 90)), 4)},

@@ -23,6 +23,7 @@ VLA_FLAG_NO_PDL = 1
 VLA_FLAG_NORM_KERNELS = 2
 VLA_FLAG_NO_PERSIST = 4
 VLA_FLAG_FP8_WEIGHTS = 8
+VLA_FLAG_PERSIST = 16
 KERNEL_KINDS = ["gemm_qkv", "attention", "gemm_o", "gemm_gateup", "gemm_down", "norm", "embed",
                 "final_euler", "time_mlp", "denoise_persist"]
 
@@ -82,6 +83,7 @@ _SIGNATURES = {
     "vla_gemm_bf16_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "vla_selftest_wait_timeout": (_I, [_P, _I, _P]),
     "vla_gemm_status": (_I, [_P]),
+    "vla_persist_info": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "vla_last_error": (ctypes.c_char_p, []),
     "vla_version": (ctypes.c_char_p, []),
 }
@@ -156,6 +158,12 @@ def vla_device_status(h, stream):
 
 def vla_selftest_wait_timeout(h, limit_us, stream):
     _check(load_library().vla_selftest_wait_timeout(h, limit_us, stream))
+
+
+def vla_persist_info(h):
+    a, b, c = _I(), _I(), _I()
+    _check(load_library().vla_persist_info(h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return {"ctas": a.value, "cluster": b.value, "max_clusters": c.value}
 
 
 def vla_gemm_status(stream):

@@ -122,9 +122,35 @@ PersistGemm persist_plan(int n_feat, int k_dim, int G) {
   g.n_tiles = n_feat / 128;
   g.nkb = k_dim / 64;
   int S = g.n_tiles >= G ? 1 : G / g.n_tiles;
+  S = std::max(S, (g.nkb + 7) / 8);   // at most 8 K blocks (128 KB of weights) per item
   S = std::min(S, g.nkb);
   S = std::min(S, 20);
   g.splits = std::max(S, 1);
+  g.tpc = 0;
+  return g;
+}
+
+// Cluster size of the persistent kernel when clusters are used.
+constexpr int kPersistCluster = 8;
+
+// Cluster plan: the splits of a tile are consecutive ranks of one cluster (S in 8, 4, 2,
+// 1, at most the K blocks), as many as fit every tile into one round over nc clusters;
+// splits = 0 when no split count fits with at most 8 K blocks (128 KB of weights) per CTA.
+PersistGemm persist_plan_cluster(int n_feat, int k_dim, int nc) {
+  PersistGemm g;
+  g.n_tiles = n_feat / 128;
+  g.nkb = k_dim / 64;
+  g.splits = 0;
+  g.tpc = 0;
+  for (int S = kPersistCluster; S >= 1; S >>= 1) {
+    if (S > g.nkb) continue;
+    if ((g.nkb + S - 1) / S > 8) break;   // more than 128 KB of weights per CTA: too slow
+    if (g.n_tiles <= nc * (kPersistCluster / S)) {
+      g.splits = S;
+      g.tpc = kPersistCluster / S;
+      return g;
+    }
+  }
   return g;
 }
 
@@ -248,11 +274,13 @@ struct vla_expert {
   int np = 0;                    // phases per Euler step
   PersistGemm pg[PH_COUNT] = {};
   int p_max_tiles = 0;
+  int p_cs = 1, p_nclusters = 0, p_G = 0;   // cluster size, clusters, CTAs of the launch
+  int p_max_clusters = 0;                   // clusters of kPersistCluster the device holds
   int *p_done = nullptr, *p_tctr = nullptr;
   float *p_ws = nullptr, *p_ws_att = nullptr, *p_ws_ml = nullptr;
   float *p_rstat_a = nullptr, *p_rstat_b = nullptr;   // [contributor][64]
   float *p_ain_rm = nullptr, *p_st_rm = nullptr;      // embed maps [W][in padded to 4]
-  unsigned long long* p_trace = nullptr;   // [np][G][8] stamps of the first step (diagnostics)
+  unsigned long long* p_trace = nullptr;   // [np][G][16] stamps of the first step (diagnostics)
 
   struct GraphEntry {
     cudaGraph_t g = nullptr;
@@ -342,8 +370,11 @@ int validate(const vla_config* c, const vla_weights* w) {
   if (c->max_steps < 1 || c->max_steps > kMaxSteps)
     return fail(VLA_ERR_SHAPE, "max_steps must be in [1, %d]", kMaxSteps);
   if (!(c->eps > 0.0f)) return fail(VLA_ERR_ARG, "eps must be > 0");
-  if (c->flags & ~(VLA_FLAG_NO_PDL | VLA_FLAG_NORM_KERNELS | VLA_FLAG_NO_PERSIST | VLA_FLAG_FP8_WEIGHTS))
+  if (c->flags & ~(VLA_FLAG_NO_PDL | VLA_FLAG_NORM_KERNELS | VLA_FLAG_NO_PERSIST | VLA_FLAG_FP8_WEIGHTS |
+                   VLA_FLAG_PERSIST))
     return fail(VLA_ERR_ARG, "unknown flag bits 0x%x", c->flags);
+  if ((c->flags & VLA_FLAG_PERSIST) && (c->flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS)))
+    return fail(VLA_ERR_ARG, "VLA_FLAG_PERSIST contradicts VLA_FLAG_NO_PERSIST / VLA_FLAG_NORM_KERNELS");
   if ((c->flags & VLA_FLAG_FP8_WEIGHTS) && (c->flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS)))
     return fail(VLA_ERR_UNSUPPORTED, "FP8 weights run on the persistent one-tile path only");
   if ((c->flags & VLA_FLAG_FP8_WEIGHTS) &&
@@ -771,14 +802,15 @@ int make_act_maps(vla_expert* h, int B, ActMaps* am) {
 }
 
 bool use_persist(const vla_expert* h, int B) {
-  return h->persist_ok && B <= h->persist_bmax &&
-         !(h->cfg.flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS));
+  return h->persist_ok && B <= h->persist_bmax && (h->fp8 || (h->cfg.flags & VLA_FLAG_PERSIST));
 }
 
 void persist_params(const vla_expert* h, int B, int steps, int slot, PersistParams* pp) {
   PersistParams& P = *pp;
   P = PersistParams{};
-  P.G = h->sm_count;
+  P.G = h->p_G;
+  P.cs = h->p_cs;
+  P.nclusters = h->p_nclusters;
   P.fp8 = h->fp8 ? 1 : 0;
   P.sc_qkv = h->sc_qkv; P.sc_o = h->sc_o; P.sc_gu = h->sc_gu; P.sc_down = h->sc_down;
   P.L = h->L; P.W = h->W; P.H = h->H; P.D = h->D; P.F = h->F; P.A = h->A; P.C = h->C; P.S = h->S;
@@ -794,11 +826,18 @@ void persist_params(const vla_expert* h, int B, int steps, int slot, PersistPara
   const int key_tiles = cdiv(h->cfg.n_static_max, kt) + cdiv(h->cfg.n_sliding, kt) + cdiv(h->S, kt);
   // at most 24 splits: an owner's merge input (splits x owned rows x (D + 4) fp32) fits the
   // kernel's 96 KB work area for every head_dim up to 256
-  P.att_splits = std::max(1, std::min(std::min(key_tiles, 24), h->sm_count / (B * P.att_qtiles)));
+  P.att_splits = std::max(1, std::min(std::min(key_tiles, 24), P.G / (B * P.att_qtiles)));
+  // with clusters, one cluster per query tile and its ranks as the key splits (merged in
+  // distributed shared memory), when the query tiles fit the clusters
+  P.att_cluster = 0;
+  if (h->p_cs == kPersistCluster && B * P.att_qtiles <= h->p_nclusters) {
+    P.att_cluster = 1;
+    P.att_splits = kPersistCluster;
+  }
   // feature groups per EMBED row and action groups per FINAL row: spread the rows over
-  // the SMs (at most 8 groups; every group at least one feature / action)
-  P.embed_splits = std::max(1, std::min(std::min(8, h->W / 128), h->sm_count / (B * h->S)));
-  P.final_splits = std::max(1, std::min(std::min(8, h->A), h->sm_count / (B * h->C)));
+  // the CTAs (at most 8 groups; every group at least one feature / action)
+  P.embed_splits = std::max(1, std::min(std::min(8, h->W / 128), P.G / (B * h->S)));
+  P.final_splits = std::max(1, std::min(std::min(8, h->A), P.G / (B * h->C)));
   P.tbl = h->tables[slot];
   P.table_stride = h->table_stride;
   P.ctbl = h->ada ? h->ctables[slot] : nullptr;
@@ -826,8 +865,8 @@ int enqueue_persist(vla_expert* h, int B, int steps, int slot, const ActMaps& am
   m.hb = am.hb; m.ob = am.ob; m.ub = am.ub; m.eb = am.eb; m.h1b = am.h1b;
   m.qa = h->tm_qa; m.ka = h->tm_ka; m.va = h->tm_va;
   const size_t phases = static_cast<size_t>(steps) * h->np;
-  CU(cudaMemsetAsync(h->p_done, 0, phases * sizeof(int), s));
-  CU(cudaMemsetAsync(h->p_tctr, 0, phases * h->p_max_tiles * sizeof(int), s));
+  CU(cudaMemsetAsync(h->p_done, 0, phases * 2 * sizeof(int), s));
+  CU(cudaMemsetAsync(h->p_tctr, 0, phases * h->p_max_tiles * 2 * sizeof(int), s));
   CU(launch_denoise_persist(h->D, m, P, s));
   return VLA_OK;
 }
@@ -1111,22 +1150,54 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
 
   // ---- persistent whole-denoise kernel (batches whose suffix tokens fit one 64-token tile)
   h->persist_bmax = std::min(cfg->max_batch, 64 / h->S);
-  if (h->persist_bmax >= 1) {
+  int max_clusters = 0;
+  const bool want_persist = h->fp8 || (cfg->flags & VLA_FLAG_PERSIST);
+  if (h->persist_bmax >= 1 && want_persist) {
     int per_sm = 0;
-    CU(configure_denoise_persist(D, &per_sm));
+    CU(configure_denoise_persist(D, &per_sm, kPersistCluster, &max_clusters));
     h->persist_ok = per_sm >= 1;
   }
   if (h->persist_ok) {
-    const int G = h->sm_count;
+    h->p_max_clusters = max_clusters;
     h->np = 2 + 2 * (h->pi0 ? 1 : 0) + 5 * L;
-    h->pg[PH_QKV] = persist_plan(h->qkv_rows, W, G);
-    h->pg[PH_O] = persist_plan(W, h->HD, G);
-    h->pg[PH_GU] = persist_plan(2 * F, W, G);
-    h->pg[PH_DOWN] = persist_plan(W, F, G);
-    if (h->pi0) {
-      h->pg[PH_TMLP1] = persist_plan(W, W, G);
-      h->pg[PH_TMLP2] = persist_plan(W, W, G);
+    // Clusters of kPersistCluster CTAs (the projection splits of a tile then sum through
+    // distributed shared memory) when the device holds enough of them and every projection
+    // fits one round; otherwise one CTA per SM with the splits summed through global memory.
+    // VLA_PERSIST_CLUSTER=1 forces the latter (diagnostics).
+    const char* env = getenv("VLA_PERSIST_CLUSTER");
+    const bool want = !(env && atoi(env) == 1);
+    h->p_cs = 1;
+    if (want && max_clusters * kPersistCluster >= (h->sm_count * 3) / 4) {
+      // each projection sums its splits through DSMEM when its tiles fit one round of the
+      // clusters, else through global memory over all CTAs of the launch
+      const int nc = max_clusters, G = nc * kPersistCluster;
+      h->p_cs = kPersistCluster;
+      h->p_nclusters = nc;
+      h->p_G = G;
+      auto pick = [&](int n_feat, int k_dim) {
+        PersistGemm c = persist_plan_cluster(n_feat, k_dim, nc);
+        return c.splits ? c : persist_plan(n_feat, k_dim, G);
+      };
+      h->pg[PH_QKV] = pick(h->qkv_rows, W);
+      h->pg[PH_O] = pick(W, h->HD);
+      h->pg[PH_GU] = pick(2 * F, W);
+      h->pg[PH_DOWN] = pick(W, F);
+      if (h->pi0) h->pg[PH_TMLP1] = h->pg[PH_TMLP2] = pick(W, W);
     }
+    if (h->p_cs == 1) {
+      const int G = h->sm_count;
+      h->p_G = G;
+      h->p_nclusters = 0;
+      h->pg[PH_QKV] = persist_plan(h->qkv_rows, W, G);
+      h->pg[PH_O] = persist_plan(W, h->HD, G);
+      h->pg[PH_GU] = persist_plan(2 * F, W, G);
+      h->pg[PH_DOWN] = persist_plan(W, F, G);
+      if (h->pi0) {
+        h->pg[PH_TMLP1] = persist_plan(W, W, G);
+        h->pg[PH_TMLP2] = persist_plan(W, W, G);
+      }
+    }
+    const int G = h->p_G;
     const int qtiles = cdiv(static_cast<long>(h->S) * H, attn_q_tile());
     int items = 0, tiles = h->persist_bmax * qtiles;
     for (int k = 0; k < PH_COUNT; ++k) {
@@ -1136,18 +1207,19 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     h->p_max_tiles = tiles;
     const size_t att_slots = static_cast<size_t>(std::max(G, h->persist_bmax * qtiles));
     const size_t phases = static_cast<size_t>(cfg->max_steps) * h->np;
-    if ((rc = dalloc(h, &h->p_done, phases))) return cleanup(rc);
-    if ((rc = dalloc(h, &h->p_tctr, phases * tiles))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_done, phases * 2))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_tctr, phases * tiles * 2))) return cleanup(rc);
     if ((rc = dalloc(h, &h->p_ws, static_cast<size_t>(items) * 128 * 64))) return cleanup(rc);
     if ((rc = dalloc(h, &h->p_ws_att, att_slots * attn_q_tile() * D))) return cleanup(rc);
     if ((rc = dalloc(h, &h->p_ws_ml, att_slots * attn_q_tile() * 4))) return cleanup(rc);
     // contributor rows: at most one per (tile, split) item, plus the embed feature groups
-    if ((rc = dalloc(h, &h->p_rstat_a, static_cast<size_t>(G + 16) * 64))) return cleanup(rc);
-    if ((rc = dalloc(h, &h->p_rstat_b, static_cast<size_t>(G + 16) * 64))) return cleanup(rc);
+    const size_t contrib_rows = static_cast<size_t>(std::max(G, items)) + 16;
+    if ((rc = dalloc(h, &h->p_rstat_a, contrib_rows * 64))) return cleanup(rc);
+    if ((rc = dalloc(h, &h->p_rstat_b, contrib_rows * 64))) return cleanup(rc);
     if ((rc = upload_f32_rowpad(h, &h->p_ain_rm, w->action_in_w, W, h->A))) return cleanup(rc);
     if (h->hs && (rc = upload_f32_rowpad(h, &h->p_st_rm, w->state_in_w, W, h->Sd))) return cleanup(rc);
     if (getenv("VLA_TRACE_FILE") &&
-        (rc = dalloc(h, &h->p_trace, static_cast<size_t>(h->np) * G * 8)))
+        (rc = dalloc(h, &h->p_trace, static_cast<size_t>(h->np) * G * 16)))
       return cleanup(rc);
   }
   if (h->fp8 && !(h->persist_ok && h->persist_bmax >= cfg->max_batch))
@@ -1236,12 +1308,14 @@ void vla_expert_destroy(vla_expert* h) {
     }
   }
   if (h->p_trace && !h->trace_file.empty()) {
-    const size_t n = static_cast<size_t>(h->np) * h->sm_count * 8;
+    const size_t G = static_cast<size_t>(h->p_G);
+    const size_t n = static_cast<size_t>(h->np) * G * 16;
     std::vector<unsigned long long> t(n);
     if (cudaMemcpy(t.data(), h->p_trace, n * 8, cudaMemcpyDeviceToHost) == cudaSuccess) {
       if (FILE* f = fopen(h->trace_file.c_str(), "a")) {
+        fprintf(f, "persist_config,%d,%d,%d\n", h->p_G, h->p_cs, h->p_nclusters);
         for (size_t i = 0; i < n; ++i)
-          if (t[i]) fprintf(f, "persist,%zu,%zu,%zu,%llu\n", i / (8 * h->sm_count), (i / 8) % h->sm_count, i % 8, t[i]);
+          if (t[i]) fprintf(f, "persist,%zu,%zu,%zu,%llu\n", i / (16 * G), (i / 16) % G, i % 16, t[i]);
         fclose(f);
       }
     }
@@ -1375,6 +1449,15 @@ int vla_device_status(vla_expert* h, void* cuda_stream) {
     cudaDeviceSynchronize();
     return fail(VLA_ERR_TIMEOUT, "a kernel wait timed out (device status %d); the status word was cleared", v);
   }
+  return VLA_OK;
+}
+
+int vla_persist_info(vla_expert* h, int* ctas, int* cluster, int* max_clusters) {
+  g_err.clear();
+  if (!h) return fail(VLA_ERR_ARG, "null handle");
+  if (ctas) *ctas = h->persist_ok ? h->p_G : 0;
+  if (cluster) *cluster = h->p_cs;
+  if (max_clusters) *max_clusters = h->p_max_clusters;
   return VLA_OK;
 }
 

@@ -57,6 +57,8 @@ constexpr int A_BYTES = 128 * 64 * 2;
 constexpr int B_BYTES = 64 * 64 * 2;
 constexpr int TN = 64;                // token tile (MMA N)
 constexpr int kTmemCols = 128;        // two 64-column fp32 accumulators
+constexpr int kL2Ahead = 0;           // weight tiles prefetched into L2 beyond the ring (0: off;
+                                      // measured: 16 made the denoise slower)
 // Work area shared by the phases, never by two at once: the attention operands (Q, two
 // K/V stages) in ATT phases; in projection phases the partials of the owned feature
 // pairs (first half) and the per-token sum-of-squares rows (second half); the weight
@@ -64,6 +66,9 @@ constexpr int kTmemCols = 128;        // two 64-column fp32 accumulators
 constexpr int kArea = 96 * 1024;
 constexpr int kAreaHalf = kArea / 2;
 constexpr int kMergeW = 128;          // attention merge weights (owned rows x splits)
+// Cluster-mode attention record of one query row: D bf16 (o / l) then (m, l, 0, 0) fp32.
+template <int D>
+constexpr int kAttRec = D * 2 + 16;
 
 template <int D>
 struct PCfg {
@@ -83,7 +88,7 @@ enum : int {
   BAR_AFULL = 0, BAR_AEMPTY = BAR_AFULL + NA, BAR_BFULL = BAR_AEMPTY + NA, BAR_BEMPTY = BAR_BFULL + NB,
   BAR_ACCFULL = BAR_BEMPTY + NB, BAR_ACCEMPTY = BAR_ACCFULL + 2, BAR_QFULL = BAR_ACCEMPTY + 2,
   BAR_KVFULL = BAR_QFULL + 1, BAR_DRAIN = BAR_KVFULL + 2, BAR_STAGE = BAR_DRAIN + 1, BAR_A8FULL = BAR_STAGE + 1,
-  BAR_COUNT = BAR_A8FULL + NA
+  BAR_RECV = BAR_A8FULL + NA, BAR_COUNT = BAR_RECV + 1
 };
 static_assert(BAR_COUNT * 8 <= 512, "barrier area");
 
@@ -101,8 +106,34 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
-// Spin until *ctr >= target (acquire). Gives up (false) after the wait limit, reporting
-// a timeout, or as soon as the status word shows another wait gave up.
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Inter-CTA barriers are arrival counters: each participant, after its writes, fences and
+// adds 1; waiters poll the count.
+__device__ __forceinline__ void barrier_arrive(int* ctr, int) {
+  __threadfence();
+  atomicAdd(ctr, 1);
+}
+
+// Spin until *ctr >= target (acquire loads). Gives up (false) after
+// the wait limit, reporting a timeout, or as soon as the status word shows another wait
+// gave up.
 __device__ __forceinline__ bool wait_counter(const int* ctr, int target, int* err) {
   if (ld_acquire(ctr) >= target) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -118,13 +149,28 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, int* er
   }
 }
 
+// try_wait that suspends the thread until the phase completes or about 20 us pass,
+// instead of returning at once: the waiting warp stops taking issue slots from the warps
+// that work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+
 // mbarrier wait that also gives up when the status word is set.
 __device__ __forceinline__ bool mbar_wait_ab(uint32_t bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (int it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255) == 255) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((it & 7) == 7) {
       if (ld_volatile(err)) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         report(err, kDevTimeout);
@@ -137,9 +183,11 @@ __device__ __forceinline__ bool mbar_wait_ab(uint32_t bar, uint32_t parity, int*
 // Optional timeline of the first Euler step (diagnostics only): slot k of (phase, CTA):
 // 0 epilogue starts the phase, 1 dependency seen by the epilogue, 2 accumulator (or Q)
 // ready, 3 partial written and counted, 4 all partials of the tile in, 5 item done,
-// 6 dependency seen by the activation producer, 7 accumulator committed by the MMA warp.
+// 6 dependency seen by the activation producer, 7 accumulator committed by the MMA warp,
+// 8 partial staged, 9 partial rows sent, 10 owner epilogue starts, 11 owner epilogue ends,
+// 12 rinv ready, 13 residual prefetch issued.
 __device__ __forceinline__ void pstamp(const PersistParams& P, int gph, int slot) {
-  if (P.trace && gph < P.np) P.trace[(static_cast<size_t>(gph) * gridDim.x + blockIdx.x) * 8 + slot] = globaltimer_ns();
+  if (P.trace && gph < P.np) P.trace[(static_cast<size_t>(gph) * gridDim.x + blockIdx.x) * 16 + slot] = globaltimer_ns();
 }
 
 // Two E4M3 bytes -> two bf16 (exact: every E4M3 value is a bf16 value), through the
@@ -210,6 +258,11 @@ __device__ __forceinline__ PhaseId decode_phase(const PersistParams& P, int i) {
 
 __device__ __forceinline__ bool is_gemm(int kind) {
   return kind == PH_TMLP1 || kind == PH_TMLP2 || kind == PH_QKV || kind == PH_O || kind == PH_GU || kind == PH_DOWN;
+}
+
+// FP8 weights cover the four per-layer projections; the Pi0 action-time MLP stays bf16.
+__device__ __forceinline__ bool fp8_kind(const PersistParams& P, int kind) {
+  return P.fp8 && (kind == PH_QKV || kind == PH_O || kind == PH_GU || kind == PH_DOWN);
 }
 
 __device__ __forceinline__ int n_items(const PersistParams& P, int kind) {
@@ -296,74 +349,190 @@ __device__ __forceinline__ void split_range(int nkb, int S, int s, int& kb0, int
   kb1 = ((s + 1) * nkb) / S;
 }
 
+// The round-th projection item of this CTA (false when it has no more). Without cluster
+// splits (no clusters, or tpc = 0 for this projection) item i = cta + round * G is (tile
+// i % n_tiles, split i / n_tiles). With cluster splits the splits of a tile are the
+// consecutive ranks of one cluster of cs CTAs: rank r is split r % S of the tile slot
+// r / S, and cluster c takes tile slots (round * nclusters + c) * tpc + r / S.
+__device__ __forceinline__ bool gemm_item(const PersistParams& P, const PersistGemm& pg, int round, int& tile,
+                                          int& split) {
+  if (P.cs <= 1 || pg.tpc == 0) {
+    const int it = blockIdx.x + round * gridDim.x;
+    tile = it % pg.n_tiles;
+    split = it / pg.n_tiles;
+    return it < pg.n_tiles * pg.splits;
+  }
+  const int c = blockIdx.x / P.cs, r = blockIdx.x % P.cs;
+  if (r / pg.splits >= pg.tpc) return false;
+  tile = (round * P.nclusters + c) * pg.tpc + r / pg.splits;
+  split = r % pg.splits;
+  return tile < pg.n_tiles;
+}
+
+// Walks this CTA's projection weight tiles in the order the ring consumes them (every
+// projection phase of every Euler step, its items, their K blocks).
+struct WeightCursor {
+  int gph = -1, rd = 0, kb = 0, kb1 = 0, tile = 0, split = 0, w_row0 = 0, kind = 0;
+  bool done = false;
+  __device__ __forceinline__ bool item(const PersistParams& P) {
+    const PersistGemm& pg = P.g[kind];
+    if (!gemm_item(P, pg, rd, tile, split)) return false;
+    int kb0;
+    split_range(pg.nkb, pg.splits, split, kb0, kb1);
+    kb = kb0;
+    return true;
+  }
+  // Advances to the next tile; false once the work list is exhausted.
+  __device__ __forceinline__ bool next(const PersistParams& P, int nph) {
+    if (done) return false;
+    if (gph >= 0 && ++kb < kb1) return true;
+    if (gph >= 0) {
+      ++rd;
+      if (item(P)) return true;
+    }
+    for (++gph; gph < nph; ++gph) {
+      const int k = gph / P.np;
+      const PhaseId ph = decode_phase(P, gph - k * P.np);
+      if (!is_gemm(ph.kind)) continue;
+      kind = ph.kind;
+      rd = 0;
+      w_row0 = kind == PH_QKV ? ph.layer * P.qkv_rows
+             : kind == PH_GU  ? ph.layer * 2 * P.F
+             : (kind == PH_O || kind == PH_DOWN) ? ph.layer * P.W : 0;
+      if (item(P)) return true;
+    }
+    done = true;
+    return false;
+  }
+};
+
+__device__ __forceinline__ const CUtensorMap* weight_map(const PersistMaps& maps, int kind) {
+  switch (kind) {
+    case PH_QKV: return &maps.wqkv;
+    case PH_O: return &maps.wo;
+    case PH_GU: return &maps.wgu;
+    case PH_DOWN: return &maps.wdown;
+    case PH_TMLP1: return &maps.w1a;
+    default: return &maps.w2;
+  }
+}
+
 // ------------------------------------------------------------------ epilogue helpers
 
 // Owner of feature pair pr (or row pr) when n pairs are split S ways as [s*n/S, (s+1)*n/S).
 __device__ __forceinline__ int owner_of(int pr, int S, int n) { return ((pr + 1) * S - 1) / n; }
 
-// Projection partials are laid out so that everything an owner sums is contiguous:
-// [tile][owner o][split s][row of o][64 tokens] fp32 (o owns rows 2*p0(o) .. 2*p1(o)).
-__device__ __forceinline__ size_t part_offset(int tile, int S, int o, int s, int lr) {
-  const int p0 = (o * 64) / S, rows = 2 * (((o + 1) * 64) / S - p0);
-  return (static_cast<size_t>(tile) * S * 128 + static_cast<size_t>(2 * p0) * S + static_cast<size_t>(s) * rows + lr) * TN;
+// Projection partials are laid out so that everything an owner sums is contiguous, token
+// by token: [tile][owner o][split s][token (64)][row of o] fp32 (o owns rows 2*p0(o) ..
+// 2*p1(o)). Base of owner o's block:
+__device__ __forceinline__ size_t part_base(int tile, int S, int o) {
+  const int p0 = (o * 64) / S;
+  return (static_cast<size_t>(tile) * S * 128 + static_cast<size_t>(2 * p0) * S) * TN;
 }
 
-// Owner reduction of one projection tile from the partials staged in shared memory
-// (st = [split][owned rows][64]): sums the S partials of the feature pairs [p0, p1) in
-// split order and applies the phase's epilogue. 128 threads: token m = t % 64, pair group
-// t / 64 (pairs p0 + pg, p0 + pg + 2, ...). For residual writers the per-token sum of
-// squares of the pairs written here is one contributor row.
-__device__ void owner_epilogue(const GemmParams& p, int epi, const float* st, int S, int tile, int p0, int p1,
-                               int contrib, const float* s_rinv, float* s_red) {
+// Items of an owner's epilogue: thread t takes feature pair p0 + t % npp of tokens
+// t / npp, t / npp + tpp, ... (tpp = 128 / npp tokens per pass), so that neighbouring
+// threads touch neighbouring features of one token row (coalesced stores), and read the
+// staged partials ([split][token][owned rows]) without bank conflicts.
+struct OwnerMap {
+  int npp, tpp, pl, m0;
+  bool active;
+  __device__ __forceinline__ OwnerMap(int p0, int p1, int t) {
+    npp = p1 - p0;
+    tpp = kEpiThreads / npp;
+    pl = t % npp;
+    m0 = t / npp;
+    active = m0 < tpp;
+  }
+};
+
+// Residual writers: the old residual of the first items, loaded before the tile's partials
+// are complete (it was written two phases earlier).
+constexpr int kPre = 4;
+struct ResidPre {
+  float2 v[kPre];
+};
+
+__device__ __forceinline__ void prefetch_resid(const GemmParams& p, int epi, int tile, int p0, const OwnerMap& om,
+                                               ResidPre& pre) {
+  if (epi != EPI_RESID || !om.active) return;
+  const int fn0 = tile * 128 + 2 * (p0 + om.pl);
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    const int m = om.m0 + k * om.tpp;
+    pre.v[k] = m < p.m_tok ? __ldcg(reinterpret_cast<const float2*>(p.resid + static_cast<size_t>(m) * p.ld_resid + fn0))
+                           : make_float2(0.0f, 0.0f);
+  }
+}
+
+// Owner reduction of one projection tile from the partials in shared memory (each
+// [tokens][rows]: split slots split_stride floats apart in st, and with clusters this CTA's
+// own split at own_st): sums the S partials of the feature pairs [p0, p1) in split order
+// and applies the phase's epilogue. For residual writers the per-token sum of
+// squares of the pairs written here is one contributor row (summed in pair order through
+// the shared tile s_ss [64][npp]).
+__device__ void owner_epilogue(const GemmParams& p, int epi, const float* st, int split_stride, int own,
+                               const float* own_st, int S, int tile, int p0, int p1, int contrib, const float* s_rinv,
+                               float* s_ss, const ResidPre& pre) {
   const int t = threadIdx.x - kEpiWarp0 * 32;
-  const int m = t & 63, pg = t >> 6;
-  const bool valid = m < p.m_tok;
+  const OwnerMap om(p0, p1, t);
+  const int rows = 2 * om.npp;
   const bool resid_w = epi == EPI_RESID || epi == EPI_BIAS_STORE;
   const bool folded = p.rstat_in != nullptr;
-  const float rv = folded && valid ? s_rinv[m] : 1.0f;
-  const int rows = 2 * (p1 - p0);
-  float ss = 0.0f;
-  if (valid) {
-    for (int pr = p0 + pg; pr < p1; pr += 2) {
-      const float* src = st + 2 * (pr - p0) * TN + m;
+  const int fn0 = tile * 128 + 2 * (p0 + om.pl);
+  // per-feature operands
+  float2 g2 = make_float2(1.0f, 1.0f), zm2 = make_float2(0.0f, 0.0f), cv2 = make_float2(0.0f, 0.0f);
+  float2 sc2 = make_float2(1.0f, 1.0f);
+  if (om.active) {
+    if (p.wscale) sc2 = *reinterpret_cast<const float2*>(p.wscale + fn0);
+    if (resid_w) {
+      if (p.vec) g2 = *reinterpret_cast<const float2*>(p.vec + fn0);
+      if (p.zout) zm2 = *reinterpret_cast<const float2*>(p.zmod + fn0);
+    } else if (folded && p.cvec) {
+      cv2 = *reinterpret_cast<const float2*>(p.cvec + fn0);
+    }
+  }
+  if (om.active) {
+    for (int k = 0, m = om.m0; m < p.m_tok; ++k, m += om.tpp) {
+      const int e = m * rows + 2 * om.pl;
       float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll 6
+#pragma unroll 4
       for (int sp = 0; sp < S; ++sp) {
-        v0 += src[sp * rows * TN];
-        v1 += src[sp * rows * TN + TN];
+        // split sp's partial: this CTA's own (cluster mode) or slot sp of the staged ones
+        const float* src = sp == own ? own_st : st + (own < 0 || sp < own ? sp : sp - 1) * split_stride;
+        const float2 a = *reinterpret_cast<const float2*>(src + e);
+        v0 += a.x;
+        v1 += a.y;
       }
-      const int fn0 = tile * 128 + 2 * pr;
-      if (p.wscale) {   // FP8 weights: the MMA used the unscaled E4M3 values
-        v0 *= p.wscale[fn0];
-        v1 *= p.wscale[fn0 + 1];
-      }
+      v0 *= sc2.x;   // FP8 weights: the MMA used the unscaled E4M3 values
+      v1 *= sc2.y;
       if (resid_w) {
         const size_t off = static_cast<size_t>(m) * p.ld_resid + fn0;
         float2 r;
         bool wrote = true;
         if (epi == EPI_RESID) {
-          const float g0 = p.vec ? p.vec[fn0] : 1.0f, g1 = p.vec ? p.vec[fn0 + 1] : 1.0f;
-          const float2 old = __ldcg(reinterpret_cast<const float2*>(p.resid + off));
-          r = make_float2(fmaf(g0, v0, old.x), fmaf(g1, v1, old.y));
+          const float2 old = k < kPre ? pre.v[k < kPre ? k : 0]
+                                      : __ldcg(reinterpret_cast<const float2*>(p.resid + off));
+          r = make_float2(fmaf(g2.x, v0, old.x), fmaf(g2.y, v1, old.y));
           *reinterpret_cast<float2*>(p.resid + off) = r;
         } else {
           wrote = !(p.has_state && (m % p.seq) == 0);
           r = make_float2(v0 + p.vec[fn0], v1 + p.vec[fn0 + 1]);
           if (wrote) *reinterpret_cast<float2*>(p.resid + off) = r;
         }
+        float ss = 0.0f;
         if (wrote) {
-          ss += r.x * r.x + r.y * r.y;
-          if (p.zout) {
-            const float2 zm = *reinterpret_cast<const float2*>(p.zmod + fn0);
+          ss = r.x * r.x + r.y * r.y;
+          if (p.zout)
             *reinterpret_cast<__nv_bfloat162*>(p.zout + off) =
-                __floats2bfloat162_rn(r.x * (1.0f + zm.x), r.y * (1.0f + zm.y));
-          }
+                __floats2bfloat162_rn(r.x * (1.0f + zm2.x), r.y * (1.0f + zm2.y));
         }
+        if (p.rstat_out) s_ss[m * om.npp + om.pl] = ss;
       } else {
         if (folded) {
-          const float2 cv = p.cvec ? *reinterpret_cast<const float2*>(p.cvec + fn0) : make_float2(0.0f, 0.0f);
-          v0 = fmaf(rv, v0, cv.x);
-          v1 = fmaf(rv, v1, cv.y);
+          const float rv = s_rinv[m];
+          v0 = fmaf(rv, v0, cv2.x);
+          v1 = fmaf(rv, v1, cv2.y);
         }
         switch (epi) {
           case EPI_QKV: epi_pair<EPI_QKV>(p, fn0, m, v0, v1); break;
@@ -374,11 +543,13 @@ __device__ void owner_epilogue(const GemmParams& p, int epi, const float* st, in
       }
     }
   }
-  (void)rows;
   if (resid_w && p.rstat_out) {
-    if (pg == 1) s_red[m] = ss;
     named_bar_sync(kBarEpi, kEpiThreads);
-    if (pg == 0 && valid) p.rstat_out[static_cast<size_t>(p.rstat_slot0 + contrib) * TN + m] = ss + s_red[m];
+    if (t < p.m_tok) {
+      float ss = 0.0f;
+      for (int q = 0; q < om.npp; ++q) ss += s_ss[t * om.npp + q];
+      p.rstat_out[static_cast<size_t>(p.rstat_slot0 + contrib) * TN + t] = ss;
+    }
   }
 }
 
@@ -444,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(B_(BAR_DRAIN), 1);
     mbar_init(B_(BAR_STAGE), 1);
     for (int i = 0; i < NA; ++i) mbar_init(B_(BAR_A8FULL + i), 1);
+    mbar_init(B_(BAR_RECV), 1);
     fence_mbar_init();
     const CUtensorMap* all[14] = {&maps.wqkv, &maps.wo, &maps.wgu, &maps.wdown, &maps.w1a, &maps.w2, &maps.hb,
                                   &maps.ob,   &maps.ub, &maps.eb,  &maps.h1b,   &maps.qa, &maps.ka, &maps.va};
@@ -457,6 +629,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = static_cast<uint32_t>(s_flag[1]);
+  // every receive barrier of the cluster is initialised before any CTA pushes to it
+  if (P.cs > 1) cluster_sync_all();
 
   const int nph = P.steps * P.np;
 
@@ -465,7 +639,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       int g = 0;   // ring position
+      int n8[NA];  // E4M3 loads issued per slot (their barrier completes once per such load)
+      bool last8[NA];
+      for (int i = 0; i < NA; ++i) {
+        n8[i] = 0;
+        last8[i] = false;
+      }
       bool ok = true;
+      // L2 prefetch of the tiles kL2Ahead positions beyond the ring, so that a slot freed by
+      // the MMA refills from L2 rather than HBM and HBM keeps streaming during the waits
+      WeightCursor pf;
+      if (kL2Ahead > 0)
+        for (int i = 0; i < NA + kL2Ahead && pf.next(P, nph); ++i) {
+          if (i >= NA) tma_prefetch_l2_2d(weight_map(maps, pf.kind), pf.kb * 64, pf.w_row0 + pf.tile * 128);
+        }
       for (int gph = 0; gph < nph && ok; ++gph) {
         const int k = gph / P.np;
         const PhaseId ph = decode_phase(P, gph - k * P.np);
@@ -473,23 +660,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const PersistGemm& pg = P.g[ph.kind];
         GemmPhase gp;
         gemm_phase(P, maps, ph.kind, ph.layer, k, gp);
-        for (int it = cta; it < pg.n_tiles * pg.splits && ok; it += Gd) {
-          const int tile = it % pg.n_tiles, split = it / pg.n_tiles;
+        int tile, split;
+        for (int rd = 0; ok && gemm_item(P, pg, rd, tile, split); ++rd) {
           int kb0, kb1;
           split_range(pg.nkb, pg.splits, split, kb0, kb1);
           for (int kb = kb0; kb < kb1; ++kb, ++g) {
             const int s = g % NA;
+            if (kL2Ahead > 0 && pf.next(P, nph))
+              tma_prefetch_l2_2d(weight_map(maps, pf.kind), pf.kb * 64, pf.w_row0 + pf.tile * 128);
             if (g >= NA && !mbar_wait_ab(B_(BAR_AEMPTY + s), ((g / NA) - 1) & 1, err)) {
               ok = false;
               break;
             }
-            if (P.fp8) {   // E4M3 bytes into the upper half of the slot, widened by warp 3
+            if (fp8_kind(P, ph.kind)) {   // E4M3 bytes into the upper half, widened by warp 3
               mbar_arrive_expect_tx(B_(BAR_A8FULL + s), A_BYTES / 2);
               tma_load_2d(smem_u32(sA + s * A_BYTES + A_BYTES / 2), gp.tw, B_(BAR_A8FULL + s), kb * 64,
                           gp.w_row0 + tile * 128, pol);
+              ++n8[s];
+              last8[s] = true;
             } else {
               mbar_arrive_expect_tx(B_(BAR_AFULL + s), A_BYTES);
               tma_load_2d(smem_u32(sA + s * A_BYTES), gp.tw, B_(BAR_AFULL + s), kb * 64, gp.w_row0 + tile * 128, pol);
+              last8[s] = false;
             }
           }
         }
@@ -497,7 +689,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: every issued load has landed before the CTA may exit
       for (int s = 0; s < NA && s < g; ++s) {
         const int last = s + ((g - 1 - s) / NA) * NA;
-        mbar_wait(B_((P.fp8 ? BAR_A8FULL : BAR_AFULL) + s), (last / NA) & 1, nullptr);
+        if (last8[s])
+          mbar_wait(B_(BAR_A8FULL + s), (n8[s] - 1) & 1, nullptr);
+        else
+          mbar_wait(B_(BAR_AFULL + s), (last / NA) & 1, nullptr);
       }
     }
     __syncwarp();
@@ -512,15 +707,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const PhaseId ph = decode_phase(P, gph - k * P.np);
         if (!is_gemm(ph.kind)) continue;
         const PersistGemm& pg = P.g[ph.kind];
-        if (cta >= pg.n_tiles * pg.splits) continue;
-        const PhaseId prev = decode_phase(P, (gph - 1) - ((gph - 1) / P.np) * P.np);
-        if (!wait_counter(P.done + gph - 1, n_items(P, prev.kind), err)) break;
+        int tile, split;
+        if (!gemm_item(P, pg, 0, tile, split)) continue;
+        GemmPhase gp;   // operand maps resolved before the wait: nothing left but the copies
+        gemm_phase(P, maps, ph.kind, ph.layer, k, gp);
+        if (!wait_counter(P.done + 2 * (gph - 1), n_items(P, decode_phase(P, (gph - 1) % P.np).kind), err)) break;
         pstamp(P, gph, 6);
         fence_proxy_async_global();
-        GemmPhase gp;
-        gemm_phase(P, maps, ph.kind, ph.layer, k, gp);
-        for (int it = cta; it < pg.n_tiles * pg.splits && ok; it += Gd) {
-          const int split = it / pg.n_tiles;
+        for (int rd = 0; ok && gemm_item(P, pg, rd, tile, split); ++rd) {
           int kb0, kb1;
           split_range(pg.nkb, pg.splits, split, kb0, kb1);
           for (int kb = kb0; kb < kb1; ++kb, ++g) {
@@ -551,8 +745,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const PhaseId ph = decode_phase(P, gph - k * P.np);
         if (!is_gemm(ph.kind)) continue;
         const PersistGemm& pg = P.g[ph.kind];
-        for (int it = cta; it < pg.n_tiles * pg.splits && ok; it += Gd, ++ai) {
-          const int split = it / pg.n_tiles;
+        int tile, split;
+        for (int rd = 0; ok && gemm_item(P, pg, rd, tile, split); ++rd, ++ai) {
           int kb0, kb1;
           split_range(pg.nkb, pg.splits, split, kb0, kb1);
           const int b = ai & 1;
@@ -590,20 +784,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- FP8 weight widening
     if (P.fp8) {
       int g = 0;
+      int u8[NA];   // E4M3 uses of each slot so far (bf16 tiles of the time MLP pass by)
+      for (int i = 0; i < NA; ++i) u8[i] = 0;
       bool ok = true;
       for (int gph = 0; gph < nph && ok; ++gph) {
         const int k = gph / P.np;
         const PhaseId ph = decode_phase(P, gph - k * P.np);
         if (!is_gemm(ph.kind)) continue;
         const PersistGemm& pg = P.g[ph.kind];
-        for (int it = cta; it < pg.n_tiles * pg.splits && ok; it += Gd) {
-          const int split = it / pg.n_tiles;
+        const bool f8 = fp8_kind(P, ph.kind);
+        int tile, split;
+        for (int rd = 0; ok && gemm_item(P, pg, rd, tile, split); ++rd) {
           int kb0, kb1;
           split_range(pg.nkb, pg.splits, split, kb0, kb1);
+          if (!f8) {
+            g += kb1 - kb0;
+            continue;
+          }
           for (int kb = kb0; kb < kb1; ++kb, ++g) {
             const int s = g % NA;
             int landed = 0;
-            if (lane == 0) landed = mbar_wait_ab(B_(BAR_A8FULL + s), (g / NA) & 1, err) ? 1 : 0;
+            if (lane == 0) landed = mbar_wait_ab(B_(BAR_A8FULL + s), u8[s] & 1, err) ? 1 : 0;
+            ++u8[s];
             landed = __shfl_sync(0xffffffffu, landed, 0);
             if (!landed) {
               ok = false;
@@ -625,6 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ai = 0;                     // accumulator uses
     int nq = 0, kvu0 = 0, kvu1 = 0;  // attention barrier uses
     int nst = 0;                    // staging barrier uses
+    int nrecv = 0;                  // receive barrier uses (cluster mode)
     bool ok = true;
     float* area = reinterpret_cast<float*>(sAtt);
     // uniform wait helpers: thread 0 waits, the verdict is shared through shared memory
@@ -643,12 +846,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r;
     };
     // release this CTA's item of phase gph (all epilogue threads' writes first)
-    auto signal = [&](int* ctr) {
+    // arrive at the inter-CTA barrier bar2 of `target` participants (all epilogue threads'
+    // writes first)
+    auto signal = [&](int* bar2, int target) {
       named_bar_sync(kBarEpi, kEpiThreads);
       if (t == 0) {
-        fence_proxy_async_global();
-        __threadfence();
-        atomicAdd(ctr, 1);
+        fence_proxy_async_all();   // generic writes (global and shared) before later async copies
+        barrier_arrive(bar2, target);
       }
     };
     // Bulk-copies up to two global ranges (written by other CTAs and released to this one
@@ -674,13 +878,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int k = gph / P.np;
       const PhaseId ph = decode_phase(P, gph - k * P.np);
       const int nit = n_items(P, ph.kind);
-      if (cta >= nit) continue;   // no item here (the MMA warp skips it too)
-      if (t == 0) pstamp(P, gph, 0);
-      int prev_target = 0;
-      if (gph > 0) {
-        const int pk = gph - 1 - ((gph - 1) / P.np) * P.np;
-        prev_target = n_items(P, decode_phase(P, pk).kind);
+      if (is_gemm(ph.kind)) {
+        int tl, sp;
+        if (!gemm_item(P, P.g[ph.kind], 0, tl, sp)) continue;   // no item here (nor for the MMA warp)
+      } else if (cta >= nit) {
+        continue;
       }
+      if (t == 0) pstamp(P, gph, 0);
+      const int prev_target = gph > 0 ? n_items(P, decode_phase(P, (gph - 1) % P.np).kind) : 0;
       if (ph.kind == PH_EMBED) {
         // ---------------------------------------------------------------- embed item
         const float* tk = P.tbl + static_cast<long>(k) * P.table_stride;
@@ -688,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int E = P.embed_splits;
         for (int it = cta; it < nit && ok; it += Gd) {
           const int m = it % P.M, e = it / P.M;
-          if (gph > 0 && !all_wait_counter(P.done + gph - 1, prev_target)) {
+          if (gph > 0 && !all_wait_counter(P.done + 2 * (gph - 1), prev_target)) {
             ok = false;
             break;
           }
@@ -737,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) s_red[ew] = ss;
           named_bar_sync(kBarEpi, kEpiThreads);
           if (t == 0) P.rstat_a[e * TN + m] = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
-          signal(P.done + gph);
+          signal(P.done + 2 * gph, nit);
           if (t == 0) pstamp(P, gph, 5);
         }
         continue;
@@ -750,7 +955,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int BC = P.B * P.C;
         for (int it = cta; it < nit && ok; it += Gd) {
           const int bc = it % BC, ag = it / BC;
-          if (!all_wait_counter(P.done + gph - 1, prev_target)) {
+          if (!all_wait_counter(P.done + 2 * (gph - 1), prev_target)) {
             ok = false;
             break;
           }
@@ -800,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
-          signal(P.done + gph);
+          signal(P.done + 2 * gph, nit);
           if (t == 0) pstamp(P, gph, 5);
         }
         continue;
@@ -815,9 +1020,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int H = P.H, R = P.S * H;
         const int per_obs = P.att_qtiles * P.att_splits;
         const int NS = P.att_splits;
-        for (int it = cta; it < nit && ok; it += Gd) {
-          const int b = it / per_obs, rem = it - b * per_obs;
-          const int qt = rem % P.att_qtiles, sp = rem / P.att_qtiles;
+        // cluster mode: cluster c takes query group c, its ranks are the key splits
+        const bool aclus = P.att_cluster != 0;
+        const int it_first = aclus ? ((cta / P.cs) < P.B * P.att_qtiles ? (cta / P.cs) * NS + cta % P.cs : nit) : cta;
+        const int it_step = aclus ? nit : Gd;
+        for (int it = it_first; it < nit && ok; it += it_step) {
+          int b, qt, sp;
+          if (aclus) {
+            b = (it / NS) / P.att_qtiles;
+            qt = (it / NS) % P.att_qtiles;
+            sp = it % NS;
+          } else {
+            b = it / per_obs;
+            const int rem = it - b * per_obs;
+            qt = rem % P.att_qtiles;
+            sp = rem / P.att_qtiles;
+          }
+          if (aclus && t == 0)   // the other splits' rows for this CTA arrive through DSMEM
+            mbar_arrive_expect_tx(B_(BAR_RECV), static_cast<uint32_t>((NS - 1) * (kQT / NS) * kAttRec<D>));
           const int row0 = qt * kQT;
           const CacheDesc cd = *P.cache;
           Segs sg;
@@ -852,7 +1072,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // cached key tiles do not depend on this step: load them before the wait
             for (int tt = t_begin; tt < t_end && tt < t_begin + 2 && tt < ncached; ++tt) issue(tt, policy_evict_last());
           }
-          bool good = all_wait_counter(P.done + gph - 1, prev_target);
+          bool good = all_wait_counter(P.done + 2 * (gph - 1), prev_target);
           if (t == 0) pstamp(P, gph, 1);
           bool q_inflight = false;
           if (t == 0 && good) {
@@ -902,15 +1122,94 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // unnormalised partial O and (m, l) of this split, laid out so that the rows an
-          // owner merges are contiguous: [group][owner o][split][row of o][D] (+ [4] for
-          // (m, l))
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             acc.l_run[h2] += __shfl_xor_sync(0xffffffffu, acc.l_run[h2], 1);
             acc.l_run[h2] += __shfl_xor_sync(0xffffffffu, acc.l_run[h2], 2);
           }
           const int grp = b * P.att_qtiles + qt;
+          if (aclus) {
+            // Each split normalises its rows (o / l, bf16) and sends owner o's rows
+            // [o*64/NS, (o+1)*64/NS) with their (m, l) to o's receive slots (the idle
+            // activation ring) through DSMEM; owners merge the NS splits in order:
+            // o = sum_s w_s (o_s / l_s), w_s = l_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+            constexpr int REC = kAttRec<D>;      // bytes per row: D bf16 + (m, l, 0, 0) fp32
+            const int RO = kQT / NS;             // rows per owner
+            uint8_t* stg = sAtt;                 // own records [owner][row][REC] (area is free now)
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int r = wrow + g8 + 8 * h2;
+              const float inv = acc.l_run[h2] > 0.0f ? 1.0f / acc.l_run[h2] : 0.0f;
+              uint8_t* rec = stg + r * REC;      // owner-major order equals row order here
+#pragma unroll
+              for (int i = 0; i < D / 8; ++i)
+                *reinterpret_cast<__nv_bfloat162*>(rec + (i * 8 + qd * 2) * 2) =
+                    __floats2bfloat162_rn(acc.o[i][2 * h2] * inv, acc.o[i][2 * h2 + 1] * inv);
+              if (qd == 0)
+                *reinterpret_cast<float4*>(rec + D * 2) = make_float4(acc.m_run[h2], acc.l_run[h2], 0.f, 0.f);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarEpi, kEpiThreads);
+            uint8_t* rcv = sB;                   // receive slots [sender slot][RO rows][REC]
+            if (t == 0) {
+              const int rank0 = static_cast<int>(cluster_ctarank()) - sp;
+              const uint32_t bytes = static_cast<uint32_t>(RO * REC);
+              for (int q = 0; q < NS; ++q) {
+                if (q == sp) continue;
+                const uint32_t slot = static_cast<uint32_t>(sp < q ? sp : sp - 1);
+                bulk_copy_to_peer(mapa_shared(smem_u32(rcv) + slot * bytes, rank0 + q),
+                                  smem_u32(stg + q * RO * REC), bytes, mapa_shared(B_(BAR_RECV), rank0 + q));
+              }
+              bulk_commit();
+              pstamp(P, gph, 3);
+            }
+            if (!all_wait_mbar(B_(BAR_RECV), nrecv & 1)) {
+              if (t == 0) bulk_wait_all();
+              ok = false;
+              break;
+            }
+            ++nrecv;
+            if (t == 0) pstamp(P, gph, 4);
+            auto rec_of = [&](int q, int rr) -> const uint8_t* {
+              return q == sp ? stg + (sp * RO + rr) * REC : rcv + ((q < sp ? q : q - 1) * RO + rr) * REC;
+            };
+            for (int rr = t; rr < RO; rr += kEpiThreads) {
+              float M = -INFINITY;
+              for (int q = 0; q < NS; ++q) M = fmaxf(M, reinterpret_cast<const float*>(rec_of(q, rr) + D * 2)[0]);
+              float wsum = 0.0f;
+              for (int q = 0; q < NS; ++q) {
+                const float* ml = reinterpret_cast<const float*>(rec_of(q, rr) + D * 2);
+                const float w = ml[0] == -INFINITY ? 0.0f : ml[1] * exp2_approx(ml[0] - M);
+                s_w[rr * NS + q] = w;
+                wsum += w;
+              }
+              const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+              for (int q = 0; q < NS; ++q) s_w[rr * NS + q] *= inv;
+            }
+            named_bar_sync(kBarEpi, kEpiThreads);
+            constexpr int D2 = D / 2;
+            for (int i = t; i < RO * D2; i += kEpiThreads) {
+              const int rr = i / D2, d = (i % D2) * 2;
+              const int row = row0 + sp * RO + rr;
+              if (row >= R) continue;
+              float2 a2 = make_float2(0.f, 0.f);
+              for (int q = 0; q < NS; ++q) {
+                const float w = s_w[rr * NS + q];
+                const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(rec_of(q, rr) + d * 2));
+                a2.x = fmaf(w, v.x, a2.x);
+                a2.y = fmaf(w, v.y, a2.y);
+              }
+              *reinterpret_cast<__nv_bfloat162*>(P.ob + (static_cast<size_t>(b) * R + row) * D + d) =
+                  __floats2bfloat162_rn(a2.x, a2.y);
+            }
+            if (t == 0) bulk_wait_all();   // own records read out before the area is reused
+            signal(P.done + 2 * gph, nit);
+            if (t == 0) pstamp(P, gph, 5);
+            continue;
+          }
+          // unnormalised partial O and (m, l) of this split, laid out so that the rows an
+          // owner merges are contiguous: [group][owner o][split][row of o][D] (+ [4] for
+          // (m, l))
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int r = wrow + g8 + 8 * h2;
@@ -925,8 +1224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (qd == 0)
               __stcg(reinterpret_cast<float4*>(P.ws_att_ml + slot * 4), make_float4(acc.m_run[h2], acc.l_run[h2], 0.f, 0.f));
           }
-          int* tc = P.tctr + static_cast<size_t>(gph) * P.max_tiles + grp;
-          signal(tc);
+          int* tc = P.tctr + 2 * (static_cast<size_t>(gph) * P.max_tiles + grp);
+          signal(tc, NS);
           if (t == 0) pstamp(P, gph, 3);
           if (!all_wait_counter(tc, NS)) {
             ok = false;
@@ -976,7 +1275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(a4.x, a4.y);
             *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(a4.z, a4.w);
           }
-          signal(P.done + gph);
+          signal(P.done + 2 * gph, nit);
           if (t == 0) pstamp(P, gph, 5);
         }
         continue;
@@ -986,10 +1285,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       GemmPhase gp;
       gemm_phase(P, maps, ph.kind, ph.layer, k, gp);
       const int S = pg.splits;
-      for (int it = cta; it < nit && ok; it += Gd, ++ai) {
-        const int tile = it % pg.n_tiles, split = it / pg.n_tiles;
+      const bool clus = P.cs > 1 && pg.tpc > 0;   // splits meet through DSMEM
+      int tile, split;
+      for (int rd = 0; ok && gemm_item(P, pg, rd, tile, split); ++rd, ++ai) {
         const int bsel = ai & 1;
-        if (!all_wait_counter(P.done + gph - 1, prev_target)) {
+        const int p0 = (split * 64) / S, p1 = ((split + 1) * 64) / S;
+        const int rows = 2 * (p1 - p0);
+        if (clus && S > 1 && t == 0)   // the other splits' rows of this CTA arrive through DSMEM
+          mbar_arrive_expect_tx(B_(BAR_RECV), static_cast<uint32_t>((S - 1) * P.M * rows * 4));
+        if (!all_wait_counter(P.done + 2 * (gph - 1), prev_target)) {
           ok = false;
           break;
         }
@@ -1003,61 +1307,103 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           rinv_from_stage(gp.p, sr, s_rinv, s_red);
+          if (t == 0) pstamp(P, gph, 12);
         }
+        ResidPre pre;
+        prefetch_resid(gp.p, gp.epi, tile, p0, OwnerMap(p0, p1, t), pre);
+        if (t == 0) pstamp(P, gph, 13);
         if (!all_wait_mbar(B_(BAR_ACCFULL + bsel), (ai >> 1) & 1)) {
           ok = false;
           break;
         }
         if (t == 0) pstamp(P, gph, 2);
         tc_fence_after();
-        // partial tile (features x tokens) -> global scratch at its owner's place, valid
-        // token columns only
-        {
-          const int r = ew * 32 + lane;   // TMEM lane = feature row of the tile
-          const uint32_t taddr = tmem + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(bsel * TN);
-          const int o = owner_of(r >> 1, S, 64);
-          const int lr = r - 2 * ((o * 64) / S);
-          float* dst = P.ws + part_offset(tile, S, o, split, lr);
-          const int ncol = (P.M + 15) & ~15;
-          if (ncol > 32) {
+        const int r = ew * 32 + lane;   // TMEM lane = feature row of the tile
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(ew * 32) << 16) + static_cast<uint32_t>(bsel * TN);
+        const int o = owner_of(r >> 1, S, 64);
+        const int p0o = (o * 64) / S, rows_o = 2 * (((o + 1) * 64) / S - p0o);
+        const float* own_st = nullptr;
+        if (clus) {
+          // partial tile -> this CTA's staging (the idle activation ring) as
+          // [owner][token][owned rows], then owner o's block -> o's receive slot for this split
+          float* stg = reinterpret_cast<float*>(sB);
+          float* dst = stg + static_cast<size_t>(o) * TN * rows_o + (r - 2 * p0o);
+          for (int c = 0; c < P.M; c += 32) {
             float v[32];
-            tmem_ld32(taddr, v);
+            tmem_ld32(taddr + c, v);
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              __stcg(reinterpret_cast<float4*>(dst + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
-            tmem_ld32(taddr + 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              if (32 + j < ncol)
-                __stcg(reinterpret_cast<float4*>(dst + 32 + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
-          } else {
-            float v[32];
-            tmem_ld32(taddr, v);
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              if (j < ncol) __stcg(reinterpret_cast<float4*>(dst + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+            for (int j = 0; j < 32; ++j)
+              if (c + j < P.M) dst[(c + j) * rows_o] = v[j];
           }
+          if (t == 0) pstamp(P, gph, 8);
+          tc_fence_before();
+          fence_proxy_async_smem();
+          named_bar_sync(kBarEpi, kEpiThreads);
+          if (t == 0) {
+            pstamp(P, gph, 9);
+            mbar_arrive(B_(BAR_ACCEMPTY + bsel));
+            const int rank0 = static_cast<int>(cluster_ctarank()) - split;   // split 0 of this tile
+            const uint32_t bytes = static_cast<uint32_t>(P.M * rows * 4);   // every owner has `rows` rows
+            for (int q = 0; q < S; ++q) {
+              if (q == split) continue;
+              const uint32_t slot = static_cast<uint32_t>(split < q ? split : split - 1);
+              const uint32_t dst_s = smem_u32(area) + slot * bytes;
+              bulk_copy_to_peer(mapa_shared(dst_s, rank0 + q), smem_u32(stg + static_cast<size_t>(q) * TN * rows), bytes,
+                                mapa_shared(B_(BAR_RECV), rank0 + q));
+            }
+            bulk_commit();
+            pstamp(P, gph, 3);
+          }
+          own_st = stg + static_cast<size_t>(split) * TN * rows;
+          if (S > 1) {
+            if (!all_wait_mbar(B_(BAR_RECV), nrecv & 1)) {
+              if (t == 0) bulk_wait_all();
+              ok = false;
+              break;
+            }
+            ++nrecv;
+          }
+          if (t == 0) pstamp(P, gph, 4);
+          owner_epilogue(gp.p, gp.epi, area, P.M * rows, split, own_st, S, tile, p0, p1, tile * S + split, s_rinv,
+                         area + kAreaHalf / 4, pre);
+          if (t == 0) pstamp(P, gph, 11);
+          if (t == 0) bulk_wait_all();   // the staging is read out before the ring refills
+        } else {
+          // partial tile -> global scratch at its owner's place, token by token (valid token
+          // columns only); neighbouring lanes hold neighbouring rows
+          float* dst = P.ws + part_base(tile, S, o) + static_cast<size_t>(split) * TN * rows_o + (r - 2 * p0o);
+          for (int c = 0; c < P.M; c += 32) {
+            float v[32];
+            tmem_ld32(taddr + c, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < P.M) __stcg(dst + (c + j) * rows_o, v[j]);
+          }
+          if (t == 0) pstamp(P, gph, 8);
+          tc_fence_before();
+          named_bar_sync(kBarEpi, kEpiThreads);
+          if (t == 0) pstamp(P, gph, 9);
+          if (t == 0) mbar_arrive(B_(BAR_ACCEMPTY + bsel));
+          int* tc = P.tctr + 2 * (static_cast<size_t>(gph) * P.max_tiles + tile);
+          signal(tc, S);
+          if (t == 0) pstamp(P, gph, 3);
+          if (!all_wait_counter(tc, S)) {
+            ok = false;
+            break;
+          }
+          if (t == 0) pstamp(P, gph, 4);
+          if (t == 0) fence_proxy_async_global();
+          if (!stage(area, P.ws + part_base(tile, S, split), static_cast<uint32_t>(S * rows * TN * 4), nullptr, nullptr,
+                     0)) {
+            ok = false;
+            break;
+          }
+          if (t == 0) pstamp(P, gph, 10);
+          owner_epilogue(gp.p, gp.epi, area, TN * rows, -1, nullptr, S, tile, p0, p1, tile * S + split, s_rinv,
+                         area + kAreaHalf / 4, pre);
+          if (t == 0) pstamp(P, gph, 11);
         }
-        tc_fence_before();
-        named_bar_sync(kBarEpi, kEpiThreads);
-        if (t == 0) mbar_arrive(B_(BAR_ACCEMPTY + bsel));
-        int* tc = P.tctr + static_cast<size_t>(gph) * P.max_tiles + tile;
-        signal(tc);
-        if (t == 0) pstamp(P, gph, 3);
-        if (!all_wait_counter(tc, S)) {
-          ok = false;
-          break;
-        }
-        if (t == 0) pstamp(P, gph, 4);
-        const int p0 = (split * 64) / S, p1 = ((split + 1) * 64) / S;
-        if (t == 0) fence_proxy_async_global();
-        if (!stage(area, P.ws + part_offset(tile, S, split, 0, 0), static_cast<uint32_t>(S * 2 * (p1 - p0) * TN * 4),
-                   nullptr, nullptr, 0)) {
-          ok = false;
-          break;
-        }
-        owner_epilogue(gp.p, gp.epi, area, S, tile, p0, p1, tile * S + split, s_rinv, s_red);
-        signal(P.done + gph);
+        signal(P.done + 2 * gph, nit);
         if (t == 0) pstamp(P, gph, 5);
       }
     }
@@ -1065,6 +1411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // no CTA leaves while a peer may still push into its shared memory
+  if (P.cs > 1) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -1078,7 +1426,13 @@ static cudaError_t launch_d(const PersistMaps& maps, const PersistParams& p, cud
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = PCfg<D>::SMEM;
   cfg.stream = s;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cs > 1 ? p.cs : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.cs > 1 ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, denoise_persist_kernel<D>, maps, p);
 }
 
@@ -1093,7 +1447,7 @@ cudaError_t launch_denoise_persist(int head_dim, const PersistMaps& maps, const 
 }
 
 template <int D>
-static cudaError_t configure_d(int* per_sm) {
+static cudaError_t configure_d(int* per_sm, int cs, int* max_clusters) {
   cudaError_t e = cudaFuncSetAttribute(denoise_persist_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(PCfg<D>::SMEM));
   if (e == cudaSuccess)
@@ -1101,17 +1455,36 @@ static cudaError_t configure_d(int* per_sm) {
                              cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, denoise_persist_kernel<D>, kThreads, PCfg<D>::SMEM);
+  *max_clusters = 0;
+  if (e == cudaSuccess && cs > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = PCfg<D>::SMEM;
+    cfg.gridDim = dim3(cs, 1, 1);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(max_clusters, denoise_persist_kernel<D>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      *max_clusters = 0;
+    }
+  }
   return e;
 }
 
-// Sets the kernel attributes for head_dim and returns how many CTAs fit on one SM.
-cudaError_t configure_denoise_persist(int head_dim, int* ctas_per_sm) {
+// Sets the kernel attributes for head_dim and returns how many CTAs fit on one SM and how
+// many clusters of cs CTAs can be resident at once.
+cudaError_t configure_denoise_persist(int head_dim, int* ctas_per_sm, int cs, int* max_clusters) {
   *ctas_per_sm = 0;
   switch (head_dim) {
-    case 32: return configure_d<32>(ctas_per_sm);
-    case 64: return configure_d<64>(ctas_per_sm);
-    case 128: return configure_d<128>(ctas_per_sm);
-    case 256: return configure_d<256>(ctas_per_sm);
+    case 32: return configure_d<32>(ctas_per_sm, cs, max_clusters);
+    case 64: return configure_d<64>(ctas_per_sm, cs, max_clusters);
+    case 128: return configure_d<128>(ctas_per_sm, cs, max_clusters);
+    case 256: return configure_d<256>(ctas_per_sm, cs, max_clusters);
     default: return cudaErrorInvalidValue;
   }
 }

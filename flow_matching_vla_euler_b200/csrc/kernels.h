@@ -219,6 +219,7 @@ struct PersistGemm {
   int n_tiles;   // 128-feature weight tiles
   int nkb;       // 64-wide K blocks
   int splits;    // K splits per tile (items = n_tiles * splits)
+  int tpc;       // cluster mode: tiles per cluster and round (cluster size / splits)
 };
 
 struct PersistMaps {
@@ -229,6 +230,8 @@ struct PersistMaps {
 
 struct PersistParams {
   int G;                                        // CTAs (one per SM)
+  int cs, nclusters;                            // thread-block clusters of cs CTAs (cs = 1: none);
+                                                // projection splits then sum through DSMEM
   int fp8;                                      // weights are E4M3 bytes (maps wqkv..wdown)
   const float *sc_qkv, *sc_o, *sc_gu, *sc_down; // FP8: per-row scales in the packed row order
   int L, W, H, D, F, A, C, S, Sd, hs, HD, qkv_rows, kcap, ring_off, dyn_off, max_batch;
@@ -236,6 +239,8 @@ struct PersistParams {
   float eps, dt, scale_log2;
   PersistGemm g[PH_COUNT];                      // projection phases
   int att_qtiles, att_splits;                   // per observation (splits <= 24)
+  int att_cluster;                              // 1: one cluster per query tile, its ranks the
+                                                // key splits (att_splits = cs), merged in DSMEM
   int embed_splits, final_splits;               // feature / action groups per row
   const float* tbl;                             // time tables [steps][...]
   long table_stride;
@@ -251,8 +256,8 @@ struct PersistParams {
   const CacheDesc* cache;
   float *rstat_a, *rstat_b;                     // [contributor][64] sums of squares
   int ld_rstat;
-  int* done;             // [steps * np] items finished per phase (zeroed before launch)
-  int* tctr;             // [steps * np][max_tiles] partials arrived per tile (zeroed)
+  int* done;             // [steps * np][2] per phase: items finished, go flag (zeroed before launch)
+  int* tctr;             // [steps * np][max_tiles][2] per tile: partials arrived, go flag (zeroed)
   int max_tiles;
   float* ws;             // projection partials [tile][owner][split][owned rows][64]
   float* ws_att;         // attention partials [group][owner][split][owned rows][D]
@@ -262,8 +267,9 @@ struct PersistParams {
 };
 
 cudaError_t launch_denoise_persist(int head_dim, const PersistMaps& maps, const PersistParams& p, cudaStream_t s);
-// Sets the kernel attributes and reports how many CTAs of it fit on one SM.
-cudaError_t configure_denoise_persist(int head_dim, int* ctas_per_sm);
+// Sets the kernel attributes and reports how many CTAs of it fit on one SM, and how many
+// clusters of cs CTAs the device can hold at once (0 if none).
+cudaError_t configure_denoise_persist(int head_dim, int* ctas_per_sm, int cs, int* max_clusters);
 
 // Arms an mbarrier nothing arrives on and waits on it for limit_ns, so the wait gives up
 // and records a timeout in *err (failure-path self-test).

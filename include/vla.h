@@ -78,10 +78,10 @@ typedef enum vla_time_kind {
                                     instead of folding them into the projections (cross-check;
                                     larger batches always use norm kernels; implies
                                     VLA_FLAG_NO_PERSIST) */
-#define VLA_FLAG_NO_PERSIST 4u   /* with one token tile, run the denoise as one kernel launch
-                                    per projection / attention / embed / final step (captured
-                                    in a graph) instead of the single persistent kernel that
-                                    runs the whole loop (cross-check) */
+#define VLA_FLAG_NO_PERSIST 4u   /* never run the single persistent kernel: the denoise is
+                                    one kernel launch per projection / attention / embed /
+                                    final step, captured in a graph (the default for bf16
+                                    weights; not combinable with VLA_FLAG_FP8_WEIGHTS) */
 #define VLA_FLAG_FP8_WEIGHTS 8u  /* the projection matrices wq, wk, wv, wo, w_gate, w_up,
                                     w_down are FP8 E4M3 bytes with fp32 per-output-row scales
                                     (vla_weights *_scale); streamed as FP8 and widened to bf16
@@ -89,6 +89,11 @@ typedef enum vla_time_kind {
                                     FP8 configuration). Needs max_batch x suffix <= 64 (the
                                     persistent one-tile path); not combinable with
                                     VLA_FLAG_NO_PERSIST or VLA_FLAG_NORM_KERNELS. */
+#define VLA_FLAG_PERSIST 16u     /* with bf16 weights and one token tile (max_batch x suffix
+                                    <= 64), run the whole denoise loop as the single
+                                    persistent kernel instead of the launch chain (FP8
+                                    weights always use it). Ignored for larger batches;
+                                    not combinable with VLA_FLAG_NO_PERSIST. */
 
 typedef struct vla_config {
   int n_layers;      /* L */
@@ -321,6 +326,16 @@ VLA_API int vla_gemm_bf16_noalloc(const uint16_t* W, const uint16_t* X, float* Y
  * query (that call's Y is then not valid), or VLA_ERR_CUDA. Allocates nothing.
  */
 VLA_API int vla_gemm_status(void* cuda_stream);
+
+/*
+ * vla_persist_info -- launch shape of the persistent whole-denoise kernel that vla_denoise
+ * uses for batches whose suffix tokens fit one 64-token tile (HOST ints, any may be NULL):
+ * *ctas = CTAs of the launch (0 if the kernel is not available on this handle), *cluster =
+ * CTAs per thread-block cluster (1: no clusters; the projection K-splits then meet in global
+ * memory instead of distributed shared memory), *max_clusters = clusters of 8 the device
+ * can hold at once. Errors: VLA_ERR_ARG.
+ */
+VLA_API int vla_persist_info(vla_expert* h, int* ctas, int* cluster, int* max_clusters);
 
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VLA_API const char* vla_last_error(void);

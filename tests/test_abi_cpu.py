@@ -95,9 +95,11 @@ def test_host_argument_checks(lib):
                                  ctypes.byref(h)) == V.VLA_ERR_UNSUPPORTED
     assert lib.vla_expert_create(ctypes.byref(_cfg(time_kind=7)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG
-    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=16)), ctypes.byref(w),
+    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=32)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG
     assert "flag" in V.vla_last_error()
+    assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_PERSIST | V.VLA_FLAG_NO_PERSIST)),
+                                 ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
     # FP8 weights: every scale pointer is required, and only the persistent one-tile path
     assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_FP8_WEIGHTS)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG

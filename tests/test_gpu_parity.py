@@ -146,9 +146,9 @@ def _first_obs(wl, inp, n):
 @pytest.mark.parametrize("name, obs", [("tiny", None), ("mid_d128", None), ("mid_pi0_b3", 1), ("mid_ada_b2", 1),
                                        ("pi0_1view", None), ("pi05_3view", None)])
 def test_persistent_kernel_matches_oracle_and_the_launch_chain(name, obs):
-    """The whole denoise as one persistent kernel (the default for one token tile: D = 32,
+    """The whole denoise as one persistent kernel (VLA_FLAG_PERSIST, one token tile: D = 32,
     64, 128, 256; AdaRMSNorm and Pi0 time MLP with a state token; two observations in one
-    tile) and as the chain of per-step kernel launches (VLA_FLAG_NO_PERSIST), on the same
+    tile) and as the chain of per-step kernel launches (the bf16 default), on the same
     inputs: both within the acceptance tolerance of the oracle and of each other; the
     persistent kernel's result is bit-identical across calls (its split sums run in a
     fixed order)."""
@@ -163,11 +163,12 @@ def test_persistent_kernel_matches_oracle_and_the_launch_chain(name, obs):
         ref = oracle_actions(wl, inp)
     assert wl.batch * wl.expert.suffix_len <= 64
     outs = []
-    for flags in (0, V.VLA_FLAG_NO_PERSIST):
+    for flags in (V.VLA_FLAG_PERSIST, 0):
         ex, _ = make_expert(wl, inp, flags=flags)
+        assert (V.vla_persist_info(ex.handle)["ctas"] > 0) == (flags == V.VLA_FLAG_PERSIST)
         load_prefix(ex, inp)
         outs.append(run(ex, inp, wl.steps))
-        if flags == 0:
+        if flags:
             assert np.array_equal(run(ex, inp, wl.steps), outs[0])
         ex.device_status()
         ex.close()
