@@ -192,6 +192,24 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return VLA_OK;
 }
 
+// fp32 [rows][inner] row-major (the residual stream), boxes of 128 values x 32 rows, no
+// swizzle: [row][128] fp32 in shared memory.
+int make_tmap_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows) {
+  auto enc = get_encode();
+  if (!enc) return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {128, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(VLA_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed (%d) for %llu x %llu", static_cast<int>(r),
+                static_cast<unsigned long long>(rows), static_cast<unsigned long long>(inner));
+  return VLA_OK;
+}
+
 // uint8 [rows][inner] row-major (E4M3 weight bytes), boxes of 64 bytes x box_rows, no
 // swizzle: the persistent kernel widens each row in shared memory itself.
 int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
@@ -261,6 +279,7 @@ struct vla_expert {
   int prefix_batch = 0, n_static = 0, n_ring = 0, head = 0;
 
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
+  CUtensorMap tm_resid;              // fp32 residual [max_M][W], boxes of 128 x 32
   CUtensorMap tm_q, tm_kc, tm_vt;   // tensor-core attention operands (head_dim 256)
   CUtensorMap tm_qa, tm_ka, tm_va;  // split-KV attention operands (any head_dim)
 
@@ -508,6 +527,7 @@ GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
 // Sum-of-squares contributor rows a push-mode residual epilogue (one token tile) writes
 // per token: one per (weight tile, split owner, 32-row group).
 int contributors(const vla_expert* h, int n_feat, int k_dim, int M) {
+  if (M > 64) return n_feat / 128;   // persistent GEMM: one row per 128-feature tile
   const GemmPlan g = denoise_plan(h, n_feat, k_dim, M);
   return g.n_tiles * g.m_tiles * g.splits * (g.splits == 1 ? 2 : 1);
 }
@@ -524,9 +544,12 @@ int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensor
     p.kb_per_split = k_dim / 64;
     p.w_stream = 0;
     p.err = h->err;
+    p.ld_rstat = h->max_M;
     const int total = g0.n_tiles * g0.m_tiles;
     rec.begin(kind);
-    CU(launch_gemm_persistent(g0.tn, epi, tw, tx, p, g0.n_tiles, g0.m_tiles, std::min(total, h->sm_count), rec.s,
+    // the residual map only for the residual stream itself (rows M)
+    const CUtensorMap* tr = (epi == EPI_RESID && p.resid == h->resid) ? &h->tm_resid : nullptr;
+    CU(launch_gemm_persistent(g0.tn, epi, tw, tx, tr, p, g0.n_tiles, g0.m_tiles, std::min(total, h->sm_count), rec.s,
                               pdl));
     return rec.end(kind);
   }
@@ -559,11 +582,9 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
   // tensor-core attention once every 128-row query tile has a CTA of its own
   const bool use_tc_attn = h->vtc && B * cdiv(h->S * h->H, attn_tc_q_tile()) >= h->sm_count;
   const float dt = -1.0f / static_cast<float>(steps);
-  // All suffix tokens in one 64-token tile: the norms are folded into the QKV and gate/up
-  // GEMMs, fed by per-token sum-of-squares partials from the residual writers (unless norm
-  // kernels are asked for). With several token tiles the persistent GEMMs' epilogues are
-  // the bottleneck and separate norm kernels are faster (measured at batch 64).
-  const bool fused = M <= 64 && !(h->cfg.flags & VLA_FLAG_NORM_KERNELS);
+  // The norms are folded into the QKV and gate/up GEMMs, fed by per-token sum-of-squares
+  // partials from the residual writers (unless norm kernels are asked for).
+  const bool fused = !(h->cfg.flags & VLA_FLAG_NORM_KERNELS);
   const long cw = h->qkv_rows + 2L * h->F;
   // modulation the next norm applies to z: AdaRMSNorm (1 + scale_j) or RMSNorm (1 + w)
   auto zmod = [&](const float* tk, int j) -> const float* {
@@ -1251,6 +1272,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
     if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
   }
+  if ((rc = make_tmap_f32(&h->tm_resid, h->resid, W, h->max_M))) return cleanup(rc);
   {
     const uint64_t rows = static_cast<uint64_t>(L) * cfg->max_batch * h->kcap;
     const uint32_t bc = static_cast<uint32_t>(attn_box_cols(D)), kt = static_cast<uint32_t>(attn_key_tile(D));

@@ -612,13 +612,157 @@ struct PersistCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = TN == 256 ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * TN;       // two accumulators
-  static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  // EPI_QKV stages its bf16 output through shared memory: two buffers of 32 token rows
+  // (16 per column half) x QKV_RSTR elements, plus the tile's per-token table
+  static constexpr int QKV_RSTR = 144;           // pair half 0 at [0, 64), half 1 at [80, 144)
+  static constexpr int QKV_STAGE_BYTES = 2 * 32 * QKV_RSTR * 2;
+  static constexpr int QKV_TABLE_BYTES = TN * 8;
+  static constexpr size_t SMEM_BASE = 1024 + STAGES * STAGE_BYTES + 256;
+  // Folded norm (QKV, gate/up): 1 / rms of every token of the launch, computed once per CTA
+  // while its first main loop runs (up to RINV_ALL tokens; beyond that, per tile).
+  static constexpr int RINV_ALL = 3328;
+  static constexpr int RINV_BYTES = RINV_ALL * 4;
+  // residual writers: per-quarter sums of squares of each token, [tile parity][4][TN]
+  static constexpr int SSQ_BYTES = 2 * 4 * TN * 4;
+  // EPI_RESID in a CTA with one tile: the fp32 residual tile moves by bulk copies through
+  // the pipeline stages once the MMAs have consumed them, in sub-tiles of 32 tokens x 128
+  // features ([token][feature], 512 bytes per token)
+  static constexpr int RSUB = 32, RSUB_BYTES = RSUB * BM * 4;
+  static constexpr int RSUB_PER_STAGE = STAGE_BYTES / RSUB_BYTES;
+  static constexpr int NSUB = TN / RSUB;
+  static_assert((NSUB + RSUB_PER_STAGE - 1) / RSUB_PER_STAGE <= STAGES, "residual tile fits the stages");
+  static constexpr size_t smem(int epi) {
+    return SMEM_BASE + (epi == EPI_QKV ? RINV_BYTES + QKV_STAGE_BYTES + QKV_TABLE_BYTES
+                                       : epi == EPI_GEGLU ? RINV_BYTES
+                                       : (epi == EPI_RESID || epi == EPI_BIAS_STORE) ? SSQ_BYTES : 0);
+  }
 };
+
+// Sum over 32 lanes of 16 per-lane values (one per token of a chunk): after halving
+// exchanges with partners 16, 8, 4, 2 and a final one with partner 1, lane l holds the
+// total of token l >> 1 (lanes 2t and 2t + 1 both). Fixed order, 16 shuffles.
+__device__ __forceinline__ float warp_sum16(const float (&x)[16], int lane) {
+  float a[8], b[4], c[2];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const bool hi = lane & 16;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? x[k] : x[k + 8], 16);
+    a[k] = (hi ? x[k + 8] : x[k]) + got;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const bool hi = lane & 8;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? a[k] : a[k + 4], 8);
+    b[k] = (hi ? a[k + 4] : a[k]) + got;
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const bool hi = lane & 4;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? b[k] : b[k + 2], 4);
+    c[k] = (hi ? b[k + 2] : b[k]) + got;
+  }
+  const bool hi = lane & 2;
+  float d = (hi ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, hi ? c[0] : c[1], 2);
+  return d + __shfl_xor_sync(0xffffffffu, d, 1);
+}
+
+// EPI_QKV for several token tiles. The accumulator rows are packed feature pairs (row 2i /
+// 2i + 1 = dims i and i + D/2 of one Q head, of K or of V), so RoPE is one lane-pair
+// shuffle. The rotated bf16 values are staged as [token][dims of the tile] in shared
+// memory -- each tile row pair covers dims i0..i0+63 and i0+D/2..i0+D/2+63 of one region --
+// and leave as 16-byte stores of 8 consecutive dims: Q rows [token][H*D], K / V cache rows
+// [obs][kcap][D]. Token -> (position, cache row) comes from a per-tile table built once.
+template <int TN>
+__device__ __forceinline__ void qkv_epilogue_staged(const GemmParams& p, uint32_t taddr, int n_tile, int m0,
+                                                    int ew, int r, int lane, bf16* stage, int* tok_s,
+                                                    int* tok_kv, const float* s_rinv) {
+  using G = PersistCfg<TN>;
+  constexpr int RSTR = G::QKV_RSTR, STEPS = TN / 32;
+  const int etid = ew * 32 + lane, half = ew >> 2;
+  const int D = p.head_dim, DH = D >> 1, H = p.n_heads;
+  for (int t = etid; t < TN; t += 256) {
+    const int m = min(m0 + t, p.m_tok - 1);
+    const int b = m / p.seq, sq = m - b * p.seq;
+    tok_s[t] = sq;
+    tok_kv[t] = b * p.kcap + p.dyn_off + sq;
+  }
+  named_bar_sync(1, 256);
+  // this lane's feature (tile row r = its TMEM lane): pair pr (kind 0 = Q head, 1 = K,
+  // 2 = V, 3 = padding), element i
+  const int pr = (n_tile * G::BM + r) >> 1, second = r & 1;
+  const int kind = pr < H * DH ? 0 : (pr < (H + 1) * DH ? 1 : (pr < (H + 2) * DH ? 2 : 3));
+  const int i = kind == 0 ? pr % DH : pr - (H + kind - 1) * DH;
+  const float2* rope = reinterpret_cast<const float2*>(p.rope) + i;
+  const int pos = (second ? 80 : 0) + (r >> 1);
+  const float cv = s_rinv && p.cvec ? p.cvec[n_tile * G::BM + r] : 0.0f;
+  // rotary cos/sin of the next step's tokens are fetched while this step is applied
+  float2 cs[16];
+  if (kind < 2) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) cs[j] = rope[tok_s[half * (TN / 2) + j] * DH];
+  }
+#pragma unroll 1   // rolled: a once-per-launch epilogue runs from a cold instruction cache
+  for (int st = 0; st < STEPS; ++st) {
+    const int c = half * (TN / 2) + st * 16;
+    float v[16];
+    tmem_ld16(taddr + c, v);
+    float2 cs_next[16];
+    if (kind < 2 && st + 1 < STEPS) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) cs_next[j] = rope[tok_s[c + 16 + j] * DH];
+    }
+    if (s_rinv) {   // folded norm: rinv[token] * (W z) + W shift (s_rinv indexed from the tile)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = fmaf(s_rinv[c + j], v[j], cv);
+    }
+    if (kind < 2) {   // warp-uniform: a warp's 16 pairs lie in one region (D/2 % 16 == 0)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+        // first half: x1 c - x2 s; second half: x2 c + x1 s (own value first)
+        v[j] = second ? fmaf(v[j], cs[j].x, other * cs[j].y) : fmaf(v[j], cs[j].x, -other * cs[j].y);
+      }
+      if (st + 1 < STEPS) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cs[j] = cs_next[j];
+      }
+    }
+    bf16* sb = stage + (st & 1) * 32 * RSTR + half * 16 * RSTR + pos;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sb[j * RSTR] = __float2bfloat16_rn(v[j]);
+    named_bar_sync(1, 256);
+    // 32 tokens x 16 runs of 8 dims; the other buffer is rewritten only after the next
+    // barrier, which every thread reaches after these copies
+#pragma unroll
+    for (int u = etid; u < 512; u += 256) {
+      const int tt = u >> 4, g = u & 15, hf = g >> 3;
+      const int col = (tt >> 4) * (TN / 2) + st * 16 + (tt & 15);
+      const int m = m0 + col;
+      const int pr0 = n_tile * (G::BM / 2) + (g & 7) * 8;
+      const int k0 = pr0 < H * DH ? 0 : (pr0 < (H + 1) * DH ? 1 : (pr0 < (H + 2) * DH ? 2 : 3));
+      if (m >= p.m_tok || k0 == 3) continue;
+      const int head = k0 == 0 ? pr0 / DH : 0;
+      const int dim0 = pr0 - (k0 == 0 ? head : H + k0 - 1) * DH + hf * DH;
+      const uint4 val = *reinterpret_cast<const uint4*>(stage + (st & 1) * 32 * RSTR + tt * RSTR + hf * 80 + (g & 7) * 8);
+      bf16* dst = k0 == 0 ? p.out + static_cast<size_t>(m) * p.ld_out + head * D + dim0
+                          : (k0 == 1 ? p.kc : p.vc) + static_cast<size_t>(tok_kv[col]) * D + dim0;
+      *reinterpret_cast<uint4*>(dst) = val;
+      if (k0 == 2 && p.vtc) {   // transposed V cache column (not used on the denoise path)
+        const bf16* e = reinterpret_cast<const bf16*>(&val);
+        const int bq = (m / p.seq);
+        bf16* vt = p.vtc + static_cast<size_t>(bq) * D * p.kcap + (tok_kv[col] - bq * p.kcap);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) vt[static_cast<size_t>(dim0 + x) * p.kcap] = e[x];
+      }
+    }
+  }
+}
 
 template <int TN, int EPI>
 __global__ void __launch_bounds__(320, 1)
     gemm_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                        const GemmParams p, int n_tiles, int m_tiles) {
+                        const __grid_constant__ CUtensorMap tm_r, const GemmParams p, int n_tiles, int m_tiles,
+                        int resid_map) {
   using G = PersistCfg<TN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -627,15 +771,27 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sB = smem + G::STAGES * G::A_BYTES;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + G::STAGES * G::STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2 * G::STAGES + 4);
+  const uint32_t rf0 = smem_u32(&bar[2 * G::STAGES + 5]);      // residual sub-tile k landed
+  static_assert((2 * G::STAGES + 5 + G::NSUB) * 8 <= 256, "barrier area");
+  float* s_rinv = reinterpret_cast<float*>(smem + G::SMEM_BASE - 1024);
+  float* s_ssq = s_rinv;   // residual writers (no folded norm there)
+
+  bf16* qkv_stage = reinterpret_cast<bf16*>(smem + G::SMEM_BASE - 1024 + G::RINV_BYTES);
+  int* tok_s = reinterpret_cast<int*>(smem + G::SMEM_BASE - 1024 + G::RINV_BYTES + G::QKV_STAGE_BYTES);
+  int* tok_kv = tok_s + TN;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = p.k_dim / G::BK;
   const int total = n_tiles * m_tiles;
+  // one tile per CTA and a residual tensor map: the residual tile of EPI_RESID goes
+  // through the idle stages
+  const bool resid_bulk = EPI == EPI_RESID && resid_map && total <= static_cast<int>(gridDim.x);
   const uint32_t full0 = smem_u32(&bar[0]);
   const uint32_t empty0 = smem_u32(&bar[G::STAGES]);
   const uint32_t tfull0 = smem_u32(&bar[2 * G::STAGES]);       // accumulator b filled
   const uint32_t tempty0 = smem_u32(&bar[2 * G::STAGES + 2]);  // accumulator b drained
 
   if (threadIdx.x == 0) {
+    trace_stamp(p.trace, 0);
     for (int s = 0; s < G::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
@@ -644,9 +800,11 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(tfull0 + 8 * b, 1);
       mbar_init(tempty0 + 8 * b, 1);
     }
+    for (int k = 0; k < G::NSUB; ++k) mbar_init(rf0 + 8 * k, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_x);
+    if (resid_bulk) prefetch_tmap(&tm_r);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), G::TMEM_COLS);
@@ -662,6 +820,7 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_last(), pol_x = policy_evict_last();
       pdl_wait();
+      trace_stamp(p.trace, 1);
       int g = 0;   // global k-block counter of this CTA (ring position)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
@@ -685,6 +844,25 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
+    if (resid_bulk && blockIdx.x < total && lane == 0) {
+      // the residual tile, one TMA box of 32 tokens x 128 features per sub-tile, into the
+      // pipeline buffers once the MMAs have released all of them (the last empty phase of
+      // every stage: the A and B buffers of the stages interleave in this range); rows past
+      // the last token are zero-filled
+      const int t = blockIdx.x, m_tile = t % m_tiles, n_tile = t / m_tiles;
+      const uint64_t pol = policy_evict_first();
+      for (int st = 0; st < G::STAGES && st < nkb; ++st) {
+        const int last = st + ((nkb - 1 - st) / G::STAGES) * G::STAGES;
+        mbar_wait(empty0 + 8 * st, (last / G::STAGES) & 1, p.err);
+      }
+      for (int k = 0; k < G::NSUB; ++k) {
+        const int st = k / G::RSUB_PER_STAGE;
+        mbar_arrive_expect_tx(rf0 + 8 * k, G::RSUB_BYTES);
+        tma_load_2d(smem_u32(smem + st * G::STAGE_BYTES + (k % G::RSUB_PER_STAGE) * G::RSUB_BYTES), &tm_r,
+                    rf0 + 8 * k, n_tile * G::BM, m_tile * TN + k * G::RSUB, pol);
+      }
+      // these copies complete on the rf barriers, which the epilogue waits for
+    }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, TN);
@@ -718,23 +896,230 @@ __global__ void __launch_bounds__(320, 1)
     pdl_wait();
     const int ew = warp - 2, q = warp & 3, r = q * 32 + lane, etid = ew * 32 + lane;
     const int c_begin = (ew >> 2) * (TN / 2);
+    // Folded norm: 1 / rms per token from the residual writers' sum-of-squares rows (one row
+    // per 128 features), for every token of the launch at once when they fit, before the
+    // first accumulator is ready.
+    const bool folded = (EPI == EPI_QKV || EPI == EPI_GEGLU) && p.rstat_in != nullptr;
+    const bool rinv_all = p.m_tok <= G::RINV_ALL;
+    auto rinv_of = [&](int m) -> float {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      int c = 0;
+      for (; c + 3 < p.rstat_n; c += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] += p.rstat_in[static_cast<size_t>(c + u) * p.ld_rstat + m];
+      }
+      for (; c < p.rstat_n; ++c) acc[0] += p.rstat_in[static_cast<size_t>(c) * p.ld_rstat + m];
+      const float ss = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      return 1.0f / sqrtf(ss / static_cast<float>(p.k_dim) + p.eps);
+    };
+    if (etid == 0) trace_stamp(p.trace, 2);
+    if (folded && rinv_all) {
+      // all tokens of this thread at once (up to 13), rows four at a time: every load of a
+      // round is in flight together
+      // (indices clamped instead of branches, so that the loads of a round issue together)
+      constexpr int NT = (G::RINV_ALL + 255) / 256;
+      float acc[NT][4];
+#pragma unroll
+      for (int k = 0; k < NT; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.0f;
+      const float* col[NT];
+#pragma unroll
+      for (int k = 0; k < NT; ++k) col[k] = p.rstat_in + min(etid + 256 * k, p.m_tok - 1);
+      const size_t ld = static_cast<size_t>(p.ld_rstat);
+      int c = 0;
+      for (; c + 3 < p.rstat_n; c += 4) {
+        float x[NT][4];
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) x[k][u] = __ldcg(col[k] + (c + u) * ld);
+#pragma unroll
+        for (int k = 0; k < NT; ++k)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[k][u] += x[k][u];
+      }
+      for (; c < p.rstat_n; ++c) {
+        float x[NT];
+#pragma unroll
+        for (int k = 0; k < NT; ++k) x[k] = __ldcg(col[k] + c * ld);
+#pragma unroll
+        for (int k = 0; k < NT; ++k) acc[k][0] += x[k];
+      }
+#pragma unroll
+      for (int k = 0; k < NT; ++k) {
+        const int m = etid + 256 * k;
+        const float ss = (acc[k][0] + acc[k][1]) + (acc[k][2] + acc[k][3]);
+        if (m < p.m_tok) s_rinv[m] = 1.0f / sqrtf(ss / static_cast<float>(p.k_dim) + p.eps);
+      }
+      named_bar_sync(1, 256);
+    }
+    if (etid == 0) trace_stamp(p.trace, 3);
     int lt = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++lt) {
       const int b = lt & 1;
       const int m_tile = t % m_tiles, n_tile = t / m_tiles;
+      const int fn = n_tile * G::BM + r, m0 = m_tile * TN;
+      // per-tile fallback (the previous tile's readers of s_rinv passed the barrier at its end)
+      if (folded && !rinv_all) {
+        for (int tt = etid; tt < TN; tt += 256) s_rinv[tt] = m0 + tt < p.m_tok ? rinv_of(m0 + tt) : 0.0f;
+        named_bar_sync(1, 256);
+      }
+      const float* rinv_t = rinv_all ? s_rinv + m0 : s_rinv;   // indexed by tile column
+      // EPI_RESID: the residual values of the first chunk are fetched before the
+      // accumulator is ready, those of chunk c + 1 while chunk c is applied
+      float old[16];
+      float* rbase = nullptr;
+      if (EPI == EPI_RESID && !resid_bulk) {
+        rbase = p.resid + fn;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c_begin + j;
+          old[j] = m < p.m_tok ? rbase[static_cast<size_t>(m) * p.ld_resid] : 0.0f;
+        }
+      }
       if (!mbar_wait(tfull0 + 8 * b, (lt >> 1) & 1, p.err)) break;
+      if (etid == 0 && lt < 6) trace_stamp(p.trace, 4 + 2 * lt);
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * TN);
-      const int fn = n_tile * G::BM + r, m0 = m_tile * TN;
+      if constexpr (EPI == EPI_QKV) {
+        qkv_epilogue_staged<TN>(p, taddr, n_tile, m0, ew, r, lane, qkv_stage, tok_s, tok_kv,
+                                folded ? rinv_t : nullptr);
+      } else if (EPI == EPI_RESID && resid_bulk) {
+        // x_res += g * acc on the sub-tiles in shared memory (in place), then bulk stores of
+        // their rows; z = x_res * (1 + zmod) in bf16 and the per-quarter sums of squares
+        const int half = ew >> 2;
+        const float g = p.vec ? p.vec[fn] : 1.0f;
+        const float zm = p.zout ? 1.0f + p.zmod[fn] : 0.0f;
+        float* srow = p.rstat_out ? s_ssq + ((lt & 1) * 4 + q) * TN : nullptr;
 #pragma unroll 1
-      for (int c = c_begin; c < c_begin + TN / 2; c += 16) {   // rolled: keeps the code small
-        float v[16];
-        tmem_ld16(taddr + c, v);
-        epi_apply<EPI>(p, v, fn, m0 + c, lane);
+        for (int kk = 0; kk < G::NSUB / 2; ++kk) {
+          const int k = half * (G::NSUB / 2) + kk;
+          float* sres = reinterpret_cast<float*>(smem + (k / G::RSUB_PER_STAGE) * G::STAGE_BYTES +
+                                                 (k % G::RSUB_PER_STAGE) * G::RSUB_BYTES);
+          if (!mbar_wait(rf0 + 8 * k, 0, p.err)) break;
+#pragma unroll
+          for (int cc = 0; cc < G::RSUB; cc += 16) {
+            const int c = k * G::RSUB + cc;
+            float v[16];
+            tmem_ld16(taddr + c, v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int m = m0 + c + j;
+              float* cell = sres + (cc + j) * G::BM + r;
+              if (m < p.m_tok) {
+                v[j] = fmaf(g, v[j], *cell);
+                *cell = v[j];
+                if (p.zout) p.zout[static_cast<size_t>(m) * p.ld_resid + fn] = __float2bfloat16_rn(v[j] * zm);
+              } else {
+                v[j] = 0.0f;
+              }
+              v[j] *= v[j];
+            }
+            if (srow) {
+              const float ss = warp_sum16(v, lane);
+              if (!(lane & 1)) srow[c + (lane >> 1)] = ss;
+            }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(2 + half, 128);
+          if ((ew & 3) == 0 && lane == 0) {   // one TMA store per sub-tile
+            tma_store_2d(&tm_r, smem_u32(sres), n_tile * G::BM, m0 + k * G::RSUB);
+            bulk_commit();
+          }
+        }
+        if ((ew & 3) == 0 && lane == 0) bulk_wait_all();   // the residual is written before exit
+      } else if constexpr (EPI == EPI_RESID) {
+        // x_res += g * acc; with a next norm to feed, also z = x_res * (1 + zmod) in bf16 and
+        // one sum-of-squares row per (tile row block of 32 features) and token
+        const float g = p.vec ? p.vec[fn] : 1.0f;
+        const float zm = p.zout ? 1.0f + p.zmod[fn] : 0.0f;
+        float* srow = p.rstat_out ? s_ssq + ((lt & 1) * 4 + q) * TN : nullptr;
+#pragma unroll   // unrolled, so that the loads of chunk c + 1 stay in flight across chunk c
+        for (int c = c_begin; c < c_begin + TN / 2; c += 16) {
+          float v[16], nxt[16];
+          tmem_ld16(taddr + c, v);
+          const bool more = c + 16 < c_begin + TN / 2;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = m0 + c + 16 + j;
+            nxt[j] = more && m < p.m_tok ? rbase[static_cast<size_t>(m) * p.ld_resid] : 0.0f;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = m0 + c + j;
+            v[j] = fmaf(g, v[j], old[j]);
+            if (m < p.m_tok) {
+              rbase[static_cast<size_t>(m) * p.ld_resid] = v[j];
+              if (p.zout) p.zout[static_cast<size_t>(m) * p.ld_resid + fn] = __float2bfloat16_rn(v[j] * zm);
+            } else {
+              v[j] = 0.0f;
+            }
+            v[j] *= v[j];
+          }
+          if (srow) {
+            const float ss = warp_sum16(v, lane);
+            if (!(lane & 1)) srow[c + (lane >> 1)] = ss;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) old[j] = nxt[j];
+        }
+      } else if constexpr (EPI == EPI_BIAS_STORE) {
+        // Pi0 action-time MLP output: x_res = acc + bias on action rows (state rows belong to
+        // the embedding), plus z and the sum-of-squares rows as above
+        const float bias = p.vec[fn];
+        const float zm = p.zout ? 1.0f + p.zmod[fn] : 0.0f;
+        float* srow = p.rstat_out ? s_ssq + ((lt & 1) * 4 + q) * TN : nullptr;
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + TN / 2; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = m0 + c + j;
+            v[j] += bias;
+            if (m < p.m_tok && !(p.has_state && (m % p.seq) == 0)) {
+              p.resid[static_cast<size_t>(m) * p.ld_resid + fn] = v[j];
+              if (p.zout) p.zout[static_cast<size_t>(m) * p.ld_resid + fn] = __float2bfloat16_rn(v[j] * zm);
+            } else {
+              v[j] = 0.0f;
+            }
+            v[j] *= v[j];
+          }
+          if (srow) {
+            const float ss = warp_sum16(v, lane);
+            if (!(lane & 1)) srow[c + (lane >> 1)] = ss;
+          }
+        }
+      } else {
+        const float cv = folded && p.cvec ? p.cvec[fn] : 0.0f;
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + TN / 2; c += 16) {   // rolled: keeps the code small
+          float v[16];
+          tmem_ld16(taddr + c, v);
+          if (folded) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = fmaf(rinv_t[c + j], v[j], cv);
+          }
+          epi_apply<EPI>(p, v, fn, m0 + c, lane);
+        }
       }
       tc_fence_before();
       named_bar_sync(1, 256);
       if (etid == 0) mbar_arrive(tempty0 + 8 * b);   // accumulator b may be overwritten
+      if (etid == 0 && lt < 6) trace_stamp(p.trace, 5 + 2 * lt);
+      if constexpr (EPI == EPI_RESID || EPI == EPI_BIAS_STORE) {
+        // one sum-of-squares row per 128 features: the four lane quarters, in order. The
+        // buffer of this tile parity is rewritten two tiles later, after the next tile's
+        // closing barrier, which every thread reaches after these reads.
+        if (p.rstat_out) {
+          for (int tt = etid; tt < TN; tt += 256) {
+            const int m = m0 + tt;
+            const float* sq = s_ssq + (lt & 1) * 4 * TN + tt;
+            if (m < p.m_tok)
+              p.rstat_out[static_cast<size_t>(p.rstat_slot0 + n_tile) * p.ld_rstat + m] =
+                  (sq[0] + sq[TN]) + (sq[2 * TN] + sq[3 * TN]);
+          }
+        }
+      }
     }
   }
 
@@ -747,41 +1132,44 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 template <int TN, int EPI>
-static cudaError_t launch_persist_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
-                                      int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+static cudaError_t launch_persist_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap* tm_r,
+                                      const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s,
+                                      bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(320, 1, 1);
-  cfg.dynamicSmemBytes = PersistCfg<TN>::SMEM;
+  cfg.dynamicSmemBytes = PersistCfg<TN>::smem(EPI);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, gemm_persist_kernel<TN, EPI>, tm_w, tm_x, p, n_tiles, m_tiles);
+  return cudaLaunchKernelEx(&cfg, gemm_persist_kernel<TN, EPI>, tm_w, tm_x, tm_r ? *tm_r : tm_w, p, n_tiles, m_tiles,
+                            tm_r ? 1 : 0);
 }
 
 template <int TN>
-static cudaError_t launch_persist_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
-                                     int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+static cudaError_t launch_persist_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap* tm_r,
+                                     const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
   switch (epi) {
-    case EPI_RESID: return launch_persist_one<TN, EPI_RESID>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case EPI_QKV: return launch_persist_one<TN, EPI_QKV>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case EPI_GEGLU: return launch_persist_one<TN, EPI_GEGLU>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case EPI_SWISH_VEC: return launch_persist_one<TN, EPI_SWISH_VEC>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case EPI_BIAS_STORE: return launch_persist_one<TN, EPI_BIAS_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case EPI_STORE: return launch_persist_one<TN, EPI_STORE>(tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_RESID: return launch_persist_one<TN, EPI_RESID>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_QKV: return launch_persist_one<TN, EPI_QKV>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_GEGLU: return launch_persist_one<TN, EPI_GEGLU>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_SWISH_VEC: return launch_persist_one<TN, EPI_SWISH_VEC>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_BIAS_STORE: return launch_persist_one<TN, EPI_BIAS_STORE>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case EPI_STORE: return launch_persist_one<TN, EPI_STORE>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                                   const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl) {
+                                   const CUtensorMap* tm_r, const GemmParams& p, int n_tiles, int m_tiles, int grid,
+                                   cudaStream_t s, bool pdl) {
   if (p.splits != 1) return cudaErrorInvalidValue;
   switch (tn) {
-    case 128: return launch_persist_tn<128>(epi, tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
-    case 256: return launch_persist_tn<256>(epi, tm_w, tm_x, p, n_tiles, m_tiles, grid, s, pdl);
+    case 128: return launch_persist_tn<128>(epi, tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case 256: return launch_persist_tn<256>(epi, tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -793,7 +1181,7 @@ static cudaError_t configure_persist_tn() {
                   gemm_persist_kernel<TN, EPI_GEGLU>, gemm_persist_kernel<TN, EPI_SWISH_VEC>,
                   gemm_persist_kernel<TN, EPI_BIAS_STORE>, gemm_persist_kernel<TN, EPI_STORE>})
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(PersistCfg<TN>::SMEM))) != cudaSuccess ||
+                                  static_cast<int>(PersistCfg<TN>::smem(EPI_QKV)))) != cudaSuccess ||
         (e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
       return e;

@@ -86,8 +86,12 @@ cudaError_t launch_gemm(int tn, int epi, const CUtensorMap& tm_w, const CUtensor
 int gemm_max_cluster();   // largest co-schedulable cluster of the 64-token push kernel
 // Persistent launch over n_tiles x m_tiles output tiles (splits must be 1), grid CTAs;
 // tn 128 or 256, two TMEM accumulators so epilogues overlap the next tile's main loop.
+// tm_r (EPI_RESID, optional): fp32 tensor map over the residual [m_tok][ld_resid] with
+// boxes of 128 features x 32 tokens; with one tile per CTA the residual tile then moves by
+// TMA through the idle pipeline stages.
 cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                                   const GemmParams& p, int n_tiles, int m_tiles, int grid, cudaStream_t s, bool pdl);
+                                   const CUtensorMap* tm_r, const GemmParams& p, int n_tiles, int m_tiles, int grid,
+                                   cudaStream_t s, bool pdl);
 cudaError_t configure_gemm_kernels();
 
 // ------------------------------------------------------------------ attention

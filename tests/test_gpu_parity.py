@@ -109,13 +109,15 @@ def test_repeat_calls_are_bit_identical_and_pdl_free_equal():
 
 def test_norm_kernels_path_matches_folded_norms():
     """Norms folded into the projections (z = bf16(r (1 + mod)), rinv from partial sums of
-    squares, W.shift added in the epilogue) against separate norm kernels, on one token
-    tile: tiny and mid_d128 (AdaRMSNorm), and observation 0 of mid_pi0_b3 alone (RMSNorm,
-    Pi0 time MLP, state token; 51 tokens). Both within tolerance of the oracle and of each
-    other."""
+    squares, W.shift added in the epilogue) against separate norm kernels. One token tile
+    (cluster split-K GEMMs): tiny and mid_d128 (AdaRMSNorm), observation 0 of mid_pi0_b3
+    alone (RMSNorm, Pi0 time MLP, state token; 51 tokens). Several token tiles (persistent
+    GEMMs): all of mid_pi0_b3 (153 tokens) and mid_ada_b2 (100 tokens). Both within
+    tolerance of the oracle and of each other."""
     from dataclasses import replace
     import flow_matching_vla_euler_b200 as V
-    for name, obs in (("tiny", None), ("mid_d128", None), ("mid_pi0_b3", 1)):
+    for name, obs in (("tiny", None), ("mid_d128", None), ("mid_pi0_b3", 1), ("mid_pi0_b3", None),
+                      ("mid_ada_b2", None)):
         wl = get(name)
         inp = make_inputs(wl)
         ref = golden_actions(name)
