@@ -519,6 +519,16 @@ struct Recorder {
   }
 };
 
+// Token tile of the persistent (several token tiles) GEMM. Residual projections (one tile
+// per CTA when they fit) may take 192-token tiles: at 3200 tokens and 1024 features that is
+// 136 tiles on 148 SMs instead of 104 of 256 tokens.
+int persist_tn(int n_feat, int M, int sm_count, bool resid) {
+  const int tn = plan_gemm(n_feat, 128, M, sm_count).tn;
+  if (!resid || tn != 256) return tn;
+  auto cost = [&](int t) { return cdiv((n_feat / 128) * cdiv(M, t), sm_count) * t; };
+  return cost(192) < cost(256) ? 192 : 256;
+}
+
 GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
   const int tn = plan_gemm(n_feat, k_dim, M, h->sm_count).tn;
   return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, tn == 64 ? h->gemm_cluster : 1);
@@ -536,7 +546,11 @@ int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensor
                  const CUtensorMap& tx, GemmParams p, int n_feat, int k_dim, int M, bool pdl) {
   if (M > 64) {
     // several token tiles: persistent kernel, one CTA per SM, no K split
-    const GemmPlan g0 = plan_gemm(n_feat, k_dim, M, h->sm_count);
+    // the residual map only for the residual stream itself (rows M)
+    const CUtensorMap* tr = (epi == EPI_RESID && p.resid == h->resid) ? &h->tm_resid : nullptr;
+    GemmPlan g0 = plan_gemm(n_feat, k_dim, M, h->sm_count);
+    g0.tn = persist_tn(n_feat, M, h->sm_count, tr != nullptr);
+    g0.m_tiles = cdiv(M, g0.tn);
     p.n_feat = n_feat;
     p.k_dim = k_dim;
     p.m_tok = M;
@@ -547,8 +561,6 @@ int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensor
     p.ld_rstat = h->max_M;
     const int total = g0.n_tiles * g0.m_tiles;
     rec.begin(kind);
-    // the residual map only for the residual stream itself (rows M)
-    const CUtensorMap* tr = (epi == EPI_RESID && p.resid == h->resid) ? &h->tm_resid : nullptr;
     CU(launch_gemm_persistent(g0.tn, epi, tw, tx, tr, p, g0.n_tiles, g0.m_tiles, std::min(total, h->sm_count), rec.s,
                               pdl));
     return rec.end(kind);
@@ -808,10 +820,12 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
 int make_act_maps(vla_expert* h, int B, ActMaps* am) {
   const int M = B * h->S;
   const uint32_t tn = static_cast<uint32_t>(plan_gemm(128, 128, M, h->sm_count).tn);
+  // the inputs of the residual projections (O, down) follow their token tile
+  const uint32_t tn_res = static_cast<uint32_t>(M > 64 ? persist_tn(h->W, M, h->sm_count, true) : tn);
   int rc;
   if ((rc = make_tmap(&am->hb, h->hb, h->W, M, tn))) return rc;
-  if ((rc = make_tmap(&am->ob, h->ob, h->HD, M, tn))) return rc;
-  if ((rc = make_tmap(&am->ub, h->ub, h->F, M, tn))) return rc;
+  if ((rc = make_tmap(&am->ob, h->ob, h->HD, M, tn_res))) return rc;
+  if ((rc = make_tmap(&am->ub, h->ub, h->F, M, tn_res))) return rc;
   if (h->pi0) {
     if ((rc = make_tmap(&am->eb, h->eb, h->W, M, tn))) return rc;
     if ((rc = make_tmap(&am->h1b, h->h1b, h->W, M, tn))) return rc;

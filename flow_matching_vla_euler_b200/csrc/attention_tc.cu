@@ -13,9 +13,11 @@
 //   in the exp2 domain, which keeps every P <= 256 while rescaling O rarely.
 // V is read from the transposed cache [D][keys] so that it is a K-major MMA operand.
 //
-// Warp roles (192 threads): warp 0 TMA (Q once, then K and V^T blocks in two rings: a K
+// Warp roles (320 threads): warp 0 TMA (Q once, then K and V^T blocks in two rings: a K
 // slot frees after its score MMA, a V^T slot after its P V MMA),
-// warp 1 tcgen05.mma, warps 2..5 softmax and output (TMEM lanes = query rows).
+// warp 1 tcgen05.mma, warps 2..9 softmax and output: two warps per TMEM lane quarter
+// (query rows), each taking half of a block's 64 key columns and half of the output
+// columns; the pair agrees on the row's reference maximum through shared memory.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -33,7 +35,8 @@ constexpr int SM_V = SM_K + 2 * K_SLOT;  // V^T ring, 2 slots of [256 dims][64 k
 constexpr int V_SLOT = kTK * kD * 2;
 constexpr int SM_P = SM_V + 2 * V_SLOT;  // P [128 rows][64 keys] bf16
 constexpr int SM_BAR = SM_P + kTQ * kTK * 2;
-constexpr size_t kSmem = 1024 + SM_BAR + 256;
+constexpr int SM_XCH = SM_BAR + 256;      // [2 parity][2 halves][128 rows] block maxima, [2][128] sums
+constexpr size_t kSmem = 1024 + SM_XCH + 6 * kTQ * 4;
 
 struct Seg {
   int off[3], cnt[3], nt[3];
@@ -52,7 +55,7 @@ __device__ __forceinline__ void block_info(const Seg& sg, int t, int& row, int& 
 
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_vt, const AttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -79,9 +82,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(vfull0 + 8 * i, 1);
       mbar_init(vempty0 + 8 * i, 1);
       mbar_init(sfull0 + 8 * i, 1);
-      mbar_init(sempty0 + 8 * i, 4);     // one arrival per softmax warp
+      mbar_init(sempty0 + 8 * i, 8);     // one arrival per softmax warp
     }
-    mbar_init(pfull, 4);
+    mbar_init(pfull, 8);
     mbar_init(pempty, 1);
     mbar_init(ofull, 1);
     fence_mbar_init();
@@ -197,37 +200,37 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     const int qd = warp & 3, r = qd * 32 + lane;          // TMEM lane = query row of the tile
+    const int ch = (warp - 2) >> 2;                        // key / output column half
     const int qrow = row0 + r;
     const bool row_ok = qrow < R;
     const int s_q = qrow / p.n_heads;                      // suffix position of this query row
     const uint32_t tl = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(smem + SM_XCH);          // [2][2][128]
+    float* xsum = xmax + 4 * kTQ;                                    // [2][128]
+    const int pair_bar = 2 + qd;                                     // the two warps of lane quarter qd
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
-    // scores of block t (S buffer t & 1) -> x[] in the exp2 domain, masked
-    auto load_scores = [&](int t, float (&x)[kTK]) -> bool {
+    // this half's 32 scores of block t (S buffer t & 1) -> x[] in the exp2 domain, masked
+    auto load_scores = [&](int t, float (&x)[kTK / 2]) -> bool {
       const int sb = t & 1;
       if (!mbar_wait(sfull0 + 8 * sb, (t >> 1) & 1, p.err)) return false;
       tc_fence_after();
-      float v0[32], v1[32];
-      tmem_ld32(tl + sb * kTK, v0);
-      tmem_ld32(tl + sb * kTK + 32, v1);
+      float v[32];
+      tmem_ld32(tl + sb * kTK + ch * 32, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sempty0 + 8 * sb);
       int row, cnt, ds;
       block_info(sg, t, row, cnt, ds);
       // the state row sees only dynamic key 0: the rest of a dynamic block is masked
-      const int lim = (ds >= 0 && p.has_state && s_q == 0) ? (ds == 0 ? 1 : 0) : cnt;
+      const int lim = ((ds >= 0 && p.has_state && s_q == 0) ? (ds == 0 ? 1 : 0) : cnt) - ch * 32;
 #pragma unroll
-      for (int c = 0; c < kTK; ++c) {
-        const float sv = c < 32 ? v0[c & 31] : v1[c & 31];
-        x[c] = c < lim ? sv * p.scale_log2 : -INFINITY;
-      }
+      for (int c = 0; c < 32; ++c) x[c] = c < lim ? v[c] * p.scale_log2 : -INFINITY;
       return true;
     };
     uint8_t* sP = smem + SM_P;
     for (int t = 0; t < T && ok; ++t) {
-      float x[kTK];
+      float x[kTK / 2];
       if (!load_scores(t, x)) {
         ok = false;
         break;
@@ -235,7 +238,12 @@ __global__ void __launch_bounds__(192, 1)
       if (t < 4 && threadIdx.x == 64) trace_stamp(p.trace, 2 + t);
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kTK; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 0; c < 32; ++c) mx = fmaxf(mx, x[c]);
+      // the row's block maximum over both halves (buffers alternate by block parity: a
+      // buffer is rewritten two blocks later, after the pair's next barrier)
+      xmax[((t & 1) * 2 + ch) * kTQ + r] = mx;
+      named_bar_sync(pair_bar, 64);
+      mx = fmaxf(mx, xmax[((t & 1) * 2 + (ch ^ 1)) * kTQ + r]);
       // move the reference maximum only when this block exceeds it by more than 2^8
       float factor = 1.0f;
       const bool move = mx > m + 8.0f || (m == -INFINITY && mx != -INFINITY);
@@ -244,10 +252,10 @@ __global__ void __launch_bounds__(192, 1)
         m = mx;
         l *= factor;
       }
-      uint32_t pk[kTK / 2];
+      uint32_t pk[kTK / 4];
       float sum = 0.0f;
 #pragma unroll
-      for (int c = 0; c < kTK; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         const float p0 = m == -INFINITY ? 0.0f : exp2_approx(x[c] - m);
         const float p1 = m == -INFINITY ? 0.0f : exp2_approx(x[c + 1] - m);
         sum += p0 + p1;
@@ -260,9 +268,9 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       if (t >= 1 && __any_sync(0xffffffffu, move)) {
-        // rescale this warp's rows of O (32 rows x 256 columns) by their factors
+        // rescale this warp's rows of O (32 rows x its 128 columns) by their factors
         tc_fence_after();
-        for (int c0 = 0; c0 < kD; c0 += 32) {
+        for (int c0 = ch * 128; c0 < ch * 128 + 128; c0 += 32) {
           float v[32];
           tmem_ld32(tl + 256 + c0, v);
 #pragma unroll
@@ -271,22 +279,26 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_before();
       }
-      // row r of P: 64 keys = 8 chunks of 16 bytes, chunk j stored at j ^ (r & 7)
+      // row r of P: 64 keys = 8 chunks of 16 bytes (this half: 4), chunk j stored at j ^ (r & 7)
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(sP + r * 128 + ((j ^ (r & 7)) << 4)) =
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(sP + r * 128 + (((ch * 4 + j) ^ (r & 7)) << 4)) =
             make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(pfull);
       if (t < 4 && threadIdx.x == 64) trace_stamp(p.trace, 7 + t);
     }
+    // the row sum over both halves
+    xsum[ch * kTQ + r] = l;
+    named_bar_sync(pair_bar, 64);
+    l += xsum[(ch ^ 1) * kTQ + r];
     mbar_wait(ofull, 0, p.err);
     if (threadIdx.x == 64) trace_stamp(p.trace, 11);
     tc_fence_after();
     const float inv = (row_ok && l > 0.0f) ? 1.0f / l : 0.0f;
     bf16* dst = p.out + (static_cast<size_t>(b) * R + qrow) * kD;
-    for (int c0 = 0; c0 < kD; c0 += 32) {
+    for (int c0 = ch * 128; c0 < ch * 128 + 128; c0 += 32) {
       float v[32];
       tmem_ld32(tl + 256 + c0, v);
       if (row_ok) {
@@ -328,7 +340,7 @@ cudaError_t launch_attention_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k
   cudaLaunchConfig_t cfg = {};
   const int R = p.seq * p.n_heads;
   cfg.gridDim = dim3((R + kTQ - 1) / kTQ, batch, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -610,8 +610,8 @@ struct PersistCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = TN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = TN == 256 ? 4 : 6;
-  static constexpr int TMEM_COLS = 2 * TN;       // two accumulators
+  static constexpr int STAGES = TN == 128 ? 6 : 4;
+  static constexpr int TMEM_COLS = TN == 192 ? 512 : 2 * TN;   // two accumulators (power of 2)
   // EPI_QKV stages its bf16 output through shared memory: two buffers of 32 token rows
   // (16 per column half) x QKV_RSTR elements, plus the tile's per-token table
   static constexpr int QKV_RSTR = 144;           // pair half 0 at [0, 64), half 1 at [80, 144)
@@ -1169,6 +1169,9 @@ cudaError_t launch_gemm_persistent(int tn, int epi, const CUtensorMap& tm_w, con
   if (p.splits != 1) return cudaErrorInvalidValue;
   switch (tn) {
     case 128: return launch_persist_tn<128>(epi, tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
+    case 192:   // the residual projections only (136 tiles of 192 tokens fill the SMs at 3200 tokens)
+      if (epi != EPI_RESID) return cudaErrorInvalidValue;
+      return launch_persist_one<192, EPI_RESID>(tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
     case 256: return launch_persist_tn<256>(epi, tm_w, tm_x, tm_r, p, n_tiles, m_tiles, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
@@ -1225,6 +1228,11 @@ cudaError_t configure_gemm_kernels() {
   if ((e = configure_tn<64, true>()) != cudaSuccess) return e;
   if ((e = configure_persist_tn<128>()) != cudaSuccess) return e;
   if ((e = configure_persist_tn<256>()) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(gemm_persist_kernel<192, EPI_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(PersistCfg<192>::smem(EPI_RESID)))) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(gemm_persist_kernel<192, EPI_RESID>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+    return e;
   done = cudaSuccess;
   return done;
 }
