@@ -10,4 +10,5 @@ from .expert import (TIME_ADA_MLP, TIME_ADA_SINCOS, TIME_PI0_MLP, ada_rms_norm, 
                      decode_params, denoise, euler_integrate, expert_velocity, gelu_tanh,
                      masked_attention, rms_norm, rms_normalize, rope, sincos_embedding,
                      suffix_mask, swish, time_conditioning, time_grid)
+from .prefill import prefill_batch, prefill_kv
 from .ring import RingModel
