@@ -53,6 +53,19 @@ class vla_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
+PREFILL_WEIGHT_FIELDS = ["wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "norm1_w", "norm2_w"]
+
+
+class vla_prefill_config(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_int) for n in ["n_layers", "width", "n_heads", "head_dim", "mlp_dim", "max_tokens",
+                                             "max_batch"]] +
+                [("eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("flags", ctypes.c_uint)])
+
+
+class vla_prefill_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in PREFILL_WEIGHT_FIELDS]
+
+
 class vla_kernel_times(ctypes.Structure):
     _fields_ = [("total_ms", ctypes.c_float * 10), ("launches", ctypes.c_int * 10),
                 ("bytes", ctypes.c_double * 10), ("flops", ctypes.c_double * 10)]
@@ -84,6 +97,11 @@ _SIGNATURES = {
     "vla_selftest_wait_timeout": (_I, [_P, _I, _P]),
     "vla_gemm_status": (_I, [_P]),
     "vla_persist_info": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "vla_prefill_create": (_I, [ctypes.POINTER(vla_prefill_config), ctypes.POINTER(vla_prefill_weights),
+                                ctypes.POINTER(_P)]),
+    "vla_prefill_destroy": (None, [_P]),
+    "vla_prefill_run": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "vla_prefill_status": (_I, [_P, _P]),
     "vla_last_error": (ctypes.c_char_p, []),
     "vla_version": (ctypes.c_char_p, []),
 }
@@ -152,6 +170,24 @@ def vla_cache_export(h, K_ptr, V_ptr, batch, stream):
     return head.value, ns.value, nr.value
 
 
+def vla_prefill_create(cfg: vla_prefill_config, weights: vla_prefill_weights) -> int:
+    h = _P()
+    _check(load_library().vla_prefill_create(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(h)))
+    return h.value
+
+
+def vla_prefill_destroy(h: int):
+    load_library().vla_prefill_destroy(h)
+
+
+def vla_prefill_run(h, tokens_ptr, n_tokens, batch, K_ptr, V_ptr, stream):
+    _check(load_library().vla_prefill_run(h, tokens_ptr, n_tokens, batch, K_ptr, V_ptr, stream))
+
+
+def vla_prefill_status(h, stream):
+    _check(load_library().vla_prefill_status(h, stream))
+
+
 def vla_device_status(h, stream):
     _check(load_library().vla_device_status(h, stream))
 
@@ -217,6 +253,59 @@ def _dev_ptr(t, dtype_bytes):
     if not t.is_contiguous() or t.element_size() != dtype_bytes:
         raise TypeError(f"expected a contiguous tensor of {dtype_bytes}-byte elements")
     return t.data_ptr()
+
+
+class Prefill:
+    """One prefill handle. ``cfg`` has n_layers, width, n_heads, head_dim, mlp_dim, eps and
+    rope_base; ``params`` maps "wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "norm1.w",
+    "norm2.w" to uint16 numpy arrays of bf16 bits."""
+
+    def __init__(self, cfg, params: dict, max_tokens: int, max_batch: int = 1):
+        import numpy as np
+        c = vla_prefill_config()
+        for n in ["n_layers", "width", "n_heads", "head_dim", "mlp_dim"]:
+            setattr(c, n, int(getattr(cfg, n)))
+        c.max_tokens, c.max_batch = int(max_tokens), int(max_batch)
+        c.eps, c.rope_base, c.flags = float(cfg.eps), float(cfg.rope_base), 0
+        w = vla_prefill_weights()
+        keep = []
+        for name, arr in params.items():
+            field = name.replace(".", "_")
+            if field not in PREFILL_WEIGHT_FIELDS:
+                raise KeyError(f"unknown parameter {name}")
+            a = np.ascontiguousarray(np.asarray(arr).astype(np.uint16, copy=False))
+            keep.append(a)
+            setattr(w, field, a.ctypes.data)
+        self.cfg = cfg
+        self.handle = vla_prefill_create(c, w)
+        del keep
+
+    def close(self):
+        if getattr(self, "handle", None):
+            vla_prefill_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def run(self, tokens, K_out=None, V_out=None):
+        """tokens: CUDA fp32 [batch, n_tokens, width] -> K, V: CUDA int16 tensors (bf16 bits)
+        [L, batch, n_tokens, head_dim], allocated when not given."""
+        import torch
+        batch, n = int(tokens.shape[0]), int(tokens.shape[1])
+        shape = (self.cfg.n_layers, batch, n, self.cfg.head_dim)
+        if K_out is None:
+            K_out = torch.empty(shape, dtype=torch.int16, device=tokens.device)
+        if V_out is None:
+            V_out = torch.empty(shape, dtype=torch.int16, device=tokens.device)
+        vla_prefill_run(self.handle, _dev_ptr(tokens, 4), n, batch, _dev_ptr(K_out, 2), _dev_ptr(V_out, 2), _stream())
+        return K_out, V_out
+
+    def status(self):
+        vla_prefill_status(self.handle, _stream())
 
 
 class Expert:

@@ -313,8 +313,8 @@ struct vla_expert {
 namespace {
 
 
-template <typename T>
-int dalloc(vla_expert* h, T** p, size_t count) {
+template <typename Hd, typename T>
+int dalloc(Hd* h, T** p, size_t count) {
   void* q = nullptr;
   cudaError_t e = cudaMalloc(&q, std::max<size_t>(count, 1) * sizeof(T));
   if (e != cudaSuccess)
@@ -326,14 +326,16 @@ int dalloc(vla_expert* h, T** p, size_t count) {
   return VLA_OK;
 }
 
-int upload_bf16(vla_expert* h, bf16** dst, const uint16_t* src, size_t n) {
+template <typename Hd>
+int upload_bf16(Hd* h, bf16** dst, const uint16_t* src, size_t n) {
   int rc = dalloc(h, dst, n);
   if (rc) return rc;
   CU(cudaMemcpy(*dst, src, n * 2, cudaMemcpyHostToDevice));
   return VLA_OK;
 }
 
-int upload_f32(vla_expert* h, float** dst, const uint16_t* src, size_t n) {
+template <typename Hd>
+int upload_f32(Hd* h, float** dst, const uint16_t* src, size_t n) {
   std::vector<float> tmp(n);
   for (size_t i = 0; i < n; ++i) tmp[i] = bf16_to_f32(src[i]);
   int rc = dalloc(h, dst, n);
@@ -723,7 +725,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           if (use_tc_attn) {   // transposed V of the chunk (counted with attention)
             const size_t lofs = static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
             rec.begin(VLA_K_ATTN);
-            CU(launch_vt_dyn(p.vc, h->vtc + lofs, B, h->D, h->kcap, h->dyn_off, h->S, rec.s, pdl));
+            CU(launch_vt_dyn(p.vc, h->vtc + lofs, B, h->D, h->kcap, h->kcap, h->dyn_off, h->S, rec.s, pdl));
             rec.end(VLA_K_ATTN);
           }
           rec.begin(VLA_K_ATTN);
@@ -1315,6 +1317,10 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     if ((rc = dalloc(h, &h->trace, static_cast<size_t>(5) * 512 * 16))) return cleanup(rc);
   }
 
+  // The zero fills of dalloc run on the legacy stream, behind whatever the caller still has
+  // in flight there; the handle's own stream does not wait for them, so they must have
+  // finished before the tables below are computed on it.
+  CU(cudaDeviceSynchronize());
   cudaError_t e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cleanup(fail(VLA_ERR_CUDA, "stream create: %s", cudaGetErrorString(e)));
   int slot;
@@ -1809,3 +1815,5 @@ int vla_gemm_status(void* cuda_stream) {
 }
 
 }  // extern "C"
+
+#include "prefill_api.cuh"   // the prefix prefill handle, sharing this file's helpers

@@ -203,8 +203,9 @@ cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, i
 cudaError_t launch_cache_update(CacheDesc* desc, int n_static, int n_ring, float* rope,
                                 int seq, int head_dim, float rope_base, cudaStream_t s);
 // vt[l-slice][b][d][dyn_off + s] = vc[l-slice][b][dyn_off + s][d] for s < seq (pointers
-// to one layer's caches); D a multiple of 64.
-cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, int dyn_off, int seq,
+// to one layer's caches: vc with kcap rows, vt with rows of kcap_t positions per
+// observation); D a multiple of 64.
+cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, int kcap_t, int dyn_off, int seq,
                           cudaStream_t s, bool pdl);
 cudaError_t launch_copy_region(const bf16* kc, bf16* out, int L, int batch, int max_batch,
                                int kcap, int rows, int D, int n_static_max, int ring_off, cudaStream_t s);

@@ -366,15 +366,16 @@ cudaError_t launch_ring_append(const bf16* K, const bf16* V, int batch, int L, i
 // Transposed V of the dynamic region (the chunk's own keys) for the tensor-core
 // attention: vt[b][d][dyn_off + s] = v[b][dyn_off + s][d], s < seq, one CTA per
 // (64 dims, 64 positions, observation) through a padded shared-memory tile, so that both
-// the reads (along d) and the writes (along s) are coalesced.
+// the reads (along d) and the writes (along s) are coalesced. The source holds kcap rows
+// per observation, the destination kcap_t positions per row.
 __global__ void __launch_bounds__(256) vt_dyn_kernel(const uint16_t* __restrict__ vc, uint16_t* __restrict__ vt,
-                                                     int D, int kcap, int dyn_off, int seq) {
+                                                     int D, int kcap, int kcap_t, int dyn_off, int seq) {
   __shared__ uint16_t tile[64][66];
   pdl_wait();
   if (threadIdx.x == 0) pdl_trigger();
   const int d0 = blockIdx.x * 64, s0 = blockIdx.y * 64, b = blockIdx.z;
   const uint16_t* src = vc + (static_cast<size_t>(b) * kcap + dyn_off) * D;
-  uint16_t* dst = vt + static_cast<size_t>(b) * D * kcap + dyn_off;
+  uint16_t* dst = vt + static_cast<size_t>(b) * D * kcap_t + dyn_off;
   for (int i = threadIdx.x; i < 64 * 64; i += 256) {
     const int r = i >> 6, c = i & 63;   // r: position, c: dim
     if (s0 + r < seq) tile[c][r] = src[static_cast<size_t>(s0 + r) * D + d0 + c];
@@ -382,17 +383,17 @@ __global__ void __launch_bounds__(256) vt_dyn_kernel(const uint16_t* __restrict_
   __syncthreads();
   for (int i = threadIdx.x; i < 64 * 64; i += 256) {
     const int r = i >> 6, c = i & 63;   // r: dim, c: position
-    if (s0 + c < seq) dst[static_cast<size_t>(d0 + r) * kcap + s0 + c] = tile[r][c];
+    if (s0 + c < seq) dst[static_cast<size_t>(d0 + r) * kcap_t + s0 + c] = tile[r][c];
   }
 }
 
-cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, int dyn_off, int seq,
+cudaError_t launch_vt_dyn(const bf16* vc, bf16* vt, int batch, int D, int kcap, int kcap_t, int dyn_off, int seq,
                           cudaStream_t s, bool pdl) {
   if (D % 64) return cudaErrorInvalidValue;
   cudaLaunchAttribute attr[1];
   cudaLaunchConfig_t cfg = make_cfg(dim3(D / 64, (seq + 63) / 64, batch), dim3(256), 0, s, attr, pdl);
   return cudaLaunchKernelEx(&cfg, vt_dyn_kernel, reinterpret_cast<const uint16_t*>(vc),
-                            reinterpret_cast<uint16_t*>(vt), D, kcap, dyn_off, seq);
+                            reinterpret_cast<uint16_t*>(vt), D, kcap, kcap_t, dyn_off, seq);
 }
 
 // Descriptor + rotary table [seq][D/2] of (cos, sin) at positions pos0 + s, in double.

@@ -337,6 +337,68 @@ VLA_API int vla_gemm_status(void* cuda_stream);
  */
 VLA_API int vla_persist_info(vla_expert* h, int* ctas, int* cluster, int* max_clusters);
 
+/* ------------------------------------------------------------------ prefix prefill
+ *
+ * The language side of the policy over the perception and prompt tokens, producing the
+ * per-layer K/V that vla_cache_set_prefix takes (realtime-vla write-up, "The problem is a
+ * policy that thinks too long": vision encoder, LLM, action expert; InstinctFlash README,
+ * GRAPH layer: prefill extraction). A Gemma-class decoder: per layer
+ *   h = RMSNorm_1(x) (Gemma (1 + w) scale); q, k, v = h Wq^T, h Wk^T, h Wv^T; RoPE(q, k) at
+ *   positions 0..n_tokens-1; K[l], V[l] = k, v; x += softmax(q k^T / sqrt(D)) v Wo^T, every
+ *   prefix token seeing every other one (one bidirectional block); x += W_down (gelu_tanh(
+ *   W_gate RMSNorm_2(x)) * W_up RMSNorm_2(x)).
+ * One K/V head (GQA); no biases. The last layer's attention output and MLP feed no K/V and
+ * are not computed. Its layer count, head_dim and rope_base must match the action expert's
+ * for the two to share the cache. The first token embedding (image tokens from the vision
+ * encoder, then the embedded prompt) is the caller's.
+ */
+typedef struct vla_prefill vla_prefill;   /* opaque, owned by the library */
+
+typedef struct vla_prefill_config {
+  int n_layers;      /* L */
+  int width;         /* W, multiple of 128, <= 2048 */
+  int n_heads;       /* H query heads (one K/V head) */
+  int head_dim;      /* D: 32, 64, 128 or 256; H * D a multiple of 64 */
+  int mlp_dim;       /* F, multiple of 64 */
+  int max_tokens;    /* largest n_tokens of a run, >= 1 */
+  int max_batch;     /* largest batch of a run, >= 1 */
+  float eps;         /* RMSNorm epsilon */
+  float rope_base;   /* rotary base */
+  unsigned flags;    /* 0 */
+} vla_prefill_config;
+
+/* HOST pointers, bf16 bit patterns, matrices row-major [L][out][in]; copied at create. */
+typedef struct vla_prefill_weights {
+  const uint16_t *wq, *wk, *wv;          /* [L][H*D][W], [L][D][W], [L][D][W] */
+  const uint16_t *wo;                    /* [L][W][H*D] */
+  const uint16_t *w_gate, *w_up;         /* [L][F][W] */
+  const uint16_t *w_down;                /* [L][W][F] */
+  const uint16_t *norm1_w, *norm2_w;     /* [L][W] */
+} vla_prefill_weights;
+
+/* Allocates every device buffer for max_batch x max_tokens and uploads the repacked
+ * weights. Errors: VLA_ERR_ARG (null or missing pointer, flags), VLA_ERR_SHAPE (dims),
+ * VLA_ERR_UNSUPPORTED (not sm_100), VLA_ERR_OOM, VLA_ERR_CUDA. */
+VLA_API int vla_prefill_create(const vla_prefill_config* cfg, const vla_prefill_weights* w,
+                               vla_prefill** out);
+VLA_API void vla_prefill_destroy(vla_prefill* h);
+
+/*
+ * vla_prefill_run -- asynchronously on cuda_stream: tokens, DEVICE fp32 [batch][n_tokens][W]
+ * (read only), -> K_out, V_out, DEVICE bf16 [L][batch][n_tokens][D] (post-RoPE keys; the
+ * layout vla_cache_set_prefix reads; 16-byte aligned; written, not read). Observations are
+ * independent. Buffers must not overlap and stay valid until the stream reaches the end of
+ * the call. Errors (nothing enqueued): VLA_ERR_ARG, VLA_ERR_SHAPE (n_tokens outside
+ * [1, max_tokens] or batch outside [1, max_batch]), VLA_ERR_CUDA. A bounded device wait that
+ * gave up is reported by vla_prefill_status.
+ */
+VLA_API int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch, uint16_t* K_out,
+                            uint16_t* V_out, void* cuda_stream);
+
+/* Synchronizes cuda_stream, then reads and clears the handle's device status word:
+ * VLA_OK or VLA_ERR_TIMEOUT (a run's K/V are then not valid), or VLA_ERR_CUDA. */
+VLA_API int vla_prefill_status(vla_prefill* h, void* cuda_stream);
+
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VLA_API const char* vla_last_error(void);
 

@@ -44,6 +44,9 @@ def test_struct_layout_matches_header(lib):
              offsetof(vla_config, flags), sizeof(vla_weights), offsetof(vla_weights, w_down));
       printf("%zu %zu %zu\n", sizeof(vla_kernel_times), offsetof(vla_kernel_times, bytes),
              offsetof(vla_kernel_times, flops));
+      printf("%zu %zu %zu %zu %zu\n", sizeof(vla_prefill_config), offsetof(vla_prefill_config, eps),
+             offsetof(vla_prefill_config, flags), sizeof(vla_prefill_weights),
+             offsetof(vla_prefill_weights, norm2_w));
       return 0;
     }
     """
@@ -58,8 +61,45 @@ def test_struct_layout_matches_header(lib):
     exp = [ctypes.sizeof(V.vla_config), V.vla_config.eps.offset, V.vla_config.flags.offset,
            ctypes.sizeof(V.vla_weights), V.vla_weights.w_down.offset,
            ctypes.sizeof(V.vla_kernel_times), V.vla_kernel_times.bytes.offset,
-           V.vla_kernel_times.flops.offset]
+           V.vla_kernel_times.flops.offset,
+           ctypes.sizeof(V.vla_prefill_config), V.vla_prefill_config.eps.offset,
+           V.vla_prefill_config.flags.offset, ctypes.sizeof(V.vla_prefill_weights),
+           V.vla_prefill_weights.norm2_w.offset]
     assert got == exp
+
+
+def test_prefill_weight_fields_cover_generator_names():
+    from vla_inputs import PREFILL_WORKLOADS, prefill_param_shapes
+    for wl in PREFILL_WORKLOADS.values():
+        for name in prefill_param_shapes(wl.cfg):
+            assert name.replace(".", "_") in V.PREFILL_WEIGHT_FIELDS
+
+
+def test_prefill_create_rejects_bad_arguments_before_any_cuda_call(lib):
+    def cfg(**kw):
+        c = V.vla_prefill_config()
+        base = dict(n_layers=2, width=128, n_heads=4, head_dim=32, mlp_dim=512, max_tokens=48, max_batch=1)
+        base.update(kw)
+        for k, v in base.items():
+            setattr(c, k, v)
+        c.eps, c.rope_base = 1e-6, 10000.0
+        return c
+    h = ctypes.c_void_p()
+    w = V.vla_prefill_weights()
+    assert lib.vla_prefill_create(None, None, ctypes.byref(h)) == V.VLA_ERR_ARG
+    assert lib.vla_prefill_create(ctypes.byref(cfg()), ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
+    buf = (ctypes.c_uint16 * 4)()
+    for f in V.PREFILL_WEIGHT_FIELDS:
+        setattr(w, f, ctypes.addressof(buf))
+    for bad in [dict(width=100), dict(width=4096), dict(head_dim=48), dict(n_heads=3, head_dim=32),
+                dict(mlp_dim=100), dict(max_tokens=0), dict(max_batch=0), dict(n_layers=0)]:
+        assert lib.vla_prefill_create(ctypes.byref(cfg(**bad)), ctypes.byref(w), ctypes.byref(h)) == \
+            V.VLA_ERR_SHAPE, bad
+    c = cfg()
+    c.flags = 1
+    assert lib.vla_prefill_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
+    assert lib.vla_prefill_run(None, None, 1, 1, None, None, None) == V.VLA_ERR_ARG
+    assert lib.vla_prefill_status(None, None) == V.VLA_ERR_ARG
 
 
 def test_weight_fields_cover_generator_names():
