@@ -53,6 +53,8 @@ def parse_args(argv=None):
                    help="profiling aid: Euler steps per denoise instead of the workload's (0: keep)")
     p.add_argument("--fp8-workload", default="pi05_3view_fp8")
     p.add_argument("--no-fp8", action="store_true")
+    p.add_argument("--prefill-workload", default="prefill_pi05_3view")
+    p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--path", choices=["auto", "chain", "persistent"], default="auto",
                    help="denoise path for the bf16 lines: the library's choice, the launch "
                         "chain, or the persistent whole-denoise kernel")
@@ -426,6 +428,68 @@ def run_reference(args, budget_s: float = 150.0):
     return 0
 
 
+def prefill_flops(pwl) -> float:
+    """Algorithmic FLOPs of one prefix prefill of every observation: 2 x MACs of the
+    projections (QKV in every layer; O, gate/up and down in all but the last, whose output
+    side feeds no K/V) and of Q K^T and P V over the whole prefix in all but the last layer."""
+    c = pwl.cfg
+    P, W, H, D, F, L = pwl.n_tokens, c.width, c.n_heads, c.head_dim, c.mlp_dim, c.n_layers
+    qkv = 2.0 * P * W * (H + 2) * D
+    rest = 2.0 * P * (H * D * W + 2 * F * W + F * W) + 4.0 * H * P * P * D
+    return pwl.batch * (L * qkv + (L - 1) * rest)
+
+
+def prefill_bytes(pwl) -> float:
+    """Algorithmic HBM bytes: every weight (bf16) once, the token embeddings and the K/V."""
+    c = pwl.cfg
+    P, W, H, D, F, L = pwl.n_tokens, c.width, c.n_heads, c.head_dim, c.mlp_dim, c.n_layers
+    w = L * W * (H + 2) * D + (L - 1) * (W * H * D + 3 * F * W)
+    return 2.0 * w + pwl.batch * (4.0 * P * W + 2.0 * 2 * L * P * D)
+
+
+def run_prefill_line(args, peaks, peak_src, ws, rank):
+    """The prefix prefill (Gemma-class language side over the 788 prefix tokens) timed on
+    the device: ms per prefill and its tensor-core roofline."""
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    from vla_inputs import PREFILL_WORKLOADS, make_prefill_params, make_prefill_tokens
+    pwl = PREFILL_WORKLOADS[args.prefill_workload]
+    pf = V.Prefill(pwl.cfg, make_prefill_params(pwl.cfg, pwl.seed), max_tokens=pwl.n_tokens, max_batch=pwl.batch)
+    tok = torch.from_numpy(make_prefill_tokens(pwl, seed=pwl.seed + rank)).cuda()
+    shape = (pwl.cfg.n_layers, pwl.batch, pwl.n_tokens, pwl.cfg.head_dim)
+    K = torch.empty(shape, dtype=torch.int16, device="cuda")
+    Vv = torch.empty(shape, dtype=torch.int16, device="cuda")
+    for _ in range(max(3, min(args.warmup, 5))):
+        pf.run(tok, K, Vv)
+    k = max(10, args.steps // 10)
+    s = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(k + 1)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    ev[0].record(s)
+    for i in range(k):
+        pf.run(tok, K, Vv)
+        ev[i + 1].record(s)
+    torch.cuda.synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(k)]
+    total = max_over_ranks(ev[0].elapsed_time(ev[k]), ws)
+    pf.status()
+    pf.close()
+    ms = total / k
+    fl, by = prefill_flops(pwl), prefill_bytes(pwl)
+    peak, peak_name = tensor_peak(peaks, None)
+    return {"workload": pwl.name,
+            "metric": f"ms per prefix prefill ({pwl.n_tokens} tokens, batch {pwl.batch}, "
+                      f"{pwl.cfg.n_layers} layers x width {pwl.cfg.width})",
+            "unit": "ms", "value": round(ms, 4), "steps": k,
+            "latency_ms": {"median": round(statistics.median(per), 4)},
+            "roofline": {"bound": "tensor", "achieved": round(fl / (ms * 1e-3) / 1e12, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(fl / (ms * 1e-3) / 1e12 / peak, 4),
+                         "algorithmic_flops": fl, "algorithmic_bytes": by,
+                         "hbm_ms": round(by / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
+                         "peak_source": f"{peak_src} ({peak_name})"}}
+
+
 def denoise_bytes(wl) -> float:
     """Algorithmic HBM bytes of one denoise: every projection weight (bf16) once per Euler
     step, the bf16 action in/out maps (and the Pi0 action-time MLP and state maps), and
@@ -565,6 +629,9 @@ def run_ours(args):
         del ex3
         torch.cuda.empty_cache()
 
+    prefill = None if args.no_prefill else run_prefill_line(args, peaks, peak_src, ws, rank)
+    torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         ms_cpu = OracleRunner(wl, inp, 1).ms()
@@ -595,6 +662,7 @@ def run_ours(args):
                                       "writes), the chunk's own K/V and padded QKV rows"},
             "secondary": secondary,
             "fp8": fp8,
+            "prefill": prefill,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": None if launches_per_denoise is None else launches_per_denoise * args.steps,

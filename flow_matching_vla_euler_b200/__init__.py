@@ -102,6 +102,10 @@ _SIGNATURES = {
     "vla_prefill_destroy": (None, [_P]),
     "vla_prefill_run": (_I, [_P, _P, _I, _I, _P, _P, _P]),
     "vla_prefill_status": (_I, [_P, _P]),
+    "vla_pipeline_create": (_I, [_P, _P, _I, ctypes.POINTER(_P)]),
+    "vla_pipeline_destroy": (None, [_P]),
+    "vla_pipeline_submit": (_I, [_P, _P, _I, _P]),
+    "vla_pipeline_step": (_I, [_P, _P, _P, _P, _P, _I, _P, _P]),
     "vla_last_error": (ctypes.c_char_p, []),
     "vla_version": (ctypes.c_char_p, []),
 }
@@ -186,6 +190,24 @@ def vla_prefill_run(h, tokens_ptr, n_tokens, batch, K_ptr, V_ptr, stream):
 
 def vla_prefill_status(h, stream):
     _check(load_library().vla_prefill_status(h, stream))
+
+
+def vla_pipeline_create(ex_h, pf_h, batch) -> int:
+    h = _P()
+    _check(load_library().vla_pipeline_create(ex_h, pf_h, batch, ctypes.byref(h)))
+    return h.value
+
+
+def vla_pipeline_destroy(h):
+    load_library().vla_pipeline_destroy(h)
+
+
+def vla_pipeline_submit(h, tokens_ptr, n_tokens, stream):
+    _check(load_library().vla_pipeline_submit(h, tokens_ptr, n_tokens, stream))
+
+
+def vla_pipeline_step(h, K_ptr, V_ptr, noise_ptr, state_ptr, steps, out_ptr, stream):
+    _check(load_library().vla_pipeline_step(h, K_ptr, V_ptr, noise_ptr, state_ptr, steps, out_ptr, stream))
 
 
 def vla_device_status(h, stream):
@@ -306,6 +328,42 @@ class Prefill:
 
     def status(self):
         vla_prefill_status(self.handle, _stream())
+
+
+class Pipeline:
+    """Asynchronous prefill / denoise pipeline over an Expert and a Prefill of the same
+    layer count and head_dim (the caller keeps both alive while the pipeline exists)."""
+
+    def __init__(self, expert, prefill, batch: int = 1):
+        self.expert, self.prefill, self.batch = expert, prefill, batch
+        self.handle = vla_pipeline_create(expert.handle, prefill.handle, batch)
+
+    def submit(self, tokens):
+        """tokens: CUDA fp32 [batch, n_tokens, width] (kept alive by the caller until the
+        next step)."""
+        vla_pipeline_submit(self.handle, _dev_ptr(tokens, 4), int(tokens.shape[1]), _stream())
+
+    def step(self, noise, state=None, steps: int = 10, out=None, K_tok=None, V_tok=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(noise)
+        kp = 0 if K_tok is None else _dev_ptr(K_tok, 2)
+        vp = 0 if V_tok is None else _dev_ptr(V_tok, 2)
+        sp = 0 if state is None else _dev_ptr(state, 4)
+        vla_pipeline_step(self.handle, kp or None, vp or None, _dev_ptr(noise, 4), sp or None, steps,
+                          _dev_ptr(out, 4), _stream())
+        return out
+
+    def close(self):
+        if getattr(self, "handle", None):
+            vla_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class Expert:

@@ -1817,3 +1817,4 @@ int vla_gemm_status(void* cuda_stream) {
 }  // extern "C"
 
 #include "prefill_api.cuh"   // the prefix prefill handle, sharing this file's helpers
+#include "pipeline_api.cuh"  // the asynchronous prefill / denoise pipeline over both handles

@@ -399,6 +399,39 @@ VLA_API int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, i
  * VLA_OK or VLA_ERR_TIMEOUT (a run's K/V are then not valid), or VLA_ERR_CUDA. */
 VLA_API int vla_prefill_status(vla_prefill* h, void* cuda_stream);
 
+/* ------------------------------------------------------------- asynchronous pipeline
+ *
+ * Reflex abstract: an async pipeline decouples visual encoding from action generation (the
+ * static region of the context depends on the observation only). vla_pipeline_submit
+ * prefills a new observation on the pipeline's own stream into one of two K/V banks and
+ * returns; the next vla_pipeline_step on the caller's stream waits for it on the device (an
+ * event), copies it into the expert's static region, applies the tick's sliding token and
+ * denoises. Steps between submissions reuse the current prefix; a submission that a newer
+ * one overtakes before the next step is dropped. The pipeline uses (but does not own) the
+ * two handles: while it exists, the prefill handle must not be run elsewhere and the
+ * expert must be driven only through it. Results equal the sequential prefill, set-prefix,
+ * append and denoise calls bit for bit.
+ */
+typedef struct vla_pipeline vla_pipeline;   /* opaque, owned by the library */
+
+/* ex and pf must agree on n_layers, head_dim and rope_base; batch within both handles'
+ * max_batch. Allocates two banks of [L][batch][min(pf max_tokens, ex n_static_max)][D] bf16.
+ * Errors: VLA_ERR_ARG, VLA_ERR_SHAPE, VLA_ERR_OOM, VLA_ERR_CUDA. */
+VLA_API int vla_pipeline_create(vla_expert* ex, vla_prefill* pf, int batch, vla_pipeline** out);
+VLA_API void vla_pipeline_destroy(vla_pipeline* p);
+
+/* tokens: DEVICE fp32 [batch][n_tokens][W of the prefill] as cuda_stream leaves them (the
+ * pipeline's stream waits for cuda_stream at this point); n_tokens in [1, bank capacity].
+ * Asynchronous; the caller keeps tokens valid until the next vla_pipeline_step returns. */
+VLA_API int vla_pipeline_submit(vla_pipeline* p, const float* tokens, int n_tokens, void* cuda_stream);
+
+/* One control tick on cuda_stream: swap in the last submitted observation if any, append
+ * the sliding token (K_tok, V_tok DEVICE bf16 [L][batch][D], both NULL for none) and
+ * denoise (arguments as vla_denoise). Errors as those calls; VLA_ERR_STATE if no prefix
+ * has been set yet. */
+VLA_API int vla_pipeline_step(vla_pipeline* p, const uint16_t* K_tok, const uint16_t* V_tok, const float* noise,
+                              const float* state, int steps, float* out_actions, void* cuda_stream);
+
 /* Message of the last failed call on this thread ("" if none). Valid until the next call. */
 VLA_API const char* vla_last_error(void);
 

@@ -100,6 +100,10 @@ def test_prefill_create_rejects_bad_arguments_before_any_cuda_call(lib):
     assert lib.vla_prefill_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
     assert lib.vla_prefill_run(None, None, 1, 1, None, None, None) == V.VLA_ERR_ARG
     assert lib.vla_prefill_status(None, None) == V.VLA_ERR_ARG
+    out = ctypes.c_void_p()
+    assert lib.vla_pipeline_create(None, None, 1, ctypes.byref(out)) == V.VLA_ERR_ARG
+    assert lib.vla_pipeline_submit(None, None, 1, None) == V.VLA_ERR_ARG
+    assert lib.vla_pipeline_step(None, None, None, None, None, 1, None, None) == V.VLA_ERR_ARG
 
 
 def test_weight_fields_cover_generator_names():
