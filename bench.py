@@ -449,7 +449,8 @@ def prefill_bytes(pwl) -> float:
 
 def run_prefill_line(args, peaks, peak_src, ws, rank):
     """The prefix prefill (Gemma-class language side over the 788 prefix tokens) timed on
-    the device: ms per prefill and its tensor-core roofline."""
+    the device: ms per prefill and its tensor-core roofline; then the asynchronous
+    pipeline against the same work done call after call (a new observation every tick)."""
     import torch
     import flow_matching_vla_euler_b200 as V
     from vla_inputs import PREFILL_WORKLOADS, make_prefill_params, make_prefill_tokens
@@ -474,6 +475,7 @@ def run_prefill_line(args, peaks, peak_src, ws, rank):
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(k)]
     total = max_over_ranks(ev[0].elapsed_time(ev[k]), ws)
     pf.status()
+    pipe = run_pipeline(args, pf, tok, ws, rank)
     pf.close()
     ms = total / k
     fl, by = prefill_flops(pwl), prefill_bytes(pwl)
@@ -487,7 +489,61 @@ def run_prefill_line(args, peaks, peak_src, ws, rank):
                          "unit": "TFLOP/s", "frac": round(fl / (ms * 1e-3) / 1e12 / peak, 4),
                          "algorithmic_flops": fl, "algorithmic_bytes": by,
                          "hbm_ms": round(by / (peaks["hbm_gbs"] * 1e9) * 1e3, 4),
-                         "peak_source": f"{peak_src} ({peak_name})"}}
+                         "peak_source": f"{peak_src} ({peak_name})"},
+            "pipeline": pipe}
+
+
+def run_pipeline(args, pf, tok, ws, rank):
+    """Control ticks of the 3-view Pi05 expert with a new 788-token observation every tick:
+    prefill, set-prefix and denoise one after another, against vla_pipeline (the prefill of
+    tick t + 1's observation overlaps tick t's denoise). Device time per tick, max over ranks."""
+    import torch
+    import flow_matching_vla_euler_b200 as V
+    from vla_inputs import get, make_inputs
+    wl = get(args.workload)
+    if wl.batch != 1 or wl.n_static < tok.shape[1]:
+        return None
+    inp = make_inputs(wl, seed=wl.seed + rank)
+    ex, noise, state = build_expert(wl, inp)
+    k = max(10, args.steps // 10)
+    s = torch.cuda.current_stream()
+    out = torch.empty_like(noise)
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for i in range(k):
+            fn(i)
+        e1.record(s)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), ws) / k
+
+    def sequential(i):
+        K, Vv = pf.run(tok)
+        ex.set_prefix(K, Vv)
+        ex.denoise(noise, state, wl.steps, out)
+
+    pl = V.Pipeline(ex, pf, batch=1)
+    camera = torch.cuda.Stream()   # where the observations come from (already resident here)
+    pl.submit(tok, stream=camera)
+
+    def pipelined(i):
+        pl.step(noise, state, wl.steps, out)   # tick i on the previous observation ...
+        pl.submit(tok, stream=camera)          # ... while the next one is prefilled
+
+    seq_ms = timed(sequential)
+    pipe_ms = timed(pipelined)
+    torch.cuda.synchronize()
+    pl.close()
+    ex.device_status()
+    ex.close()
+    return {"workload": f"{wl.name} + {args.prefill_workload}, a new observation every tick",
+            "metric": "ms per control tick (prefill + denoise)", "unit": "ms",
+            "sequential": round(seq_ms, 4), "pipelined": round(pipe_ms, 4), "ticks": k}
 
 
 def denoise_bytes(wl) -> float:

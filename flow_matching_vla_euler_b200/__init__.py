@@ -338,10 +338,13 @@ class Pipeline:
         self.expert, self.prefill, self.batch = expert, prefill, batch
         self.handle = vla_pipeline_create(expert.handle, prefill.handle, batch)
 
-    def submit(self, tokens):
+    def submit(self, tokens, stream=None):
         """tokens: CUDA fp32 [batch, n_tokens, width] (kept alive by the caller until the
-        next step)."""
-        vla_pipeline_submit(self.handle, _dev_ptr(tokens, 4), int(tokens.shape[1]), _stream())
+        next step), ready once ``stream`` (a torch.cuda.Stream; default the current one)
+        reaches this point. Submitting from a stream other than the one the steps run on
+        lets the prefill overlap the step already enqueued there."""
+        sp = _stream() if stream is None else stream.cuda_stream
+        vla_pipeline_submit(self.handle, _dev_ptr(tokens, 4), int(tokens.shape[1]), sp)
 
     def step(self, noise, state=None, steps: int = 10, out=None, K_tok=None, V_tok=None):
         import torch

@@ -421,8 +421,10 @@ VLA_API int vla_pipeline_create(vla_expert* ex, vla_prefill* pf, int batch, vla_
 VLA_API void vla_pipeline_destroy(vla_pipeline* p);
 
 /* tokens: DEVICE fp32 [batch][n_tokens][W of the prefill] as cuda_stream leaves them (the
- * pipeline's stream waits for cuda_stream at this point); n_tokens in [1, bank capacity].
- * Asynchronous; the caller keeps tokens valid until the next vla_pipeline_step returns. */
+ * pipeline's stream waits for cuda_stream at this point: pass the stream that produced the
+ * tokens, not the one the steps run on, or the prefill waits for the step enqueued there);
+ * n_tokens in [1, bank capacity]. Asynchronous; the caller keeps tokens valid until the
+ * next vla_pipeline_step returns. */
 VLA_API int vla_pipeline_submit(vla_pipeline* p, const float* tokens, int n_tokens, void* cuda_stream);
 
 /* One control tick on cuda_stream: swap in the last submitted observation if any, append
