@@ -1197,12 +1197,12 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if (h->persist_ok) {
     h->p_max_clusters = max_clusters;
     h->np = 2 + 2 * (h->pi0 ? 1 : 0) + 5 * L;
-    // Clusters of kPersistCluster CTAs (the projection splits of a tile then sum through
-    // distributed shared memory) when the device holds enough of them and every projection
-    // fits one round; otherwise one CTA per SM with the splits summed through global memory.
-    // VLA_PERSIST_CLUSTER=1 forces the latter (diagnostics).
+    // One CTA per SM with the projection splits summed through global memory (measured
+    // faster: 12.0 against 14.1 ms per Pi05 denoise); VLA_PERSIST_CLUSTER=8 (diagnostics)
+    // selects clusters of kPersistCluster CTAs, the splits of a tile then summing through
+    // distributed shared memory, when the device holds enough clusters.
     const char* env = getenv("VLA_PERSIST_CLUSTER");
-    const bool want = !(env && atoi(env) == 1);
+    const bool want = env && atoi(env) == kPersistCluster;
     h->p_cs = 1;
     if (want && max_clusters * kPersistCluster >= (h->sm_count * 3) / 4) {
       // each projection sums its splits through DSMEM when its tiles fit one round of the

@@ -313,3 +313,24 @@ def test_error_paths_on_device():
         ex.append_sliding(kt, kt)            # no sliding region
     assert e.value.code == V.VLA_ERR_STATE
     ex.device_status()
+
+
+def test_persistent_kernel_cluster_mode_matches_oracle():
+    """The persistent kernel with clusters of 8 CTAs (projection splits summed through
+    distributed shared memory; VLA_PERSIST_CLUSTER=8) on the 3-view Pi05 denoise."""
+    import os
+    import flow_matching_vla_euler_b200 as V
+    wl = get("pi05_3view")
+    inp = make_inputs(wl)
+    os.environ["VLA_PERSIST_CLUSTER"] = "8"
+    try:
+        ex, _ = make_expert(wl, inp, flags=V.VLA_FLAG_PERSIST)
+    finally:
+        del os.environ["VLA_PERSIST_CLUSTER"]
+    info = V.vla_persist_info(ex.handle)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    assert np.array_equal(run(ex, inp, wl.steps), got)
+    ex.device_status()
+    ex.close()
+    check_actions(got, oracle_actions(wl, inp), f"pi05_3view persistent, clusters {info}")
