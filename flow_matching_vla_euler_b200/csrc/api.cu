@@ -281,6 +281,8 @@ struct vla_expert {
   CUtensorMap tm_wqkv, tm_wo, tm_wgu, tm_wdown, tm_w1a, tm_w2;
   CUtensorMap tm_resid;              // fp32 residual [max_M][W], boxes of 128 x 32
   CUtensorMap tm_q, tm_kc, tm_vt;   // tensor-core attention operands (head_dim 256)
+  CUtensorMap tm_kc2, tm_vt2;       // the same for the CTA-pair kernel (half blocks)
+  bool attn_pair = false;           // CTA-pair attention (VLA_ATTN_PAIR=1; measured slower)
   CUtensorMap tm_qa, tm_ka, tm_va;  // split-KV attention operands (any head_dim)
 
   // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
@@ -744,7 +746,10 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
             t.scale_log2 = a.scale_log2;
             t.err = h->err;
             t.trace = tr(1);
-            CU(launch_attention_tc(h->tm_q, h->tm_kc, h->tm_vt, t, B, rec.s, pdl));
+            if (h->attn_pair && cdiv(h->S * h->H, attn_tc_q_tile()) % 2 == 0)
+              CU(launch_attention_tc2(h->tm_q, h->tm_kc2, h->tm_vt2, t, B, rec.s, pdl));
+            else
+              CU(launch_attention_tc(h->tm_q, h->tm_kc, h->tm_vt, t, B, rec.s, pdl));
           } else {
             CU(launch_attention(h->D, h->tm_qa, h->tm_ka, h->tm_va, a, B, ap.q_tiles, rec.s, pdl));
           }
@@ -1018,6 +1023,9 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   h->max_M = cfg->max_batch * h->S;
   h->gemm_cluster = gemm_max_cluster();
   h->attn_cluster = attn_max_cluster(h->D);
+  // diagnostics: VLA_GEMM_MAX_CLUSTER / VLA_ATTN_MAX_CLUSTER cap the split clusters
+  if (const char* e = getenv("VLA_GEMM_MAX_CLUSTER")) h->gemm_cluster = std::max(1, std::min(h->gemm_cluster, atoi(e)));
+  if (const char* e = getenv("VLA_ATTN_MAX_CLUSTER")) h->attn_cluster = std::max(1, std::min(h->attn_cluster, atoi(e)));
   const int L = h->L, W = h->W, H = h->H, D = h->D, F = h->F, DH = D / 2;
 
   auto cleanup = [&](int code) {
@@ -1302,6 +1310,12 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     if ((rc = make_tmap(&h->tm_q, h->qb, D, static_cast<uint64_t>(h->max_M) * H, 128))) return cleanup(rc);
     if ((rc = make_tmap(&h->tm_kc, h->kc, D, rows * h->kcap, 64))) return cleanup(rc);
     if ((rc = make_tmap(&h->tm_vt, h->vtc, h->kcap, rows * D, 256))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_kc2, h->kc, D, rows * h->kcap, 32))) return cleanup(rc);
+    if ((rc = make_tmap(&h->tm_vt2, h->vtc, h->kcap, rows * D, 128))) return cleanup(rc);
+    // diagnostics: VLA_ATTN_PAIR=1 selects the CTA-pair attention where the query tiles pair
+    // up (38.9 against 36.9 ms per batch-64 denoise: the per-block chain, not the key / value
+    // traffic, sets the pace)
+    if (const char* e = getenv("VLA_ATTN_PAIR")) h->attn_pair = atoi(e) != 0;
     CU(configure_attention_tc_kernel());
   }
   if (h->pi0) {

@@ -137,6 +137,10 @@ struct AttnTcParams {
 };
 cudaError_t launch_attention_tc(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_vt,
                                 const AttnTcParams& p, int batch, cudaStream_t s, bool pdl);
+// CTA-pair variant (even query-tile count): tm_k2 boxes of 32 keys x 64 dims, tm_vt2 boxes
+// of 128 dims x 64 keys; clusters of 2 query tiles of one observation.
+cudaError_t launch_attention_tc2(const CUtensorMap& tm_q, const CUtensorMap& tm_k2, const CUtensorMap& tm_vt2,
+                                 const AttnTcParams& p, int batch, cudaStream_t s, bool pdl);
 cudaError_t configure_attention_tc_kernel();
 int attn_tc_q_tile();
 

@@ -191,10 +191,13 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
   const bool tc = D == 256;
   const uint64_t kv_rows = static_cast<uint64_t>(L) * B * P;
   CUtensorMap tq, tk, tv;
+  // CTA-pair attention only on request (VLA_ATTN_PAIR=1), as for the expert
+  const char* pe = getenv("VLA_ATTN_PAIR");
+  const bool pair = tc && pe && atoi(pe) != 0 && cdiv(P * H, attn_tc_q_tile()) % 2 == 0;
   if (tc) {
     if ((rc = make_tmap(&tq, h->qb, D, static_cast<uint64_t>(M) * H, 128))) return rc;
-    if ((rc = make_tmap(&tk, Kc, D, kv_rows, 64))) return rc;
-    if ((rc = make_tmap(&tv, h->vtc, h->kcap_t, static_cast<uint64_t>(L) * B * D, 256))) return rc;
+    if ((rc = make_tmap(&tk, Kc, D, kv_rows, pair ? 32 : 64))) return rc;
+    if ((rc = make_tmap(&tv, h->vtc, h->kcap_t, static_cast<uint64_t>(L) * B * D, pair ? 128 : 256))) return rc;
   } else {
     const uint32_t bc = static_cast<uint32_t>(attn_box_cols(D)), kt = static_cast<uint32_t>(attn_key_tile(D));
     if ((rc = make_tmap(&tq, h->qb, D, static_cast<uint64_t>(M) * H, attn_q_tile(), bc))) return rc;
@@ -249,7 +252,8 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
       t.has_state = 0;
       t.scale_log2 = scale_log2;
       t.err = h->err;
-      CU(launch_attention_tc(tq, tk, tv, t, B, s, true));
+      if (pair) CU(launch_attention_tc2(tq, tk, tv, t, B, s, true));
+      else CU(launch_attention_tc(tq, tk, tv, t, B, s, true));
     } else {
       AttnParams a{};
       a.out = h->ob;

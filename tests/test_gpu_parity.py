@@ -334,3 +334,28 @@ def test_persistent_kernel_cluster_mode_matches_oracle():
     ex.device_status()
     ex.close()
     check_actions(got, oracle_actions(wl, inp), f"pi05_3view persistent, clusters {info}")
+
+
+def test_cta_pair_attention_matches_single_cta_attention():
+    """The CTA-pair tensor-core attention (VLA_ATTN_PAIR=1: two query tiles of an
+    observation share each key / value block, MMAs with M = 256) against the single-CTA
+    kernel on 37 observations of the 3-view Pi05 denoise (148 query tiles), and against the
+    oracle on observation 0."""
+    import os
+    from dataclasses import replace
+    wl = replace(get("pi05_3view_b64"), batch=37)
+    inp = make_inputs(wl)
+    inp = dict(inp, noise=inp["noise"][:37], prefix_k=inp["prefix_k"][:, :37], prefix_v=inp["prefix_v"][:, :37])
+    outs = []
+    for pair in ("0", "1"):
+        os.environ["VLA_ATTN_PAIR"] = pair
+        try:
+            ex, _ = make_expert(wl, inp)
+        finally:
+            del os.environ["VLA_ATTN_PAIR"]
+        load_prefix(ex, inp)
+        outs.append(run(ex, inp, wl.steps))
+        ex.device_status()
+        ex.close()
+    check_actions(outs[1], outs[0], "pair vs single attention, 37 observations")
+    check_actions(outs[1][:1], oracle_actions(wl, inp, batch_idx=[0]), "pair attention, observation 0")

@@ -51,8 +51,11 @@ def test_prefill_matches_oracle(name):
 
 
 @pytest.mark.gpu
-def test_prefill_fewer_tokens_and_observations_than_allocated():
-    """A handle sized for 130 tokens x 2 observations runs 77 tokens x 1 observation."""
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_prefill_fewer_tokens_and_observations_than_allocated(pair):
+    """A handle sized for 130 tokens x 2 observations runs 77 tokens x 1 observation (two
+    query tiles: with VLA_ATTN_PAIR=1 through the CTA-pair attention)."""
+    import os
     import torch
     import flow_matching_vla_euler_b200 as V
     from dataclasses import replace
@@ -60,7 +63,11 @@ def test_prefill_fewer_tokens_and_observations_than_allocated():
     params = make_prefill_params(wl.cfg, wl.seed)
     tokens = make_prefill_tokens(replace(wl, batch=1, n_tokens=77), seed=5)
     pf = V.Prefill(wl.cfg, params, max_tokens=wl.n_tokens, max_batch=wl.batch)
-    K, V_ = pf.run(torch.from_numpy(tokens).cuda())
+    os.environ["VLA_ATTN_PAIR"] = pair
+    try:
+        K, V_ = pf.run(torch.from_numpy(tokens).cuda())
+    finally:
+        del os.environ["VLA_ATTN_PAIR"]
     torch.cuda.synchronize()
     pf.status()
     Kr, Vr = O.prefill_batch(wl.cfg, O.decode_params(params), tokens.astype(np.float64))
