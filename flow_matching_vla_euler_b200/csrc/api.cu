@@ -398,8 +398,6 @@ int validate(const vla_config* c, const vla_weights* w) {
     return fail(VLA_ERR_ARG, "unknown flag bits 0x%x", c->flags);
   if ((c->flags & VLA_FLAG_PERSIST) && (c->flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS)))
     return fail(VLA_ERR_ARG, "VLA_FLAG_PERSIST contradicts VLA_FLAG_NO_PERSIST / VLA_FLAG_NORM_KERNELS");
-  if ((c->flags & VLA_FLAG_FP8_WEIGHTS) && (c->flags & (VLA_FLAG_NO_PERSIST | VLA_FLAG_NORM_KERNELS)))
-    return fail(VLA_ERR_UNSUPPORTED, "FP8 weights run on the persistent one-tile path only");
   if ((c->flags & VLA_FLAG_FP8_WEIGHTS) &&
       !(w->wq_scale && w->wk_scale && w->wv_scale && w->wo_scale && w->w_gate_scale && w->w_up_scale &&
         w->w_down_scale))
@@ -701,6 +699,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.head_dim = h->D;
           p.rope = h->rope;
           p.trace = tr(0);
+          if (h->fp8) p.wscale = h->sc_qkv + static_cast<size_t>(l) * h->qkv_rows;
           if (fused) {
             p.rstat_in = h->rstat_a;
             p.rstat_n = n_a;
@@ -760,6 +759,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           o.ld_resid = W;
           o.vec = gate;
           o.trace = tr(2);
+          if (h->fp8) o.wscale = h->sc_o + static_cast<size_t>(l) * W;
           if (fused) {
             o.rstat_out = h->rstat_b;
             o.zout = h->hb;
@@ -773,6 +773,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.out = h->ub;
           p.ld_out = h->F;
           p.trace = tr(3);
+          if (h->fp8) p.wscale = h->sc_gu + static_cast<size_t>(l) * 2 * h->F;
           if (fused) {
             p.rstat_in = h->rstat_b;
             p.rstat_n = n_o;
@@ -787,6 +788,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           d.ld_resid = W;
           d.vec = gate;
           d.trace = tr(4);
+          if (h->fp8) d.wscale = h->sc_down + static_cast<size_t>(l) * W;
           if (fused) {
             d.rstat_out = h->rstat_a;
             d.zout = l + 1 < L ? h->hb : nullptr;
@@ -844,7 +846,7 @@ int make_act_maps(vla_expert* h, int B, ActMaps* am) {
 }
 
 bool use_persist(const vla_expert* h, int B) {
-  return h->persist_ok && B <= h->persist_bmax && (h->fp8 || (h->cfg.flags & VLA_FLAG_PERSIST));
+  return h->persist_ok && B <= h->persist_bmax && (h->cfg.flags & VLA_FLAG_PERSIST);
 }
 
 void persist_params(const vla_expert* h, int B, int steps, int slot, PersistParams* pp) {
@@ -1196,7 +1198,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   // ---- persistent whole-denoise kernel (batches whose suffix tokens fit one 64-token tile)
   h->persist_bmax = std::min(cfg->max_batch, 64 / h->S);
   int max_clusters = 0;
-  const bool want_persist = h->fp8 || (cfg->flags & VLA_FLAG_PERSIST);
+  const bool want_persist = (cfg->flags & VLA_FLAG_PERSIST) != 0;
   if (h->persist_bmax >= 1 && want_persist) {
     int per_sm = 0;
     CU(configure_denoise_persist(D, &per_sm, kPersistCluster, &max_clusters));
@@ -1267,7 +1269,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
         (rc = dalloc(h, &h->p_trace, static_cast<size_t>(h->np) * G * 16)))
       return cleanup(rc);
   }
-  if (h->fp8 && !(h->persist_ok && h->persist_bmax >= cfg->max_batch))
+  if (h->fp8 && cfg->max_batch * h->S > 64)
     return cleanup(fail(VLA_ERR_UNSUPPORTED, "FP8 weights need max_batch x suffix <= 64 (got %d x %d)",
                         cfg->max_batch, h->S));
 

@@ -24,6 +24,8 @@
 // the status word and winds down.
 #include <cstdio>
 
+#include <cuda_fp8.h>
+
 #include "gemm_epi.cuh"
 
 namespace vla {
@@ -173,6 +175,44 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
   }
 }
 
+// FP8 (E4M3) weight tile, widened in place by four warps: 128 rows x 64 bytes (TMA, rows
+// 64 B apart) in the upper 8 KB of the 16 KB A stage become 128 rows x 64 bf16 in the MMA's
+// K-major layout with the 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)).
+// Every thread loads its row before any thread stores (the outputs of rows >= 64 overwrite
+// inputs of other warps), hence the named barrier between the two halves.
+__device__ __forceinline__ uint32_t e4m3x2_bf16x2(uint32_t two) {
+  const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two & 0xFFFFu), __NV_E4M3);
+  const float2 f = __half22float2(__half2(hr));
+  const __nv_bfloat162 b = __float22bfloat162_rn(f);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ void widen_tile_4warps(uint8_t* stage_a, int r) {
+  const uint8_t* in = stage_a + 8192 + r * 64;
+  uint4 q[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) q[c] = *reinterpret_cast<const uint4*>(in + c * 16);
+  named_bar_sync(2, 128);
+  uint8_t* out = stage_a + r * 128;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t w4[4] = {q[c].x, q[c].y, q[c].z, q[c].w};
+    uint4 lo, hi;   // elements 16c .. 16c + 7 and 16c + 8 .. 16c + 15
+    lo.x = e4m3x2_bf16x2(w4[0]);
+    lo.y = e4m3x2_bf16x2(w4[0] >> 16);
+    lo.z = e4m3x2_bf16x2(w4[1]);
+    lo.w = e4m3x2_bf16x2(w4[1] >> 16);
+    hi.x = e4m3x2_bf16x2(w4[2]);
+    hi.y = e4m3x2_bf16x2(w4[2] >> 16);
+    hi.z = e4m3x2_bf16x2(w4[3]);
+    hi.w = e4m3x2_bf16x2(w4[3] >> 16);
+    *reinterpret_cast<uint4*>(out + (((2 * c) ^ (r & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(out + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
+  }
+  fence_proxy_async_smem();   // generic writes -> the MMA's operand reads
+  named_bar_sync(2, 128);
+}
+
 // Push-mode reduction, token tile 64: every CTA of the cluster has sent rows
 // [q*128/S, (q+1)*128/S) of its partial tile to CTA q (receive slots = the other ranks in
 // rank order); the owner sums its S partials in rank order (deterministic) and runs the
@@ -191,6 +231,8 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
   const int rp = etid % HALF, c0 = etid / HALF;
   const int lr0 = 2 * rp, fn0 = fbase + lr0;
   const bool folded = s_rinv != nullptr;
+  // FP8 weights: the per-output-row scale of the pair's two features
+  const float2 wsc = p.wscale ? *reinterpret_cast<const float2*>(p.wscale + fn0) : make_float2(1.0f, 1.0f);
   // per-feature operands
   float2 vec2 = make_float2(1.0f, 1.0f), zm2 = make_float2(0.0f, 0.0f), cv2 = make_float2(0.0f, 0.0f);
   if constexpr (RESID) {
@@ -239,6 +281,8 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
       v1 += src[4];
     }
     if (k == 0 && etid == 0) trace_stamp(p.trace, 12);
+    v0 *= wsc.x;
+    v1 *= wsc.y;
     const int m = m0 + c;
     if constexpr (RESID) {
       float ss = 0.0f;
@@ -350,12 +394,24 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t accf = smem_u32(&bar[2 * G::STAGES]);
   const uint32_t recv_bar = smem_u32(&bar[2 * G::STAGES + 1]);
   const int npre = min(nkb, stages);
+  // FP8 weights (push kernels only): 8 KB per A stage by TMA, widened to bf16 in place by
+  // warps 2..5 (idle until the epilogue), which then signal wfull[s] to the MMA warp
+  const bool fp8 = G::PUSH && p.wscale != nullptr;
+  const uint32_t a_bytes = fp8 ? 8192u : static_cast<uint32_t>(G::A_BYTES);
+  const uint32_t a_off = fp8 ? 8192u : 0u;
+  const uint32_t wfull0 = smem_u32(tmem_slot + 4 + 256);   // after the rinv staging
+  const uint32_t afull0 = wfull0 + 8 * G::STAGES;           // FP8: the weight bytes landed
+  // bytes the full barrier of a stage waits for (FP8: the activations only)
+  const uint32_t stage_tx = fp8 ? static_cast<uint32_t>(G::B_BYTES) : a_bytes + G::B_BYTES;
+  const uint32_t a_bar0 = fp8 ? afull0 : full0;
 
   if (threadIdx.x == 0) {
     trace_stamp(p.trace, 0);
     for (int s = 0; s < G::STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
+      mbar_init(wfull0 + 8 * s, 1);
+      mbar_init(afull0 + 8 * s, 1);
     }
     mbar_init(accf, 1);
     if (push) {
@@ -374,8 +430,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint64_t pol_w = p.w_stream ? policy_evict_first() : policy_evict_last();
     const int y_w = p.w_row0 + n_tile * G::BM;
     for (int i = 0; i < npre; ++i) {
-      mbar_arrive_expect_tx(full0 + 8 * i, G::STAGE_BYTES);
-      tma_load_2d(smem_u32(sA + i * G::A_BYTES), &tm_w, full0 + 8 * i, (kb0 + i) * G::BK, y_w, pol_w);
+      mbar_arrive_expect_tx(full0 + 8 * i, stage_tx);
+      if (fp8) mbar_arrive_expect_tx(afull0 + 8 * i, a_bytes);
+      tma_load_2d(smem_u32(sA + i * G::A_BYTES) + a_off, &tm_w, a_bar0 + 8 * i, (kb0 + i) * G::BK, y_w, pol_w);
     }
   }
   if (warp == 1) {
@@ -410,8 +467,9 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = npre; i < nkb; ++i) {
         const int s = i % stages;
         if (!mbar_wait(empty0 + 8 * s, ((i / stages) - 1) & 1, p.err)) break;
-        mbar_arrive_expect_tx(full0 + 8 * s, G::STAGE_BYTES);
-        tma_load_2d(smem_u32(sA + s * G::A_BYTES), &tm_w, full0 + 8 * s, (kb0 + i) * G::BK, y_w,
+        mbar_arrive_expect_tx(full0 + 8 * s, stage_tx);
+        if (fp8) mbar_arrive_expect_tx(afull0 + 8 * s, a_bytes);
+        tma_load_2d(smem_u32(sA + s * G::A_BYTES) + a_off, &tm_w, a_bar0 + 8 * s, (kb0 + i) * G::BK, y_w,
                     pol_w);
         tma_load_2d(smem_u32(sB + s * G::B_BYTES), &tm_x, full0 + 8 * s, (kb0 + i) * G::BK, y_x,
                     pol_x);
@@ -431,6 +489,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int i = 0; i < nkb; ++i) {
         const int s = i % stages;
         if (!mbar_wait(full0 + 8 * s, (i / stages) & 1, p.err)) break;
+        if (fp8 && !mbar_wait(wfull0 + 8 * s, (i / stages) & 1, p.err)) break;
         if (i == 0) trace_stamp(p.trace, 3);
         tc_fence_after();
         const uint64_t da = sdesc_k_sw128(smem_u32(sA + s * G::A_BYTES));
@@ -446,6 +505,21 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
     if (push) cluster_wait();
   } else {
+    if (fp8 && warp < 6) {
+      // warps 2..5 widen each FP8 weight stage as it lands (before the dependency wait:
+      // weights depend on no earlier kernel); one thread waits and broadcasts the outcome,
+      // so that the four warps always meet at the same named barriers
+      volatile int* s_wok = reinterpret_cast<volatile int*>(tmem_slot + 2);
+      const int rr = (warp - 2) * 32 + lane;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages;
+        if (warp == 2 && lane == 0) *s_wok = mbar_wait(afull0 + 8 * s, (i / stages) & 1, p.err) ? 1 : 0;
+        named_bar_sync(2, 128);
+        if (!*s_wok) break;
+        widen_tile_4warps(sA + s * G::A_BYTES, rr);
+        if (warp == 2 && lane == 0) mbar_arrive(wfull0 + 8 * s);
+      }
+    }
     pdl_wait();
     // warps 2..9: the push path uses all eight (two per TMEM lane quarter, each half of
     // the token columns); the other paths use warps 2..5 with whole rows

@@ -80,20 +80,18 @@ typedef enum vla_time_kind {
                                     VLA_FLAG_NO_PERSIST) */
 #define VLA_FLAG_NO_PERSIST 4u   /* never run the single persistent kernel: the denoise is
                                     one kernel launch per projection / attention / embed /
-                                    final step, captured in a graph (the default for bf16
-                                    weights; not combinable with VLA_FLAG_FP8_WEIGHTS) */
+                                    final step, captured in a graph (the default) */
 #define VLA_FLAG_FP8_WEIGHTS 8u  /* the projection matrices wq, wk, wv, wo, w_gate, w_up,
                                     w_down are FP8 E4M3 bytes with fp32 per-output-row scales
                                     (vla_weights *_scale); streamed as FP8 and widened to bf16
                                     in shared memory, exactly (InstinctFlash README: the pi05
-                                    FP8 configuration). Needs max_batch x suffix <= 64 (the
-                                    persistent one-tile path); not combinable with
-                                    VLA_FLAG_NO_PERSIST or VLA_FLAG_NORM_KERNELS. */
-#define VLA_FLAG_PERSIST 16u     /* with bf16 weights and one token tile (max_batch x suffix
-                                    <= 64), run the whole denoise loop as the single
-                                    persistent kernel instead of the launch chain (FP8
-                                    weights always use it). Ignored for larger batches;
-                                    not combinable with VLA_FLAG_NO_PERSIST. */
+                                    FP8 configuration). Needs max_batch x suffix <= 64 (one
+                                    token tile: the launch chain, or with VLA_FLAG_PERSIST the
+                                    persistent kernel). */
+#define VLA_FLAG_PERSIST 16u     /* with one token tile (max_batch x suffix <= 64), run the
+                                    whole denoise loop as the single persistent kernel
+                                    instead of the launch chain. Ignored for larger
+                                    batches; not combinable with VLA_FLAG_NO_PERSIST. */
 
 typedef struct vla_config {
   int n_layers;      /* L */

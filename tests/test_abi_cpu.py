@@ -144,12 +144,12 @@ def test_host_argument_checks(lib):
     assert "flag" in V.vla_last_error()
     assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_PERSIST | V.VLA_FLAG_NO_PERSIST)),
                                  ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
-    # FP8 weights: every scale pointer is required, and only the persistent one-tile path
+    # FP8 weights: every scale pointer is required (on either one-tile path)
     assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_FP8_WEIGHTS)), ctypes.byref(w),
                                  ctypes.byref(h)) == V.VLA_ERR_ARG
     assert "scale" in V.vla_last_error()
     assert lib.vla_expert_create(ctypes.byref(_cfg(flags=V.VLA_FLAG_FP8_WEIGHTS | V.VLA_FLAG_NO_PERSIST)),
-                                 ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_UNSUPPORTED
+                                 ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG   # scales still required
     # a valid shape with missing weights is an argument error, still before any CUDA call
     assert lib.vla_expert_create(ctypes.byref(_cfg()), ctypes.byref(w), ctypes.byref(h)) == V.VLA_ERR_ARG
     assert lib.vla_denoise(None, None, None, 4, None, 1, None) == V.VLA_ERR_ARG

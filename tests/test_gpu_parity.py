@@ -180,24 +180,28 @@ def test_persistent_kernel_matches_oracle_and_the_launch_chain(name, obs):
 
 
 @pytest.mark.parametrize("name", ["tiny_fp8", "mid_d128_fp8", "mid_pi0_b1_fp8", "pi05_3view_fp8"])
-def test_fp8_weights_match_oracle(name):
+@pytest.mark.parametrize("path", ["chain", "persistent"])
+def test_fp8_weights_match_oracle(name, path):
     """FP8 (E4M3, per-output-row fp32 scale) projection weights, streamed as bytes and
-    widened to bf16 in shared memory by the persistent kernel, against the oracle run on the
-    exact dequantised weights (E4M3 value x row scale, in fp64): the acceptance tolerance,
-    and bit-identical reruns."""
+    widened to bf16 in shared memory (by four warps of each chain GEMM, or by the persistent
+    kernel's widening warp), against the oracle run on the exact dequantised weights (E4M3
+    value x row scale, in fp64): the acceptance tolerance, and bit-identical reruns."""
+    import flow_matching_vla_euler_b200 as V
     wl = get(name)
-    ex, inp = make_expert(wl)
+    inp = make_inputs(wl)
+    ex, _ = make_expert(wl, inp, flags=V.VLA_FLAG_PERSIST if path == "persistent" else 0)
+    assert (V.vla_persist_info(ex.handle)["ctas"] > 0) == (path == "persistent")
     load_prefix(ex, inp)
     got = run(ex, inp, wl.steps)
-    check_actions(got, oracle_actions(wl, inp), name)
+    check_actions(got, oracle_actions(wl, inp), f"{name} {path}")
     assert np.array_equal(run(ex, inp, wl.steps), got)
     ex.device_status()
     ex.close()
 
 
 def test_fp8_weights_need_one_token_tile():
-    """FP8 weights run on the persistent one-tile path only: a handle whose largest batch
-    does not fit one 64-token tile is refused."""
+    """FP8 weights run with one token tile only: a handle whose largest batch does not fit
+    one 64-token tile is refused."""
     import flow_matching_vla_euler_b200 as V
     wl = get("mid_pi0_b1_fp8")
     inp = make_inputs(wl)
