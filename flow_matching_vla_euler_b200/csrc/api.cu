@@ -283,6 +283,7 @@ struct vla_expert {
   CUtensorMap tm_q, tm_kc, tm_vt;   // tensor-core attention operands (head_dim 256)
   CUtensorMap tm_kc2, tm_vt2;       // the same for the CTA-pair kernel (half blocks)
   bool attn_pair = false;           // CTA-pair attention (VLA_ATTN_PAIR=1; measured slower)
+  bool vt_kernel = false;           // transposed V by its own kernel (VLA_VT_KERNEL=1, diagnostics)
   CUtensorMap tm_qa, tm_ka, tm_va;  // split-KV attention operands (any head_dim)
 
   // optional diagnostics: %globaltimer stamps of step 0, layer 0 (env VLA_TRACE_FILE)
@@ -691,7 +692,12 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           p.ld_out = h->HD;
           p.kc = h->kc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
           p.vc = h->vc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
-          p.vtc = nullptr;   // the transposed V of the chunk is written by launch_vt_dyn below
+          // the transposed V of the chunk (tensor-core attention only): written by the
+          // persistent QKV GEMM's epilogue (several token tiles, the only case that uses it)
+          p.vtc = use_tc_attn && M > 64 && !h->vt_kernel
+                      ? h->vtc + static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D
+                      : nullptr;
+          p.kcap_t = h->kcap;
           p.kcap = h->kcap;
           p.dyn_off = h->dyn_off;
           p.seq = h->S;
@@ -723,7 +729,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
           a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(h->D));
           a.err = h->err;
           a.trace = tr(1);
-          if (use_tc_attn) {   // transposed V of the chunk (counted with attention)
+          if (use_tc_attn && !p.vtc) {   // transposed V of the chunk (counted with attention)
             const size_t lofs = static_cast<size_t>(l) * h->cfg.max_batch * h->kcap * h->D;
             rec.begin(VLA_K_ATTN);
             CU(launch_vt_dyn(p.vc, h->vtc + lofs, B, h->D, h->kcap, h->kcap, h->dyn_off, h->S, rec.s, pdl));
@@ -1318,6 +1324,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     // up (38.9 against 36.9 ms per batch-64 denoise: the per-block chain, not the key / value
     // traffic, sets the pace)
     if (const char* e = getenv("VLA_ATTN_PAIR")) h->attn_pair = atoi(e) != 0;
+    if (const char* e = getenv("VLA_VT_KERNEL")) h->vt_kernel = atoi(e) != 0;
     CU(configure_attention_tc_kernel());
   }
   if (h->pi0) {

@@ -145,7 +145,8 @@ __device__ __forceinline__ void epi_apply(const GemmParams& p, float (&v)[16], i
         const size_t row = static_cast<size_t>(bj[j]) * p.kcap + p.dyn_off + sj[j];
         const bf16 o = __float2bfloat16_rn(v[j]);
         vrow[row * D] = o;
-        if (p.vtc) p.vtc[(static_cast<size_t>(bj[j]) * D + dim) * p.kcap + p.dyn_off + sj[j]] = o;
+        if (p.vtc)
+          p.vtc[(static_cast<size_t>(bj[j]) * D + dim) * (p.kcap_t > 0 ? p.kcap_t : p.kcap) + p.dyn_off + sj[j]] = o;
       }
       return;
     }
@@ -338,9 +339,10 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
           dst[i_q] = __float2bfloat16_rn(o0);
           dst[i_q + DH] = __float2bfloat16_rn(o1);
           if (kind == 2 && p.vtc) {
-            bf16* vt = p.vtc + static_cast<size_t>(b) * D * p.kcap + p.dyn_off + sq;
-            vt[static_cast<size_t>(i_q) * p.kcap] = __float2bfloat16_rn(o0);
-            vt[static_cast<size_t>(i_q + DH) * p.kcap] = __float2bfloat16_rn(o1);
+            const int kt = p.kcap_t > 0 ? p.kcap_t : p.kcap;
+            bf16* vt = p.vtc + static_cast<size_t>(b) * D * kt + p.dyn_off + sq;
+            vt[static_cast<size_t>(i_q) * kt] = __float2bfloat16_rn(o0);
+            vt[static_cast<size_t>(i_q + DH) * kt] = __float2bfloat16_rn(o1);
           }
         }
       } else {
@@ -769,6 +771,10 @@ __device__ __forceinline__ void qkv_epilogue_staged(const GemmParams& p, uint32_
   const float2* rope = reinterpret_cast<const float2*>(p.rope) + i;
   const int pos = (second ? 80 : 0) + (r >> 1);
   const float cv = s_rinv && p.cvec ? p.cvec[n_tile * G::BM + r] : 0.0f;
+  // tiles holding V pairs also write the transposed V cache, when there is one
+  const int kcap_t = p.kcap_t > 0 ? p.kcap_t : p.kcap;
+  const bool vt_tile = p.vtc != nullptr && n_tile * (G::BM / 2) < (H + 2) * DH &&
+                       (n_tile + 1) * (G::BM / 2) > (H + 1) * DH;
   // rotary cos/sin of the next step's tokens are fetched while this step is applied
   float2 cs[16];
   if (kind < 2) {
@@ -821,12 +827,23 @@ __device__ __forceinline__ void qkv_epilogue_staged(const GemmParams& p, uint32_
       bf16* dst = k0 == 0 ? p.out + static_cast<size_t>(m) * p.ld_out + head * D + dim0
                           : (k0 == 1 ? p.kc : p.vc) + static_cast<size_t>(tok_kv[col]) * D + dim0;
       *reinterpret_cast<uint4*>(dst) = val;
-      if (k0 == 2 && p.vtc) {   // transposed V cache column (not used on the denoise path)
-        const bf16* e = reinterpret_cast<const bf16*>(&val);
-        const int bq = (m / p.seq);
-        bf16* vt = p.vtc + static_cast<size_t>(bq) * D * p.kcap + (tok_kv[col] - bq * p.kcap);
-#pragma unroll
-        for (int x = 0; x < 8; ++x) vt[static_cast<size_t>(dim0 + x) * p.kcap] = e[x];
+    }
+    if (vt_tile) {
+      // transposed V cache columns vtc[obs][dim][dyn_off + s] (the tensor-core attention's
+      // V operand): one token per lane, so a warp writes 32 consecutive positions of a dim;
+      // warps take every eighth dim of the tile
+      const int col = (lane >> 4) * (TN / 2) + st * 16 + (lane & 15);
+      const int m = m0 + col;
+      if (m < p.m_tok) {
+        const int bq = m / p.seq, sq = m - bq * p.seq;
+        bf16* vt_tok = p.vtc + static_cast<size_t>(bq) * D * kcap_t + p.dyn_off + sq;
+        const bf16* srow = stage + (st & 1) * 32 * RSTR + lane * RSTR;
+        for (int dl = ew; dl < G::BM; dl += 8) {
+          const int hf = dl >> 6, lp = dl & 63;
+          const int pr = n_tile * (G::BM / 2) + lp;
+          if (pr < (H + 1) * DH || pr >= (H + 2) * DH) continue;   // not a V pair
+          vt_tok[static_cast<size_t>(pr - (H + 1) * DH + hf * DH) * kcap_t] = srow[hf * 80 + lp];
+        }
       }
     }
   }

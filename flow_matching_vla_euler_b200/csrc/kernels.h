@@ -49,7 +49,8 @@ struct GemmParams {
   int ld_out;
   bf16* kc;           // EPI_QKV: this layer's K cache [max_batch][kcap][D]
   bf16* vc;
-  bf16* vtc;          // EPI_QKV: this layer's transposed V cache [max_batch][D][kcap], or null
+  bf16* vtc;          // EPI_QKV: this layer's transposed V cache [max_batch][D][kcap_t], or null
+  int kcap_t;         // positions per transposed-V row (0: kcap)
   int kcap, dyn_off, seq, n_heads, head_dim;
   const float* rope;  // [seq][D/2][2] (cos, sin) at positions pos0 + s
   int has_state;      // EPI_BIAS_STORE: skip row s == 0 of each observation

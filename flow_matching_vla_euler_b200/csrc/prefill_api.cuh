@@ -235,10 +235,14 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
     q.n_heads = H;
     q.head_dim = D;
     q.rope = h->rope;
+    // the transposed V for the tensor-core attention comes from the QKV epilogue
+    if (tc && l < L - 1) {
+      q.vtc = h->vtc + static_cast<size_t>(l) * B * D * h->kcap_t;
+      q.kcap_t = h->kcap_t;
+    }
     if ((rc = prefill_gemm(h, s, EPI_QKV, h->tm_wqkv, am_hb, q, h->qkv_rows, W, M, tn, true))) return rc;
     if (l == L - 1) break;   // the last layer's output side feeds no K/V
     if (tc) {
-      CU(launch_vt_dyn(q.vc, h->vtc + static_cast<size_t>(l) * B * D * h->kcap_t, B, D, P, h->kcap_t, 0, P, s, true));
       AttnTcParams t{};
       t.out = h->ob;
       t.cache = h->desc;
