@@ -1180,6 +1180,26 @@ __global__ void __launch_bounds__(320, 1)
             if (!(lane & 1)) srow[c + (lane >> 1)] = ss;
           }
         }
+      } else if constexpr (EPI == EPI_GEGLU) {
+        // 32 token columns per TMEM load and wait, two independent 16-column halves of math
+        const float cv = folded && p.cvec ? p.cvec[fn] : 0.0f;
+#pragma unroll 1
+        for (int c = c_begin; c < c_begin + TN / 2; c += 32) {
+          float w[32];
+          tmem_ld32(taddr + c, w);
+          if (folded) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) w[j] = fmaf(rinv_t[c + j], w[j], cv);
+          }
+          float v0[16], v1[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v0[j] = w[j];
+            v1[j] = w[16 + j];
+          }
+          epi_apply<EPI>(p, v0, fn, m0 + c, lane);
+          epi_apply<EPI>(p, v1, fn, m0 + c + 16, lane);
+        }
       } else {
         const float cv = folded && p.cvec ? p.cvec[fn] : 0.0f;
 #pragma unroll 1
