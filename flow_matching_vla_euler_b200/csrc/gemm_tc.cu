@@ -677,7 +677,7 @@ __global__ void __launch_bounds__(320, 1)
 // ---------------------------------------------------------------------------------
 // Persistent variant for several token tiles (no K split): one CTA per SM walks the
 // output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... with the token tile varying
-// fastest (the weight tile stays hot in L2 across token tiles). TMA keeps a 4-stage ring
+// fastest (the weight tile stays hot in L2 across token tiles). TMA keeps a ring of 4 to 6 stages
 // streaming across tile boundaries; the MMA warp alternates between two TMEM
 // accumulators, so the epilogue of one tile overlaps the main loop of the next.
 template <int TN>
@@ -686,7 +686,8 @@ struct PersistCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = TN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = TN == 128 ? 6 : 4;
+  // 192-token tiles (one tile per CTA, residual epilogue) have room for a fifth stage
+  static constexpr int STAGES = TN == 128 ? 6 : (TN == 192 ? 5 : 4);
   static constexpr int TMEM_COLS = TN == 192 ? 512 : 2 * TN;   // two accumulators (power of 2)
   // EPI_QKV stages its bf16 output through shared memory: two buffers of 32 token rows
   // (16 per column half) x QKV_RSTR elements, plus the tile's per-token table
