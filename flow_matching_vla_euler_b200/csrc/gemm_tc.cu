@@ -357,12 +357,13 @@ __device__ __forceinline__ void push_reduce(const GemmParams& p, const float* re
 // CL = true (TN = 64): the p.splits CTAs of a tile are one thread-block cluster; each
 // stages its partial tile in its own shared memory and pushes rows [r*128/S, (r+1)*128/S)
 // to CTA rank r, which sums the S partials in rank order (deterministic).
-template <int TN, int EPI, bool CL>
+template <int TN, int EPI, bool CL, bool F8>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                    const GemmParams p) {
   using G = GemmCfg<TN, CL>;
   static_assert(!CL || TN == 64, "cluster (split-K push) kernels take one 64-token tile");
+  static_assert(!F8 || G::PUSH, "FP8 weights only in the split-K push kernels");
   static_assert(!G::PUSH || G::push_need(1) <= 2 * G::STAGE_BYTES,
                 "the partial tile fits in two idle pipeline stages");
   extern __shared__ uint8_t smem_raw[];
@@ -396,9 +397,10 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t accf = smem_u32(&bar[2 * G::STAGES]);
   const uint32_t recv_bar = smem_u32(&bar[2 * G::STAGES + 1]);
   const int npre = min(nkb, stages);
-  // FP8 weights (push kernels only): 8 KB per A stage by TMA, widened to bf16 in place by
-  // warps 2..5 (idle until the epilogue), which then signal wfull[s] to the MMA warp
-  const bool fp8 = G::PUSH && p.wscale != nullptr;
+  // FP8 weights (push kernels only; an instantiation of its own, so that the bf16 kernels
+  // carry none of this code): 8 KB per A stage by TMA, widened to bf16 in place by warps
+  // 2..5 (idle until the epilogue), which then signal wfull[s] to the MMA warp
+  constexpr bool fp8 = F8;
   const uint32_t a_bytes = fp8 ? 8192u : static_cast<uint32_t>(G::A_BYTES);
   const uint32_t a_off = fp8 ? 8192u : 0u;
   const uint32_t wfull0 = smem_u32(tmem_slot + 4 + 256);   // after the rinv staging
@@ -1303,16 +1305,16 @@ static cudaError_t configure_persist_tn() {
   return cudaSuccess;
 }
 
-template <int TN, int EPI, bool CL>
+template <int TN, int EPI, bool CL, bool F8 = false>
 static cudaError_t configure_one() {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(GemmCfg<TN, CL>::SMEM));
   if (e == cudaSuccess && CL)
-    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL, F8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   // every kernel of the denoise chain asks for the largest shared-memory carve-out, so an
   // SM configured by one of them has room for a CTA of the next (PDL overlap)
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    e = cudaFuncSetAttribute(gemm_tc_kernel<TN, EPI, CL, F8>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared);
   return e;
 }
@@ -1325,6 +1327,12 @@ static cudaError_t configure_tn() {
   if ((e = configure_one<TN, EPI_GEGLU, CL>()) != cudaSuccess) return e;
   if ((e = configure_one<TN, EPI_SWISH_VEC, CL>()) != cudaSuccess) return e;
   if ((e = configure_one<TN, EPI_BIAS_STORE, CL>()) != cudaSuccess) return e;
+  if constexpr (CL && TN == 64) {
+    // FP8 weights: the projections of the expert's layers
+    if ((e = configure_one<TN, EPI_RESID, CL, true>()) != cudaSuccess) return e;
+    if ((e = configure_one<TN, EPI_QKV, CL, true>()) != cudaSuccess) return e;
+    if ((e = configure_one<TN, EPI_GEGLU, CL, true>()) != cudaSuccess) return e;
+  }
   return configure_one<TN, EPI_STORE, CL>();
 }
 
@@ -1366,14 +1374,14 @@ int gemm_max_cluster() {
     attr[0].val.clusterDim.z = c;
     cfg.gridDim = dim3(1, 1, c);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<64, EPI_RESID, true>, &cfg) == cudaSuccess && n > 0)
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<64, EPI_RESID, true, false>, &cfg) == cudaSuccess && n > 0)
       return c;
     cudaGetLastError();
   }
   return 1;
 }
 
-template <int TN, int EPI, bool CL>
+template <int TN, int EPI, bool CL, bool F8 = false>
 static cudaError_t launch_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const GemmParams& p,
                               int n_tiles, int m_tiles, cudaStream_t s, bool pdl) {
   using G = GemmCfg<TN, CL>;
@@ -1414,13 +1422,25 @@ static cudaError_t launch_one(const CUtensorMap& tm_w, const CUtensorMap& tm_x, 
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI, CL>, tm_w, tm_x, q);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<TN, EPI, CL, F8>, tm_w, tm_x, q);
 }
 
 template <int TN, bool CL>
 static cudaError_t launch_tn(int epi, const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                              const GemmParams& p, int n_tiles, int m_tiles, cudaStream_t s,
                              bool pdl) {
+  if (p.wscale) {
+    // FP8 weights: the split-K push kernels of the layer projections only
+    if constexpr (CL && TN == 64) {
+      switch (epi) {
+        case EPI_RESID: return launch_one<TN, EPI_RESID, CL, true>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+        case EPI_QKV: return launch_one<TN, EPI_QKV, CL, true>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+        case EPI_GEGLU: return launch_one<TN, EPI_GEGLU, CL, true>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+    return cudaErrorInvalidValue;
+  }
   switch (epi) {
     case EPI_RESID: return launch_one<TN, EPI_RESID, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
     case EPI_QKV: return launch_one<TN, EPI_QKV, CL>(tm_w, tm_x, p, n_tiles, m_tiles, s, pdl);
