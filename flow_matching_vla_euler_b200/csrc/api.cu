@@ -234,6 +234,7 @@ struct vla_expert {
   vla_config cfg;
   int dev = 0, sm_count = 148;
   int gemm_cluster = 1;   // largest split cluster of the 64-token push GEMM
+  int qkv_tn = 0;         // token tile of the persistent QKV GEMM (0: the plan's)
   int attn_cluster = 1;
   int L, W, H, D, F, A, C, Sd, S, hs, HD, Td, Cd, qkv_rows, kcap, ring_off, dyn_off, max_M;
   bool ada, pi0;
@@ -494,6 +495,7 @@ int ensure_tables(vla_expert* h, int steps, cudaStream_t s, int* slot_out) {
 
 struct ActMaps {
   CUtensorMap hb, ob, ub, eb, h1b;
+  CUtensorMap hb_qkv;   // the QKV projection's view of hb (its own token tile)
 };
 
 struct Recorder {
@@ -532,6 +534,10 @@ int persist_tn(int n_feat, int M, int sm_count, bool resid) {
   return cost(192) < cost(256) ? 192 : 256;
 }
 
+int qkv_tn(const vla_expert* h, int M) {
+  return h->qkv_tn ? h->qkv_tn : persist_tn(h->qkv_rows, M, h->sm_count, false);
+}
+
 GemmPlan denoise_plan(const vla_expert* h, int n_feat, int k_dim, int M) {
   const int tn = plan_gemm(n_feat, k_dim, M, h->sm_count).tn;
   return plan_gemm_cluster(n_feat, k_dim, M, h->sm_count, tn == 64 ? h->gemm_cluster : 1);
@@ -552,7 +558,7 @@ int enqueue_gemm(vla_expert* h, Recorder& rec, int kind, int epi, const CUtensor
     // the residual map only for the residual stream itself (rows M)
     const CUtensorMap* tr = (epi == EPI_RESID && p.resid == h->resid) ? &h->tm_resid : nullptr;
     GemmPlan g0 = plan_gemm(n_feat, k_dim, M, h->sm_count);
-    g0.tn = persist_tn(n_feat, M, h->sm_count, tr != nullptr);
+    g0.tn = kind == VLA_K_GEMM_QKV ? qkv_tn(h, M) : persist_tn(n_feat, M, h->sm_count, tr != nullptr);
     g0.m_tiles = cdiv(M, g0.tn);
     p.n_feat = n_feat;
     p.k_dim = k_dim;
@@ -712,7 +718,7 @@ int enqueue_denoise(vla_expert* h, int B, int steps, int slot, const ActMaps& am
             p.cvec = h->ada ? h->ctables[slot] + (static_cast<long>(k) * L + l) * cw : nullptr;
             p.eps = h->cfg.eps;
           }
-          int rc = enqueue_gemm(h, rec, VLA_K_GEMM_QKV, EPI_QKV, h->tm_wqkv, am.hb, p, h->qkv_rows, W, M, pdl);
+          int rc = enqueue_gemm(h, rec, VLA_K_GEMM_QKV, EPI_QKV, h->tm_wqkv, am.hb_qkv, p, h->qkv_rows, W, M, pdl);
           if (rc) return rc;
           AttnParams a{};
           a.layer = l;
@@ -839,6 +845,8 @@ int make_act_maps(vla_expert* h, int B, ActMaps* am) {
   const uint32_t tn_res = static_cast<uint32_t>(M > 64 ? persist_tn(h->W, M, h->sm_count, true) : tn);
   int rc;
   if ((rc = make_tmap(&am->hb, h->hb, h->W, M, tn))) return rc;
+  const uint32_t tn_qkv = static_cast<uint32_t>(M > 64 ? qkv_tn(h, M) : tn);
+  if ((rc = make_tmap(&am->hb_qkv, h->hb, h->W, M, tn_qkv))) return rc;
   if ((rc = make_tmap(&am->ob, h->ob, h->HD, M, tn_res))) return rc;
   if ((rc = make_tmap(&am->ub, h->ub, h->F, M, tn_res))) return rc;
   if (h->pi0) {
@@ -1034,6 +1042,11 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   // diagnostics: VLA_GEMM_MAX_CLUSTER / VLA_ATTN_MAX_CLUSTER cap the split clusters
   if (const char* e = getenv("VLA_GEMM_MAX_CLUSTER")) h->gemm_cluster = std::max(1, std::min(h->gemm_cluster, atoi(e)));
   if (const char* e = getenv("VLA_ATTN_MAX_CLUSTER")) h->attn_cluster = std::max(1, std::min(h->attn_cluster, atoi(e)));
+  // diagnostics: VLA_QKV_TN = 128 or 256 sets the persistent QKV GEMM's token tile
+  if (const char* e = getenv("VLA_QKV_TN")) {
+    const int v = atoi(e);
+    if (v == 128 || v == 256) h->qkv_tn = v;
+  }
   const int L = h->L, W = h->W, H = h->H, D = h->D, F = h->F, DH = D / 2;
 
   auto cleanup = [&](int code) {
