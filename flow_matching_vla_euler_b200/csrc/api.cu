@@ -534,6 +534,22 @@ int persist_tn(int n_feat, int M, int sm_count, bool resid) {
   return cost(192) < cost(256) ? 192 : 256;
 }
 
+// Token tile by rounds of n_feat / 128 x cdiv(M, t) tiles over the SMs: the candidate (128,
+// 256, and 192 for the residual projections) with the fewest token columns per CTA, where a
+// 128-token column costs 1.5 when its tiles take several rounds (the smaller tile's extra
+// operand traffic per FLOP, measured: 788 tokens, gate/up in 13 rounds of 128-token tiles
+// 5.13 ms per prefill against 4.38 ms in 7 rounds of 256). Ties go to the larger tile.
+int persist_tn_rounds(int n_feat, int M, int sm_count, bool resid) {
+  auto cost = [&](int t) {
+    const int rounds = cdiv((n_feat / 128) * cdiv(M, t), sm_count);
+    return t == 128 && rounds > 1 ? rounds * 192 : rounds * t;
+  };
+  int best = 256;
+  if (resid && cost(192) < cost(best)) best = 192;
+  if (cost(128) < cost(best)) best = 128;
+  return best;
+}
+
 int qkv_tn(const vla_expert* h, int M) {
   return h->qkv_tn ? h->qkv_tn : persist_tn(h->qkv_rows, M, h->sm_count, false);
 }

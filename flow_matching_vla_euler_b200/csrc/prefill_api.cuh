@@ -178,13 +178,16 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
   const int M = B * P;
   bf16* Kc = reinterpret_cast<bf16*>(K_out);
   bf16* Vc = reinterpret_cast<bf16*>(V_out);
-  // token tiles: at least 128 (the persistent GEMM), 192 for the residual projections
-  // when that fills the SMs better
-  const int tn = std::max(128, plan_gemm(128, 128, M, h->sm_count).tn);
-  const int tn_res = std::max(128, persist_tn(W, M, h->sm_count, true));
-  CUtensorMap am_hb, am_ob, am_ub;
+  // token tiles per projection, by rounds of tiles over the SMs (788 tokens: 128 for QKV, O
+  // and down, e.g. 140 QKV tiles in one round instead of 80 tiles of 256 tokens; 256 for
+  // gate/up, seven rounds)
+  const int tn_qkv = persist_tn_rounds(h->qkv_rows, M, h->sm_count, false);
+  const int tn_gu = persist_tn_rounds(2 * F, M, h->sm_count, false);
+  const int tn_res = persist_tn_rounds(W, M, h->sm_count, true);
+  CUtensorMap am_hb, am_hb_gu, am_ob, am_ub;
   int rc;
-  if ((rc = make_tmap(&am_hb, h->hb, W, M, tn))) return rc;
+  if ((rc = make_tmap(&am_hb, h->hb, W, M, tn_qkv))) return rc;
+  if ((rc = make_tmap(&am_hb_gu, h->hb, W, M, tn_gu))) return rc;
   if ((rc = make_tmap(&am_ob, h->ob, h->HD, M, tn_res))) return rc;
   if ((rc = make_tmap(&am_ub, h->ub, F, M, tn_res))) return rc;
   // attention operands over this run's K / V (the caller's buffers, [L][B][P][D])
@@ -240,7 +243,7 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
       q.vtc = h->vtc + static_cast<size_t>(l) * B * D * h->kcap_t;
       q.kcap_t = h->kcap_t;
     }
-    if ((rc = prefill_gemm(h, s, EPI_QKV, h->tm_wqkv, am_hb, q, h->qkv_rows, W, M, tn, true))) return rc;
+    if ((rc = prefill_gemm(h, s, EPI_QKV, h->tm_wqkv, am_hb, q, h->qkv_rows, W, M, tn_qkv, true))) return rc;
     if (l == L - 1) break;   // the last layer's output side feeds no K/V
     if (tc) {
       AttnTcParams t{};
@@ -286,7 +289,7 @@ int vla_prefill_run(vla_prefill* h, const float* tokens, int n_tokens, int batch
     g.w_row0 = l * 2 * F;
     g.out = h->ub;
     g.ld_out = F;
-    if ((rc = prefill_gemm(h, s, EPI_GEGLU, h->tm_wgu, am_hb, g, 2 * F, W, M, tn, true))) return rc;
+    if ((rc = prefill_gemm(h, s, EPI_GEGLU, h->tm_wgu, am_hb_gu, g, 2 * F, W, M, tn_gu, true))) return rc;
     GemmParams d{};
     d.w_row0 = l * W;
     d.resid = h->resid;
