@@ -100,56 +100,95 @@ cudaError_t launch_norm(const NormParams& p, cudaStream_t s, bool pdl) {
 }
 
 // ------------------------------------------------------------------------ embed
-// One CTA per suffix row. State row: state_in(state); action rows: action_in(x), both
+// R suffix rows per CTA (R = 1 for few rows; 8 for many, so that each weight element read
+// from L2 serves eight rows). State row: state_in(state); action rows: action_in(x), both
 // fp32, with the maps stored transposed ([in][W]) so a warp reads 32 consecutive output
 // features per input element. Pi0 routes the action embedding (bf16) into the
-// action-time MLP instead of the residual.
+// action-time MLP instead of the residual. Every row's arithmetic (bias, then the inputs in
+// order; its sum of squares per thread, per warp, then over the warps in order) is the
+// same for any R.
+template <int R>
 __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
-  __shared__ float vin[256];
+  __shared__ float vin[R][256];
+  __shared__ float red[8][R];
   if (threadIdx.x == 0) pdl_trigger();
   pdl_wait();
-  const int m = blockIdx.x;
-  const int b = m / p.S, s = m - b * p.S;
-  const bool st = p.has_state && s == 0;
-  const int len = st ? p.Sd : p.A;
-  const float* src = st ? p.state + static_cast<size_t>(b) * p.Sd
-                        : p.x + (static_cast<size_t>(b) * p.C + (s - p.has_state)) * p.A;
-  const float* wt = st ? p.w_st : p.w_in;     // [len][W]
-  const float* bias = st ? p.b_st : p.b_in;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) vin[i] = src[i];
+  const int M = p.B * p.S;
+  const int m0 = blockIdx.x * R;
+  bool ok[R], st[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int m = m0 + r;
+    ok[r] = m < M;
+    const int b = m / p.S, s = m - b * p.S;
+    st[r] = ok[r] && p.has_state && s == 0;
+    if (!ok[r]) continue;
+    const int len = st[r] ? p.Sd : p.A;
+    const float* src = st[r] ? p.state + static_cast<size_t>(b) * p.Sd
+                             : p.x + (static_cast<size_t>(b) * p.C + (s - p.has_state)) * p.A;
+    for (int i = threadIdx.x; i < len; i += blockDim.x) vin[r][i] = src[i];
+  }
   __syncthreads();
-  float ss = 0.0f;
+  float ss[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) ss[r] = 0.0f;
   for (int n = threadIdx.x; n < p.W; n += blockDim.x) {
-    float acc = bias[n];
-#pragma unroll 8
-    for (int a = 0; a < len; ++a) acc = fmaf(wt[static_cast<size_t>(a) * p.W + n], vin[a], acc);
-    if (p.e_out && !st) {
-      p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(acc);
-    } else {
-      p.resid[static_cast<size_t>(m) * p.W + n] = acc;
-      ss += acc * acc;
-      if (p.zout) p.zout[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(acc * (1.0f + p.zmod[n]));
-      if (p.e_out) p.e_out[static_cast<size_t>(m) * p.W + n] = __float2bfloat16_rn(0.0f);
+    float acc[R];
+    const float bi = p.b_in[n];
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[r] = bi;
+    // action rows: one read of each weight element for all of them
+#pragma unroll 4
+    for (int a = 0; a < p.A; ++a) {
+      const float w = p.w_in[static_cast<size_t>(a) * p.W + n];
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if (ok[r] && !st[r]) acc[r] = fmaf(w, vin[r][a], acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!ok[r]) continue;
+      const size_t o = static_cast<size_t>(m0 + r) * p.W + n;
+      if (st[r]) {   // the state row (Pi0): its own map
+        float as = p.b_st[n];
+        for (int a = 0; a < p.Sd; ++a) as = fmaf(p.w_st[static_cast<size_t>(a) * p.W + n], vin[r][a], as);
+        acc[r] = as;
+      }
+      if (p.e_out && !st[r]) {
+        p.e_out[o] = __float2bfloat16_rn(acc[r]);
+      } else {
+        p.resid[o] = acc[r];
+        ss[r] += acc[r] * acc[r];
+        if (p.zout) p.zout[o] = __float2bfloat16_rn(acc[r] * (1.0f + p.zmod[n]));
+        if (p.e_out) p.e_out[o] = __float2bfloat16_rn(0.0f);
+      }
     }
   }
   if (p.rstat) {
-    // sum of squares of the residual row written here (0 for rows left to the time MLP)
-    __shared__ float red[8];
-    ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    // sum of squares of each residual row written here (0 for rows left to the time MLP)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float w = warp_sum(ss[r]);
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5][r] = w;
+    }
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < R && m0 + static_cast<int>(threadIdx.x) < M) {
       float t = 0.0f;
-      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
-      p.rstat[m] = t;
+      for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i][threadIdx.x];
+      p.rstat[m0 + threadIdx.x] = t;
     }
   }
 }
 
 cudaError_t launch_embed(const EmbedParams& p, cudaStream_t s, bool pdl) {
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = make_cfg(dim3(p.B * p.S), dim3(256), 0, s, attr, pdl);
-  return cudaLaunchKernelEx(&cfg, embed_kernel, p);
+  const int M = p.B * p.S;
+  if (M >= 1024) {
+    cudaLaunchConfig_t cfg = make_cfg(dim3((M + 7) / 8), dim3(256), 0, s, attr, pdl);
+    return cudaLaunchKernelEx(&cfg, embed_kernel<8>, p);
+  }
+  cudaLaunchConfig_t cfg = make_cfg(dim3(M), dim3(256), 0, s, attr, pdl);
+  return cudaLaunchKernelEx(&cfg, embed_kernel<1>, p);
 }
 
 // ------------------------------------------------------------------------ final
@@ -479,7 +518,8 @@ cudaError_t configure_small_kernels() {
   cudaError_t e = cudaSuccess;
   const void* fns[] = {reinterpret_cast<const void*>(norm_kernel<2>), reinterpret_cast<const void*>(norm_kernel<4>),
                        reinterpret_cast<const void*>(norm_kernel<8>), reinterpret_cast<const void*>(norm_kernel<16>),
-                       reinterpret_cast<const void*>(embed_kernel), reinterpret_cast<const void*>(final_kernel),
+                       reinterpret_cast<const void*>(embed_kernel<1>), reinterpret_cast<const void*>(embed_kernel<8>),
+                       reinterpret_cast<const void*>(final_kernel),
                        reinterpret_cast<const void*>(vt_dyn_kernel)};
   for (const void* fn : fns)
     if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
