@@ -1,5 +1,7 @@
 """The CUDA denoise path (through the C ABI) against the fp64 oracle on the same seeded
 inputs, element by element, for every workload shape; plus the exact special cases."""
+from dataclasses import replace
+
 import numpy as np
 import pytest
 
@@ -52,6 +54,29 @@ def test_batch64_every_observation_matches_batch1_runs():
                    prefix_v=inp["prefix_v"][:, b:b + 1])
         load_prefix(ex, one)
         check_actions(got[b:b + 1], run(ex, one, wl.steps), f"b64 row {b} vs batch-1 run")
+    ex.device_status()
+    ex.close()
+
+
+def test_pi0_many_rows_match_batch1_runs():
+    """A Pi0 expert (state token) at 21 observations, 1071 suffix rows: the embedding takes
+    eight rows per CTA there, state and action rows mixed in one CTA, and one row per CTA
+    in the batch-1 runs it is compared with, every row at the acceptance tolerance; the
+    oracle checks a sample."""
+    wl = replace(get("mid_pi0_b3"), name="mid_pi0_b21", batch=21)
+    assert wl.batch * wl.expert.suffix_len >= 1024
+    ex, inp = make_expert(wl)
+    load_prefix(ex, inp)
+    got = run(ex, inp, wl.steps)
+    ex.device_status()
+    assert got.shape[0] == wl.batch and np.all(np.isfinite(got))
+    idx = [0, 20]
+    check_actions(got[idx], oracle_actions(wl, inp, batch_idx=idx), "pi0 b21 oracle sample")
+    for b in range(wl.batch):
+        one = dict(inp, noise=inp["noise"][b:b + 1], state=inp["state"][b:b + 1],
+                   prefix_k=inp["prefix_k"][:, b:b + 1], prefix_v=inp["prefix_v"][:, b:b + 1])
+        load_prefix(ex, one)
+        check_actions(got[b:b + 1], run(ex, one, wl.steps), f"pi0 b21 row {b} vs batch-1 run")
     ex.device_status()
     ex.close()
 
