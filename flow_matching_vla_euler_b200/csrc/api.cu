@@ -47,6 +47,16 @@ int fail(int code, const char* fmt, ...) {
                   #expr, cudaGetErrorString(e_), __FILE__, __LINE__);                     \
   } while (0)
 
+// CU inside a create function once its handle exists: the half-built handle is released
+// (the function's `cleanup`) before the error returns
+#define CU_CLEANUP(expr)                                                                  \
+  do {                                                                                    \
+    cudaError_t e_ = (expr);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return cleanup(fail(e_ == cudaErrorMemoryAllocation ? VLA_ERR_OOM : VLA_ERR_CUDA, "%s: %s (%s:%d)", \
+                          #expr, cudaGetErrorString(e_), __FILE__, __LINE__));            \
+  } while (0)
+
 constexpr int kTableSlots = 4;
 constexpr int kMaxSteps = 64;
 
@@ -1107,9 +1117,9 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
       }
     if (h->fp8) {
       if ((rc = dalloc(h, &h->wqkv8, pk.size()))) return cleanup(rc);
-      CU(cudaMemcpy(h->wqkv8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
+      CU_CLEANUP(cudaMemcpy(h->wqkv8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
       if ((rc = dalloc(h, &h->sc_qkv, sc.size()))) return cleanup(rc);
-      CU(cudaMemcpy(h->sc_qkv, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
+      CU_CLEANUP(cudaMemcpy(h->sc_qkv, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
     } else if ((rc = upload_bf16(h, &h->wqkv, reinterpret_cast<const uint16_t*>(pk.data()), pk.size() / 2))) {
       return cleanup(rc);
     }
@@ -1132,9 +1142,9 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
       }
     if (h->fp8) {
       if ((rc = dalloc(h, &h->wgu8, pk.size()))) return cleanup(rc);
-      CU(cudaMemcpy(h->wgu8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
+      CU_CLEANUP(cudaMemcpy(h->wgu8, pk.data(), pk.size(), cudaMemcpyHostToDevice));
       if ((rc = dalloc(h, &h->sc_gu, sc.size()))) return cleanup(rc);
-      CU(cudaMemcpy(h->sc_gu, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
+      CU_CLEANUP(cudaMemcpy(h->sc_gu, sc.data(), sc.size() * 4, cudaMemcpyHostToDevice));
     } else if ((rc = upload_bf16(h, &h->wgu, reinterpret_cast<const uint16_t*>(pk.data()), pk.size() / 2))) {
       return cleanup(rc);
     }
@@ -1142,13 +1152,13 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   if (h->fp8) {
     const size_t no = static_cast<size_t>(L) * W * h->HD, nd = static_cast<size_t>(L) * W * F;
     if ((rc = dalloc(h, &h->wo8, no))) return cleanup(rc);
-    CU(cudaMemcpy(h->wo8, w->wo, no, cudaMemcpyHostToDevice));
+    CU_CLEANUP(cudaMemcpy(h->wo8, w->wo, no, cudaMemcpyHostToDevice));
     if ((rc = dalloc(h, &h->wdown8, nd))) return cleanup(rc);
-    CU(cudaMemcpy(h->wdown8, w->w_down, nd, cudaMemcpyHostToDevice));
+    CU_CLEANUP(cudaMemcpy(h->wdown8, w->w_down, nd, cudaMemcpyHostToDevice));
     if ((rc = dalloc(h, &h->sc_o, static_cast<size_t>(L) * W))) return cleanup(rc);
-    CU(cudaMemcpy(h->sc_o, w->wo_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
+    CU_CLEANUP(cudaMemcpy(h->sc_o, w->wo_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
     if ((rc = dalloc(h, &h->sc_down, static_cast<size_t>(L) * W))) return cleanup(rc);
-    CU(cudaMemcpy(h->sc_down, w->w_down_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
+    CU_CLEANUP(cudaMemcpy(h->sc_down, w->w_down_scale, static_cast<size_t>(L) * W * 4, cudaMemcpyHostToDevice));
   } else {
     if ((rc = upload_bf16(h, &h->wo, w->wo, static_cast<size_t>(L) * W * h->HD))) return cleanup(rc);
     if ((rc = upload_bf16(h, &h->wdown, w->w_down, static_cast<size_t>(L) * W * F))) return cleanup(rc);
@@ -1236,7 +1246,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   const bool want_persist = (cfg->flags & VLA_FLAG_PERSIST) != 0;
   if (h->persist_bmax >= 1 && want_persist) {
     int per_sm = 0;
-    CU(configure_denoise_persist(D, &per_sm, kPersistCluster, &max_clusters));
+    CU_CLEANUP(configure_denoise_persist(D, &per_sm, kPersistCluster, &max_clusters));
     h->persist_ok = per_sm >= 1;
   }
   if (h->persist_ok) {
@@ -1354,7 +1364,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
     // traffic, sets the pace)
     if (const char* e = getenv("VLA_ATTN_PAIR")) h->attn_pair = atoi(e) != 0;
     if (const char* e = getenv("VLA_VT_KERNEL")) h->vt_kernel = atoi(e) != 0;
-    CU(configure_attention_tc_kernel());
+    CU_CLEANUP(configure_attention_tc_kernel());
   }
   if (h->pi0) {
     if ((rc = make_tmap(&h->tm_w1a, h->w1a, W, W, 128))) return cleanup(rc);
@@ -1372,7 +1382,7 @@ int vla_expert_create(const vla_config* cfg, const vla_weights* w, vla_expert** 
   // The zero fills of dalloc run on the legacy stream, behind whatever the caller still has
   // in flight there; the handle's own stream does not wait for them, so they must have
   // finished before the tables below are computed on it.
-  CU(cudaDeviceSynchronize());
+  CU_CLEANUP(cudaDeviceSynchronize());
   cudaError_t e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cleanup(fail(VLA_ERR_CUDA, "stream create: %s", cudaGetErrorString(e)));
   int slot;

@@ -80,10 +80,12 @@ int vla_prefill_create(const vla_prefill_config* cfg, const vla_prefill_weights*
   CU(cudaGetDevice(&dev));
   CU(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
   if (major != 10) return fail(VLA_ERR_UNSUPPORTED, "device is sm_%d0; this library is built for sm_100a", major);
+  int sm_count = 0;
+  CU(cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev));
   vla_prefill* h = new vla_prefill();
   h->cfg = *cfg;
   h->dev = dev;
-  CU(cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, dev));
+  h->sm_count = sm_count;
   const int L = cfg->n_layers, W = cfg->width, H = cfg->n_heads, D = cfg->head_dim, F = cfg->mlp_dim;
   h->L = L; h->W = W; h->H = H; h->D = D; h->F = F; h->HD = H * D;
   h->qkv_rows = cdiv((H + 2) * D, 128) * 128;   // padding rows stay zero
@@ -141,18 +143,18 @@ int vla_prefill_create(const vla_prefill_config* cfg, const vla_prefill_weights*
   if ((rc = dalloc(h, &h->desc, 1))) return cleanup(rc);
   if ((rc = dalloc(h, &h->err, 1))) return cleanup(rc);
 
-  CU(configure_gemm_kernels());
-  CU(configure_small_kernels());
-  CU(configure_attention_kernels());
-  if (D == 256) CU(configure_attention_tc_kernel());
+  CU_CLEANUP(configure_gemm_kernels());
+  CU_CLEANUP(configure_small_kernels());
+  CU_CLEANUP(configure_attention_kernels());
+  if (D == 256) CU_CLEANUP(configure_attention_tc_kernel());
   if ((rc = make_tmap(&h->tm_wqkv, h->wqkv, W, static_cast<uint64_t>(L) * h->qkv_rows, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wo, h->wo, h->HD, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wgu, h->wgu, W, static_cast<uint64_t>(L) * 2 * F, 128))) return cleanup(rc);
   if ((rc = make_tmap(&h->tm_wdown, h->wdown, F, static_cast<uint64_t>(L) * W, 128))) return cleanup(rc);
   if ((rc = make_tmap_f32(&h->tm_resid, h->resid, W, Mx))) return cleanup(rc);
   // the rotary table at positions 0..max_tokens-1 and an empty cache descriptor, once
-  CU(launch_cache_update(h->desc, 0, 0, h->rope, cfg->max_tokens, D, cfg->rope_base, 0));
-  CU(cudaDeviceSynchronize());
+  CU_CLEANUP(launch_cache_update(h->desc, 0, 0, h->rope, cfg->max_tokens, D, cfg->rope_base, 0));
+  CU_CLEANUP(cudaDeviceSynchronize());
   *out = h;
   return VLA_OK;
 }
