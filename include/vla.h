@@ -73,11 +73,10 @@ typedef enum vla_time_kind {
 
 /* Option bits for vla_config.flags. */
 #define VLA_FLAG_NO_PDL 1u      /* launch without programmatic dependent launch edges */
-#define VLA_FLAG_NORM_KERNELS 2u /* with one token tile (batch x suffix <= 64), run the
-                                    pre-attention / pre-MLP norms as kernels of their own
-                                    instead of folding them into the projections (cross-check;
-                                    larger batches always use norm kernels; implies
-                                    VLA_FLAG_NO_PERSIST) */
+#define VLA_FLAG_NORM_KERNELS 2u /* run the pre-attention / pre-MLP norms as kernels of
+                                    their own instead of folding them into the projections
+                                    (a cross-check of the folded norms, at any batch; not
+                                    combinable with VLA_FLAG_PERSIST) */
 #define VLA_FLAG_NO_PERSIST 4u   /* never run the single persistent kernel: the denoise is
                                     one kernel launch per projection / attention / embed /
                                     final step, captured in a graph (the default) */
