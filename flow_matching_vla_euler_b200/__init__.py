@@ -247,6 +247,9 @@ def vla_gemm_bf16_noalloc(W_ptr, X_ptr, Y_ptr, n_feat, k_dim, m_tok, split_k, st
 def gemm(W, X, split_k: int = 0):
     """Y = X @ W^T on the tensor-core kernel; W [n, k], X [m, k] CUDA bf16 -> fp32 [m, n]."""
     import torch
+    if W.dim() != 2 or X.dim() != 2:
+        raise ValueError("W and X must be 2-D")
+    _expect(X, (X.shape[0], W.shape[1]), "X")
     Y = torch.empty((X.shape[0], W.shape[0]), dtype=torch.float32, device=X.device)
     vla_gemm_bf16(_dev_ptr(W, 2), _dev_ptr(X, 2), _dev_ptr(Y, 4), int(W.shape[0]), int(W.shape[1]),
                   int(X.shape[0]), int(split_k), _stream())
@@ -266,6 +269,46 @@ def vla_version() -> str:
 def _stream():
     import torch
     return torch.cuda.current_stream().cuda_stream
+
+
+def _expect(t, shape, name, dtype=None):
+    """The shape (and, for fp32 operands, the dtype) a raw-pointer argument must have: the
+    library reads or writes exactly that many elements behind the pointer, so a mismatch is
+    refused here, before any call."""
+    got = tuple(int(d) for d in t.shape)
+    if got != tuple(int(d) for d in shape):
+        raise ValueError(f"{name}: shape {got}, expected {tuple(int(d) for d in shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
+def _check_denoise_args(cfg, noise, state, out, batch=None):
+    """noise [batch, chunk, action_dim] fp32, state [batch, state_dim] fp32 (when the expert
+    has a state token), out like noise."""
+    if len(noise.shape) != 3:
+        raise ValueError("noise: expected [batch, chunk, action_dim]")
+    b = int(noise.shape[0]) if batch is None else int(batch)
+    f32 = _f32_of(noise)
+    _expect(noise, (b, cfg.chunk, cfg.action_dim), "noise", f32)
+    if state is not None and cfg.state_dim > 0:   # a missing state is the library's to refuse
+        _expect(state, (b, cfg.state_dim), "state", f32)
+    if out is not None:
+        _expect(out, (b, cfg.chunk, cfg.action_dim), "out", f32)
+
+
+def _check_token_kv(cfg, K_tok, V_tok, batch):
+    shape = (cfg.n_layers, int(batch), cfg.n_kv_heads * cfg.head_dim)
+    _expect(K_tok, shape, "K_tok")
+    _expect(V_tok, shape, "V_tok")
+
+
+def _f32_of(t):
+    """float32 in the array library of t (torch or numpy)."""
+    import numpy as np
+    if isinstance(t, np.ndarray):
+        return np.dtype(np.float32)
+    import torch
+    return torch.float32
 
 
 def _dev_ptr(t, dtype_bytes):
@@ -317,8 +360,14 @@ class Prefill:
         """tokens: CUDA fp32 [batch, n_tokens, width] -> K, V: CUDA int16 tensors (bf16 bits)
         [L, batch, n_tokens, head_dim], allocated when not given."""
         import torch
+        if tokens.dim() != 3:
+            raise ValueError("tokens: expected [batch, n_tokens, width]")
         batch, n = int(tokens.shape[0]), int(tokens.shape[1])
+        _expect(tokens, (batch, n, self.cfg.width), "tokens", torch.float32)
         shape = (self.cfg.n_layers, batch, n, self.cfg.head_dim)
+        for t, nm in ((K_out, "K_out"), (V_out, "V_out")):
+            if t is not None:
+                _expect(t, shape, nm)
         if K_out is None:
             K_out = torch.empty(shape, dtype=torch.int16, device=tokens.device)
         if V_out is None:
@@ -343,11 +392,21 @@ class Pipeline:
         next step), ready once ``stream`` (a torch.cuda.Stream; default the current one)
         reaches this point. Submitting from a stream other than the one the steps run on
         lets the prefill overlap the step already enqueued there."""
+        import torch
+        if tokens.dim() != 3:
+            raise ValueError("tokens: expected [batch, n_tokens, width]")
+        _expect(tokens, (self.batch, tokens.shape[1], self.prefill.cfg.width), "tokens", torch.float32)
+        ptr = _dev_ptr(tokens, 4)
         sp = _stream() if stream is None else stream.cuda_stream
-        vla_pipeline_submit(self.handle, _dev_ptr(tokens, 4), int(tokens.shape[1]), sp)
+        vla_pipeline_submit(self.handle, ptr, int(tokens.shape[1]), sp)
 
     def step(self, noise, state=None, steps: int = 10, out=None, K_tok=None, V_tok=None):
         import torch
+        _check_denoise_args(self.expert.cfg, noise, state, out, self.batch)
+        if (K_tok is None) != (V_tok is None):
+            raise ValueError("K_tok and V_tok go together")
+        if K_tok is not None:
+            _check_token_kv(self.expert.cfg, K_tok, V_tok, self.batch)
         if out is None:
             out = torch.empty_like(noise)
         kp = 0 if K_tok is None else _dev_ptr(K_tok, 2)
@@ -420,17 +479,26 @@ class Expert:
 
     def set_prefix(self, K, V):
         """K, V: CUDA tensors (2-byte elements, bf16 bits) [L, batch, n_tokens, D]."""
+        if K.dim() != 4:
+            raise ValueError("K: expected [L, batch, n_tokens, D]")
         batch, n = int(K.shape[1]), int(K.shape[2])
+        shape = (self.cfg.n_layers, batch, n, self.cfg.n_kv_heads * self.cfg.head_dim)
+        _expect(K, shape, "K")
+        _expect(V, shape, "V")
         vla_cache_set_prefix(self.handle, _dev_ptr(K, 2), _dev_ptr(V, 2), n, batch, _stream())
 
     def append_sliding(self, K_tok, V_tok):
         """K_tok, V_tok: CUDA tensors [L, batch, D] of bf16 bits."""
+        if K_tok.dim() != 3:
+            raise ValueError("K_tok: expected [L, batch, D]")
+        _check_token_kv(self.cfg, K_tok, V_tok, int(K_tok.shape[1]))
         vla_cache_append_sliding(self.handle, _dev_ptr(K_tok, 2), _dev_ptr(V_tok, 2),
                                  int(K_tok.shape[1]), _stream())
 
     def denoise(self, noise, state=None, steps: int = 10, out=None):
         """noise: CUDA fp32 [batch, C, A]; state: CUDA fp32 [batch, state_dim] or None."""
         import torch
+        _check_denoise_args(self.cfg, noise, state, out)
         out = torch.empty_like(noise) if out is None else out
         sp = _dev_ptr(state, 4) if state is not None else None
         vla_denoise(self.handle, _dev_ptr(noise, 4), sp, int(steps), _dev_ptr(out, 4),
@@ -441,8 +509,9 @@ class Expert:
         """Host (numpy fp32) buffers in and out; synchronous."""
         import numpy as np
         noise = np.ascontiguousarray(noise, dtype=np.float32)
-        out = np.empty_like(noise)
         st = None if state is None else np.ascontiguousarray(state, dtype=np.float32)
+        _check_denoise_args(self.cfg, noise, st, None)
+        out = np.empty_like(noise)
         vla_denoise_host(self.handle, noise.ctypes.data, None if st is None else st.ctypes.data,
                          int(steps), out.ctypes.data, int(noise.shape[0]), _stream())
         return out
@@ -461,6 +530,7 @@ class Expert:
 
     def profile_kernels(self, noise, state=None, steps: int = 10):
         import torch
+        _check_denoise_args(self.cfg, noise, state, None)
         out = torch.empty_like(noise)
         sp = _dev_ptr(state, 4) if state is not None else None
         t = vla_profile_kernels(self.handle, _dev_ptr(noise, 4), sp, int(steps), _dev_ptr(out, 4),
